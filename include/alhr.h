@@ -1,0 +1,190 @@
+/*
+ * alhr.h -- C ABI of the B200 (sm_100a) inference path of ALHR tree attention.
+ *
+ * Source of the method: the project README "ALHR (Adaptive learnable Hierarchical
+ * routing): sub-quadratic tree attention without meaningful accuracy loss, trained in
+ * three phases against a dense reference" (GitHub project
+ * Adaptive-Learnable-Hierarchical-Routing-), cited below as [README §<section>], and the
+ * openai-hub analysis "ALHR把注意力变成树搜索", cited as [openai-hub §<section>].
+ *
+ * Problem statement fixed for this library (the README leaves the numeric formats open):
+ *   - per (batch b, head h) there are n keys, n a power of two, head dimension d in {64,128};
+ *   - Q and K are int8 with |value| <= value_bound (16 unless stated), so every tree sum and
+ *     every routing score is an exact integer;
+ *   - V is bf16 (passed as raw uint16 bit patterns); outputs are fp32;
+ *   - budgets come from 32 classes, class c meaning 3*(c+1) keys, at most 96 keys
+ *     [README §Results and Variables: "Max keys = 96 and Max Budget class = 32"];
+ *   - the neighbour window is w keys (16 in the README's setting).
+ *
+ * Memory layouts (all row-major, contiguous, device memory, 16-byte aligned base pointers):
+ *   Q      int8     [batch][heads][nq][d]        row t is the query at position q_start+t
+ *   K      int8     [batch][heads][n][d]
+ *   V      uint16   [batch][heads][n][d]         bf16 bit patterns
+ *   nodes  int32    [batch][heads][n-1][d]       level-major tree (see alhr_tree_level_offset)
+ *   W      int8     [32][2d]                     budget-predictor weights, shared by all heads
+ *   budget int32    [batch][heads][nq]           keys asked for by each query (>= 1)
+ *   idx    int32    [batch][heads][nq][max_keys] selected key positions, ascending, -1 padded
+ *   count  int32    [batch][heads][nq]           number of valid entries of idx
+ *   expansions int32 [batch][heads][nq][2]       {nodes of level >= 2 expanded, level-1 nodes expanded}
+ *   out    float    [batch][heads][nq][d]
+ *
+ * Ownership: every pointer belongs to the caller. The library allocates no device memory and
+ * keeps no state between calls; a call only reads its inputs and writes its outputs.
+ *
+ * Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). All
+ * compute entry points are asynchronous with respect to the host.
+ *
+ * Errors: arguments are checked on the host before anything is launched; on any non-OK
+ * status nothing has been launched and no output has been written. A launch failure returns
+ * ALHR_ERR_CUDA. Data errors that only the device can see (a budget below 1, a Q or K value
+ * outside [-value_bound, value_bound]) never trap: the offending value is clamped (budgets)
+ * or used as is (values), and the matching ALHR_DEVERR_* bit is OR-ed into *dev_err when
+ * dev_err is non-NULL. Kernels contain no unbounded loop and no spin-wait.
+ */
+#ifndef ALHR_H
+#define ALHR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ALHR_OK = 0,
+  ALHR_ERR_INVALID_ARG = 1,  /* a NULL required pointer, a misaligned pointer, a bad size   */
+  ALHR_ERR_UNSUPPORTED = 2,  /* sizes the kernels do not handle (d, window, max_keys, n)    */
+  ALHR_ERR_OVERFLOW = 3,     /* score_bits = 32 requested where int32 scores could overflow */
+  ALHR_ERR_CUDA = 4          /* a CUDA launch or runtime call failed                        */
+} alhr_status;
+
+/* Bits OR-ed into the optional device word *dev_err. */
+#define ALHR_DEVERR_BUDGET_LOW  0x1u /* a budget < 1 was read; it was treated as 1          */
+#define ALHR_DEVERR_VALUE_RANGE 0x2u /* a Q or K value had |value| > value_bound            */
+
+/* Problem sizes, shared by every entry point. */
+typedef struct {
+  int32_t batch;       /* >= 1                                                            */
+  int32_t heads;       /* >= 1                                                            */
+  int32_t n;           /* keys per (b,h): a power of two, 2 <= n <= 2^20                  */
+  int32_t d;           /* head dimension: 64 or 128                                       */
+  int32_t q_start;     /* first query position; prefill 0, decode n-1                     */
+  int32_t nq;          /* queries per (b,h); 0 <= nq, q_start + nq <= n                   */
+  int32_t window;      /* neighbour window w, 1 <= w <= 32                                */
+  int32_t max_keys;    /* cap on keys per query, 1 <= max_keys <= 96                      */
+  int32_t score_bits;  /* 0 = choose, 32 = int32 scores (checked), 64 = int64 scores      */
+  int32_t value_bound; /* bound on |Q|, |K|; 0 means 16; at most 127                      */
+} alhr_dims;
+
+/* Number of tree rows per (b,h): n - 1. Returns 0 when n is not a power of two in [2, 2^20]. */
+size_t alhr_tree_rows(int32_t n);
+
+/* Row offset of tree level `level` (1 <= level <= log2 n) inside one (b,h) block of `nodes`:
+ * level l holds n >> l rows starting at row n - (n >> (l-1)); row j of level l is the sum of
+ * keys [j*2^l, (j+1)*2^l). Level 0 (the keys themselves) is K and is not stored.
+ * Returns (size_t)-1 for an invalid pair. */
+size_t alhr_tree_level_offset(int32_t n, int32_t level);
+
+/* Score width the kernels will use for these sizes (32 or 64), or a negative alhr_status
+ * (-ALHR_ERR_...) when the sizes are invalid or score_bits = 32 cannot be exact. */
+int32_t alhr_score_bits(const alhr_dims* dims);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* alhr_status_string(int32_t status);
+
+/* Build identification (static storage): target architecture and library version. */
+const char* alhr_build_info(void);
+
+/*
+ * alhr_build_tree -- the static key tree [README §Inference stage, first paragraph: the tree
+ * is built on the key matrix and stored, once per layer; README opening paragraph: every
+ * branch is indexed by the sum of all key vectors beneath it].
+ *
+ * For every (b,h) writes nodes(l, j) = sum_{t in [j*2^l, (j+1)*2^l)} K[t] for l = 1..log2 n,
+ * exact in int32, level-major as described at alhr_tree_level_offset. Only dims->batch,
+ * heads, n, d and value_bound are read.
+ *   K       device, int8 [batch][heads][n][d], read only
+ *   nodes   device, int32 [batch][heads][n-1][d], fully overwritten
+ *   dev_err device uint32 or NULL; ALHR_DEVERR_VALUE_RANGE if some |K| > value_bound
+ */
+alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, int32_t* nodes,
+                            uint32_t* dev_err, void* stream);
+
+/*
+ * alhr_predict_budget -- the budget predictor [README §Inference stage, second paragraph: a
+ * trainable function of the current query and the global key sum that outputs a leaf group,
+ * i.e. the number of keys the query asks for; §Results and Variables: 32 classes, <= 96 keys].
+ *
+ * For the query at position i: G_i = sum_{t <= i} K[t] (the causal reading of "global sum"),
+ * logit_c = sum_t W[c][t] q_t + sum_t W[c][d+t] G_i[t] for c = 0..31 in int64,
+ * c* = the smallest c with the largest logit, budget = 3*(c*+1).
+ * G_i is formed from the tree: the roots of the past-only forest of [0, i-w] plus the window
+ * keys (i-w, i].
+ *   Q, K, nodes  device inputs (layouts above); W device int8 [32][2d]
+ *   budget       device int32 [batch][heads][nq], overwritten
+ *   dev_err      as above (ALHR_DEVERR_VALUE_RANGE for |q| > value_bound)
+ */
+alhr_status alhr_predict_budget(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
+                                const int32_t* nodes, const int8_t* W, int32_t* budget,
+                                uint32_t* dev_err, void* stream);
+
+/*
+ * alhr_route -- neighbour search plus budget-limited tree descent [README §Inference stage,
+ * third and fourth paragraphs; §Training stage, last paragraph: causality by descending only
+ * the subtrees that hold past keys].
+ *
+ * For the query at position i with budget B (read from `budget`):
+ *   B_eff = min(max(B,1), i+1, max_keys);
+ *   window: keys i, i-1, ..., max(0, i-w+1), nearest first, cut to B_eff;
+ *   r = B_eff - |window|; if r > 0 and i >= w, descend the forest of aligned power-of-two
+ *   roots of [0, i-w] (the maximal past-only subtrees, largest first): repeatedly replace every
+ *   non-leaf frontier node by its two children and keep the r nodes with the largest exact
+ *   integer q . node_sum (ties: lower start position), until every frontier node is a key.
+ *   The routed keys are the final frontier; the selection is window + routed.
+ *   idx        device int32 [..][max_keys]: selection ascending, -1 padded (required)
+ *   count      device int32: |selection| = min(B_eff, i+1) (required)
+ *   expansions device int32 [..][2] or NULL: {level >= 2 nodes expanded, level-1 nodes expanded}
+ *   dev_err    as above (ALHR_DEVERR_BUDGET_LOW, ALHR_DEVERR_VALUE_RANGE)
+ */
+alhr_status alhr_route(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
+                       const int32_t* nodes, const int32_t* budget, int32_t* idx, int32_t* count,
+                       int32_t* expansions, uint32_t* dev_err, void* stream);
+
+/*
+ * alhr_attend -- exact attention over the selected keys [README §Inference stage, fifth
+ * paragraph: once each query has its keys, standard dot-product attention and sum run].
+ *
+ * out_i = sum_j softmax_j(s) V[j] over j in idx[0..count), s_j = (q_i . K[j]) / sqrt(d), with the
+ * integer dot product exact and the softmax and sum in fp32. A query with count <= 0 gets a
+ * zero row. Entries of idx outside [0, i] are not read (they are skipped).
+ *   Q, K, V, idx, count  device inputs (layouts above)
+ *   out                  device float [batch][heads][nq][d], overwritten
+ */
+alhr_status alhr_attend(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
+                        const uint16_t* V, const int32_t* idx, const int32_t* count, float* out,
+                        uint32_t* dev_err, void* stream);
+
+/*
+ * alhr_forward -- the whole inference path in one kernel per query: causal key sum, budget
+ * predictor (or budget_override), window, descent and exact attention [README §Inference
+ * stage, all five paragraphs]. The tree must have been built by alhr_build_tree.
+ *   W                device int8 [32][2d]; may be NULL only when budget_override is given
+ *   budget_override  device int32 [batch][heads][nq] or NULL (NULL = use the predictor)
+ *   out              device float [batch][heads][nq][d] (required)
+ *   idx, count, expansions, budget_out  optional outputs (NULL = not written); budget_out
+ *                    receives the budget each query used (predicted or overridden, after the
+ *                    clamp to >= 1)
+ * Results equal alhr_predict_budget + alhr_route + alhr_attend on the same inputs.
+ */
+alhr_status alhr_forward(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
+                         const uint16_t* V, const int32_t* nodes, const int8_t* W,
+                         const int32_t* budget_override, float* out, int32_t* idx,
+                         int32_t* count, int32_t* expansions, int32_t* budget_out,
+                         uint32_t* dev_err, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ALHR_H */

@@ -1,0 +1,112 @@
+"""Planted mistakes: each test compiles a copy of the oracle with one plausible slip and checks
+that the pins in test_oracle_pins.py reject it. The mistakes are planted in the oracle, on the
+CPU; nothing here touches a GPU."""
+import json
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+from oracle import oracle as orc
+import test_oracle_pins as pins
+
+_SRC = os.path.join(os.path.dirname(orc.__file__), "alhr_oracle.cpp")
+
+MUTATIONS = {
+    "tie_to_higher_start": ("return a.start < b.start;", "return a.start > b.start;"),
+    "keep_lowest_scores": ("if (a.score != b.score) return a.score > b.score;",
+                           "if (a.score != b.score) return a.score < b.score;"),
+    "window_one_too_wide": ("t > int64_t(i) - w &&", "t >= int64_t(i) - w &&"),
+    "forest_covers_window_key": ("const int64_t m = int64_t(i) - w + 1;",
+                                 "const int64_t m = int64_t(i) - w + 2;"),
+    "forest_misses_a_key": ("const int64_t m = int64_t(i) - w + 1;",
+                            "const int64_t m = int64_t(i) - w;"),
+    "right_child_offset": ("right = nd.start + (int64_t(1) << cl);",
+                           "right = nd.start + (int64_t(1) << nd.level);"),
+    "level_offset_shifted": ("return n - (n >> (level - 1));", "return n - (n >> level);"),
+    "exclusive_causal_sum": ("for (int u = 0; u <= i; ++u)", "for (int u = 0; u < i; ++u)"),
+    "predictor_tie_to_higher_class": ("if (c == 0 || s > best_logit)",
+                                      "if (c == 0 || s >= best_logit)"),
+    "predictor_operands_swapped": ("s += int64_t(w[d + t]) * G[t];",
+                                   "s += int64_t(w[t]) * G[t];"),
+    "expansion_levels_misfiled": ("if (nd.level >= 2) ++exp_hi; else ++exp_l1;",
+                                  "if (nd.level >= 1) ++exp_hi; else ++exp_l1;"),
+    "no_score_scale": ("s[size_t(k)] = double(dot) * scale;",
+                       "s[size_t(k)] = double(dot);"),
+    "softmax_without_max_shift_sign": ("std::exp(s[size_t(k)] - mx)",
+                                       "std::exp(mx - s[size_t(k)])"),
+    "budget_not_clamped": ("budget = std::max(budget_override[row], 1);",
+                           "budget = budget_override[row];"),
+    "prune_keeps_one_less": ("cand.resize(size_t(r));", "cand.resize(size_t(r - 1));"),
+}
+
+PIN_TESTS = [
+    ("golden_tree", lambda g: pins.test_golden_tree(g)),
+    ("golden_causal", lambda g: pins.test_golden_causal_sums(g)),
+    ("golden_routes", lambda g: pins.test_golden_routes(g)),
+    ("golden_predictor", lambda g: pins.test_golden_predictor(g)),
+    ("golden_forward", lambda g: pins.test_golden_forward_composition(g)),
+    ("root_children", lambda g: pins.test_tree_root_and_children(64, 64)),
+    ("telescoping", lambda g: pins.test_causal_sum_telescopes_and_ends_at_root()),
+    ("numpy_argmax", lambda g: pins.test_predictor_against_numpy_argmax()),
+    ("ties_lowest_class", lambda g: pins.test_predictor_ties_go_to_lowest_class()),
+    ("wide_beam", lambda g: pins.test_wide_beam_routes_the_whole_past(256, 5)),
+    ("planted", lambda g: pins.test_planted_positive_key_is_routed(512, 16)),
+    ("dense", lambda g: pins.test_full_budget_is_dense_causal_attention(64, 8, 4)),
+    ("attention_closed_forms", lambda g: pins.test_attention_closed_forms()),
+    ("clamp", lambda g: pins.test_forward_budget_override_clamp_and_predictor()),
+]
+
+
+def _compile_mutant(name, tmpdir):
+    old, new = MUTATIONS[name]
+    with open(_SRC) as f:
+        src = f.read()
+    assert src.count(old) == 1, f"mutation anchor for {name} must occur exactly once"
+    path = os.path.join(tmpdir, f"{name}.cpp")
+    with open(path, "w") as f:
+        f.write(src.replace(old, new))
+    so = os.path.join(tmpdir, f"lib{name}.so")
+    subprocess.run(["g++", "-O1", "-std=c++17", "-shared", "-fPIC", "-o", so, path], check=True)
+    return so
+
+
+def run_pins_against(so_path: str) -> list:
+    """Names of the pins that reject the oracle build at so_path."""
+    import json as _json
+    from conftest import ROOT
+    with open(os.path.join(ROOT, "tests", "golden", "alhr_n8_d2.json")) as f:
+        golden = _json.load(f)
+    caught = []
+    with orc.use_library(so_path):
+        for pin, fn in PIN_TESTS:
+            try:
+                fn(golden)
+            except (AssertionError, OverflowError):
+                caught.append(pin)
+    return caught
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name):
+    # each mutant runs in a child process: a slip that writes out of bounds may crash it,
+    # which also counts as caught
+    here = os.path.dirname(os.path.abspath(__file__))
+    with tempfile.TemporaryDirectory() as tmp:
+        so = _compile_mutant(name, tmp)
+        code = ("import sys, json; sys.path[:0] = [%r, %r]; "
+                "import test_oracle_mutations as m; print(json.dumps(m.run_pins_against(%r)))"
+                % (here, os.path.dirname(here), so))
+        proc = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                              timeout=600)
+        if proc.returncode != 0:
+            return  # the mutant crashed the pins: caught
+        caught = json.loads(proc.stdout.strip().splitlines()[-1])
+        assert caught, f"no pin rejects the planted mistake {name}"
+
+
+def test_unmutated_oracle_passes_every_pin(golden_n8):
+    for _, fn in PIN_TESTS:
+        fn(golden_n8)

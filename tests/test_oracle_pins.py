@@ -1,0 +1,378 @@
+"""Pins of the oracle to facts that do not come from the oracle itself.
+
+Sources of truth used here:
+  * the hand-worked N=8, d=2 example in tests/golden/alhr_n8_d2.json (derived by hand from
+    the ALHR README, sections "Inference stage" and "Training stage");
+  * closed forms: the root is the sum of all keys; the causal sum telescopes; a planted key
+    is always routed; with a beam at least as wide as the past, every past key is routed and
+    every internal node of the forest is expanded exactly once;
+  * a dense causal softmax attention written independently with numpy (the Monodratic-style
+    check of a sparse selected-set attention against a dense masked one);
+  * an independent range-based formulation of the descent (recursive halving of [lo, hi)
+    intervals, node sums taken straight from K, a full Python sort) on small random inputs.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import oracle as orc
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _rand_qk(rng, shape, lo=-16, hi=16):
+    return rng.integers(lo, hi + 1, size=shape).astype(np.int8)
+
+
+def _rand_v_bits(rng, shape):
+    v = rng.standard_normal(shape).astype(np.float32)
+    bits = v.view(np.uint32)
+    # round to nearest even bf16
+    bits = ((bits + 0x7FFF + ((bits >> 16) & 1)) >> 16).astype(np.uint16)
+    return bits
+
+
+def _bits_to_f64(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------- hand-worked example
+
+def test_golden_tree(golden_n8):
+    K = np.array(golden_n8["K"], dtype=np.int8)
+    nodes = orc.build_tree(K)
+    assert nodes.tolist() == golden_n8["tree_level_major"]
+
+
+def test_golden_causal_sums(golden_n8):
+    K = np.array(golden_n8["K"], dtype=np.int8)
+    for case in golden_n8["causal_sums"]:
+        assert orc.causal_sum(K, case["i"]).tolist() == case["G"], case["why"]
+
+
+def test_golden_routes(golden_n8):
+    K = np.array(golden_n8["K"], dtype=np.int8)
+    nodes = orc.build_tree(K)
+    for case in golden_n8["routes"]:
+        sel, exp = orc.route(K, nodes, np.array(case["q"], dtype=np.int8), case["i"],
+                             case["budget"], golden_n8["window"], golden_n8["max_keys"])
+        assert sel.tolist() == case["selected"], case["why"]
+        assert list(exp) == case["expansions"], case["why"]
+
+
+def test_golden_predictor(golden_n8):
+    for case in golden_n8["predictor"]:
+        W = np.zeros((32, 4), dtype=np.int8)
+        for row, vals in case.get("W_rows", {}).items():
+            W[int(row)] = vals
+        c, _ = orc.predict(np.array(case["q"], dtype=np.int8),
+                           np.array(case["G"], dtype=np.int64), W)
+        assert c == case["class"], case["why"]
+        assert 3 * (c + 1) == case["budget"]
+
+
+def test_golden_forward_composition(golden_n8):
+    """The slice entry point reproduces the hand-worked routes when given their budgets."""
+    K = np.array(golden_n8["K"], dtype=np.int8)
+    nodes = orc.build_tree(K)
+    rng = _rng(1)
+    V = _rand_v_bits(rng, (8, 2))
+    cases = [c for c in golden_n8["routes"] if c["i"] == 7]
+    for case in cases:
+        Q = np.array([case["q"]], dtype=np.int8)
+        res = orc.forward(Q, K, V, nodes, None, np.array([case["budget"]], dtype=np.int32),
+                          q_start=7, window=2, max_keys=96)
+        c = res["count"][0]
+        assert res["idx"][0, :c].tolist() == case["selected"]
+        assert (res["idx"][0, c:] == -1).all()
+        assert res["expansions"][0].tolist() == case["expansions"]
+
+
+# ---------------------------------------------------------------- tree closed forms
+
+@pytest.mark.parametrize("n,d", [(2, 2), (8, 3), (64, 64), (1024, 64), (256, 128)])
+def test_tree_root_and_children(n, d):
+    rng = _rng(n + d)
+    K = _rand_qk(rng, (n, d))
+    nodes = orc.build_tree(K)
+    L = int(math.log2(n))
+    off = lambda l: n - (n >> (l - 1))
+    # the root is the sum of every key
+    assert (nodes[off(L)] == K.astype(np.int64).sum(0)).all()
+    # level 1 holds key pairs, every higher node the sum of its two children
+    lvl1 = nodes[off(1): off(1) + n // 2].astype(np.int64)
+    assert (lvl1 == K[0::2].astype(np.int64) + K[1::2]).all()
+    for l in range(2, L + 1):
+        par = nodes[off(l): off(l) + (n >> l)].astype(np.int64)
+        ch = nodes[off(l - 1): off(l - 1) + (n >> (l - 1))].astype(np.int64)
+        assert (par == ch[0::2] + ch[1::2]).all()
+
+
+def test_tree_planted_key_marks_its_ancestors():
+    n, d = 256, 4
+    for p in [0, 1, 77, 255]:
+        K = np.zeros((n, d), dtype=np.int8)
+        K[p] = [16, -16, 3, 0]
+        nodes = orc.build_tree(K)
+        for l in range(1, 9):
+            off = n - (n >> (l - 1))
+            for j in range(n >> l):
+                expect = K[p] if j == (p >> l) else np.zeros(d, dtype=np.int8)
+                assert (nodes[off + j] == expect).all()
+
+
+def test_tree_extreme_values_exact():
+    n, d = 4096, 64
+    K = np.full((n, d), -16, dtype=np.int8)
+    K[::3] = 16
+    nodes = orc.build_tree(K)
+    assert nodes[-1, 0] == int(K[:, 0].astype(np.int64).sum())
+
+
+# ---------------------------------------------------------------- causal sum and predictor
+
+def test_causal_sum_telescopes_and_ends_at_root():
+    rng = _rng(5)
+    n, d = 128, 16
+    K = _rand_qk(rng, (n, d))
+    nodes = orc.build_tree(K)
+    prev = np.zeros(d, dtype=np.int64)
+    for i in range(n):
+        G = orc.causal_sum(K, i)
+        assert (G - prev == K[i]).all()
+        prev = G
+    assert (prev == nodes[-1]).all()
+
+
+def test_predictor_against_numpy_argmax():
+    rng = _rng(7)
+    for d in [2, 64, 128]:
+        for _ in range(30):
+            q = _rand_qk(rng, (d,))
+            G = rng.integers(-16 * 5000, 16 * 5000, size=d).astype(np.int64)
+            W = rng.integers(-4, 5, size=(32, 2 * d)).astype(np.int8)
+            c, logits = orc.predict(q, G, W)
+            x = np.concatenate([q.astype(np.int64), G])
+            ref = W.astype(np.int64) @ x
+            assert (logits == ref).all()
+            assert c == int(np.argmax(ref))  # numpy argmax returns the first maximum
+
+
+def test_predictor_ties_go_to_lowest_class():
+    d = 8
+    q = np.ones(d, dtype=np.int8)
+    G = np.ones(d, dtype=np.int64)
+    W = np.zeros((32, 2 * d), dtype=np.int8)
+    assert orc.predict(q, G, W)[0] == 0
+    W[[5, 9, 30]] = 1
+    assert orc.predict(q, G, W)[0] == 5
+
+
+# ---------------------------------------------------------------- route closed forms
+
+def _forest_internal_counts(m):
+    """(level>=2 internal nodes, level-1 internal nodes) of the forest of [0, m)."""
+    hi = l1 = 0
+    for b in range(64):
+        if (m >> b) & 1 and b >= 1:
+            l1 += 1 << (b - 1)
+            hi += (1 << (b - 1)) - 1
+    return hi, l1
+
+
+@pytest.mark.parametrize("n,w", [(64, 16), (128, 1), (256, 5), (1024, 16)])
+def test_wide_beam_routes_the_whole_past(n, w):
+    rng = _rng(n * 31 + w)
+    d = 8
+    K = _rand_qk(rng, (n, d))
+    nodes = orc.build_tree(K)
+    for i in rng.choice(n, size=12, replace=False):
+        i = int(i)
+        q = _rand_qk(rng, (d,))
+        sel, exp = orc.route(K, nodes, q, i, budget=n + 5, window=w, max_keys=n + 5)
+        assert sel.tolist() == list(range(i + 1))
+        m = i - w + 1
+        assert exp == (_forest_internal_counts(m) if m > 0 else (0, 0))
+
+
+@pytest.mark.parametrize("n,w", [(64, 4), (512, 16), (1024, 2)])
+def test_planted_positive_key_is_routed(n, w):
+    """K is zero except key p with q . k_p > 0: every node holding p scores above every other
+    node (which all score 0), so p survives each pruning; the remaining r-1 places go to the
+    lowest positions by the tie rule."""
+    rng = _rng(n + w)
+    d = 4
+    q = np.array([1, 2, -1, 3], dtype=np.int8)
+    for _ in range(25):
+        i = int(rng.integers(w + 1, n))
+        m = i - w + 1
+        p = int(rng.integers(0, m))
+        K = np.zeros((n, d), dtype=np.int8)
+        K[p] = [5, 5, 1, 2]
+        nodes = orc.build_tree(K)
+        B = int(rng.integers(w + 1, w + 40))
+        sel, _ = orc.route(K, nodes, q, i, B, w, max_keys=96)
+        b_eff = min(B, i + 1, 96)
+        r = b_eff - w
+        others = [t for t in range(m) if t != p][: r - 1]
+        expect = sorted(set(range(i - w + 1, i + 1)) | {p} | set(others))
+        assert sel.tolist() == expect
+
+
+def test_route_structure_random():
+    rng = _rng(11)
+    n, d = 512, 16
+    K = _rand_qk(rng, (n, d))
+    nodes = orc.build_tree(K)
+    for _ in range(200):
+        i = int(rng.integers(0, n))
+        w = int(rng.integers(1, 33))
+        B = int(rng.integers(-2, 110))
+        mk = int(rng.integers(1, 97))
+        q = _rand_qk(rng, (d,))
+        sel, exp = orc.route(K, nodes, q, i, B, w, mk)
+        b_eff = min(max(B, 1), i + 1, mk)
+        assert len(sel) == b_eff  # min(B_eff, i+1) == B_eff
+        assert (np.diff(sel) > 0).all()
+        nwin = min(b_eff, w, i + 1)
+        assert sel[-nwin:].tolist() == list(range(i - nwin + 1, i + 1))
+        routed = sel[:-nwin]
+        assert (routed <= i - w).all() and (routed >= 0).all()
+
+
+def _alt_route(K, q, i, B, w, max_keys):
+    """Independent formulation: intervals [lo, hi) halved recursively, sums straight from K,
+    roots as the largest aligned blocks taken greedily from the left."""
+    b_eff = min(max(B, 1), i + 1, max_keys)
+    win = [t for t in range(i, max(-1, i - w), -1)][:b_eff]
+    r = b_eff - len(win)
+    m = i - w + 1
+    exp = [0, 0]
+    routed = []
+    if r > 0 and m > 0:
+        F, lo = [], 0
+        while lo < m:
+            size = 1
+            while lo % (2 * size) == 0 and lo + 2 * size <= m:
+                size *= 2
+            F.append((lo, lo + size))
+            lo += size
+        qq = q.astype(np.int64)
+
+        def score(iv):
+            return int(K[iv[0]: iv[1]].astype(np.int64).sum(0) @ qq)
+
+        while any(hi - lo > 1 for lo, hi in F):
+            C = []
+            for lo, hi in F:
+                if hi - lo == 1:
+                    C.append((lo, hi))
+                    continue
+                exp[0 if hi - lo >= 4 else 1] += 1
+                mid = (lo + hi) // 2
+                C += [(lo, mid), (mid, hi)]
+            if len(C) > r:
+                C = sorted(C, key=lambda iv: (-score(iv), iv[0]))[:r]
+            F = C
+        routed = [lo for lo, _ in F]
+    return sorted(win + routed), tuple(exp)
+
+
+@pytest.mark.parametrize("n,d", [(8, 2), (16, 4), (64, 64), (256, 8)])
+def test_route_matches_independent_formulation(n, d):
+    rng = _rng(n * 7 + d)
+    for trial in range(60):
+        # small value ranges make ties frequent, which exercises the tie rule
+        lo, hi = (-16, 16) if trial % 2 else (-1, 1)
+        K = _rand_qk(rng, (n, d), lo, hi)
+        nodes = orc.build_tree(K)
+        q = _rand_qk(rng, (d,), lo, hi)
+        i = int(rng.integers(0, n))
+        w = int(rng.integers(1, 6))
+        B = int(rng.integers(1, n + 2))
+        sel, exp = orc.route(K, nodes, q, i, B, w, 96)
+        ref_sel, ref_exp = _alt_route(K, q, i, B, w, 96)
+        assert sel.tolist() == ref_sel
+        assert exp == ref_exp
+
+
+# ---------------------------------------------------------------- attention
+
+def _dense_causal(Q, K, Vf, q_start):
+    """Dense causal softmax attention in float64 (numpy), independent of the oracle."""
+    nq, d = Q.shape
+    S = Q.astype(np.float64) @ K.astype(np.float64).T / math.sqrt(d)
+    pos = q_start + np.arange(nq)
+    mask = np.arange(K.shape[0])[None, :] <= pos[:, None]
+    S = np.where(mask, S, -np.inf)
+    S = S - S.max(1, keepdims=True)
+    P = np.exp(S)
+    P /= P.sum(1, keepdims=True)
+    return P @ Vf
+
+
+@pytest.mark.parametrize("n,d,w", [(64, 8, 4), (256, 64, 16), (128, 128, 1)])
+def test_full_budget_is_dense_causal_attention(n, d, w):
+    rng = _rng(n + d + w)
+    K = _rand_qk(rng, (n, d))
+    Q = _rand_qk(rng, (n, d))
+    V = _rand_v_bits(rng, (n, d))
+    nodes = orc.build_tree(K)
+    bud = np.full(n, n + 7, dtype=np.int32)
+    res = orc.forward(Q, K, V, nodes, None, bud, q_start=0, window=w, max_keys=n)
+    ref = _dense_causal(Q, K, _bits_to_f64(V), 0)
+    assert np.abs(res["out"] - ref).max() <= 1e-12
+    assert (res["count"] == np.arange(1, n + 1)).all()
+
+
+def test_attention_closed_forms():
+    rng = _rng(3)
+    n, d = 32, 64
+    K = _rand_qk(rng, (n, d))
+    V = _rand_v_bits(rng, (n, d))
+    Vf = _bits_to_f64(V)
+    q = _rand_qk(rng, (d,))
+    # one key: the output is that value row, exactly
+    assert (orc.attend(q, K, V, np.array([9], dtype=np.int32)) == Vf[9]).all()
+    # zero query: uniform weights -> mean of the selected rows
+    sel = np.array([1, 4, 5, 30], dtype=np.int32)
+    out = orc.attend(np.zeros(d, dtype=np.int8), K, V, sel)
+    assert np.abs(out - Vf[sel].mean(0)).max() < 1e-15
+    # two keys with a known score gap: weights 1/(1+e^-g) and e^-g/(1+e^-g)
+    K2 = np.zeros((2, d), dtype=np.int8)
+    K2[0, 0] = 8
+    q2 = np.zeros(d, dtype=np.int8)
+    q2[0] = 2  # score gap 16 / sqrt(64) = 2
+    V2 = _rand_v_bits(rng, (2, d))
+    out = orc.attend(q2, K2, V2, np.array([0, 1], dtype=np.int32))
+    a = 1.0 / (1.0 + math.exp(-2.0))
+    ref = a * _bits_to_f64(V2)[0] + (1 - a) * _bits_to_f64(V2)[1]
+    assert np.abs(out - ref).max() < 1e-14
+    # empty selection gives zeros
+    assert (orc.attend(q, K, V, np.zeros(0, dtype=np.int32)) == 0).all()
+
+
+def test_forward_budget_override_clamp_and_predictor():
+    rng = _rng(21)
+    n, d = 128, 64
+    K = _rand_qk(rng, (n, d))
+    Q = _rand_qk(rng, (n, d))
+    V = _rand_v_bits(rng, (n, d))
+    W = rng.integers(-4, 5, size=(32, 2 * d)).astype(np.int8)
+    nodes = orc.build_tree(K)
+    res = orc.forward(Q, K, V, nodes, W, None, q_start=0, window=16, max_keys=96)
+    for i in [0, 5, 16, 17, 100, 127]:
+        c, _ = orc.predict(Q[i], orc.causal_sum(K, i), W)
+        assert res["budget"][i] == 3 * (c + 1)
+        sel, exp = orc.route(K, nodes, Q[i], i, 3 * (c + 1), 16, 96)
+        assert res["idx"][i, : res["count"][i]].tolist() == sel.tolist()
+        assert tuple(res["expansions"][i]) == exp
+        assert np.array_equal(res["out"][i], orc.attend(Q[i], K, V, sel))
+    bud = np.array([0, -5] + [3] * (n - 2), dtype=np.int32)
+    res = orc.forward(Q, K, V, nodes, None, bud, q_start=0, window=16, max_keys=96,
+                      rows=np.array([0, 1, 2], dtype=np.int32))
+    assert res["budget"][:3].tolist() == [1, 1, 3]
+    assert res["count"][:3].tolist() == [1, 1, 3]
