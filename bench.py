@@ -1,0 +1,436 @@
+"""Benchmark of the ALHR inference path: routed queries per second on one step of the
+configured workload (tree build + fused route/attend over every query), on N GPUs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl alhr|reference]
+
+N > 1 runs one process per GPU under torch.distributed.run (weak scaling: every rank processes
+its own full workload with its own seed; no collective on the data path). Prints one JSON line
+on rank 0. Inputs are seeded synthetic tensors generated on the device; L2 is flushed by a
+512 MiB write before every timed step; the timed region holds exactly K steps bracketed by a
+barrier and a device synchronisation; each step is timed with CUDA events on the launch stream
+and the job time is the maximum over ranks.
+
+--impl reference times the oracle (the plain CPU reference that the tests use) on the host
+cores, on a bounded sample of the same workload, with the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+METRIC = "routed queries/sec and achieved HBM GB/s vs ~8 TB/s roofline, N=16384, 1 B200"
+DEFAULT_WORKLOAD = "prefill_b2h8_n16384"
+L2_FLUSH_BYTES = 512 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="alhr", choices=["alhr", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-stride", type=int, default=8,
+                    help="CPU baseline: every k-th query row of every (b,h) block")
+    ap.add_argument("--ref-stride", type=int, default=64,
+                    help="--impl reference: every k-th query row of each step's block")
+    return ap.parse_args()
+
+
+def describe(wl) -> str:
+    pred = (f"predictor W int8 U[{wl.w_lo},{wl.w_hi}] 32x{2 * wl.d}" if wl.predictor
+            else f"fixed budget min(i+1,{wl.fixed_budget_cap})")
+    extra = f", {wl.plant_pairs} planted pairs/seq" if wl.plant_pairs else ""
+    return (f"{wl.name}: batch {wl.batch}, heads {wl.heads}, N={wl.n}, d={wl.d}, "
+            f"queries [{wl.q_start},{wl.q_start + wl.nq}), w={wl.window}, max_keys={wl.max_keys}, "
+            f"Q/K int8 U[{wl.qk_lo},{wl.qk_hi}], V bf16 N(0,1), {pred}{extra}")
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import torch.distributed as dist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist, dist.get_rank(), world
+    return None, 0, 1
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(dist, x: float) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.reader.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle (CPU) timing
+
+def oracle_sample(wl, stride: int, blocks=None, inp=None) -> dict:
+    """The oracle as it stands, on the host cores, on a bounded sample of the workload: for
+    each listed (b,h) block, its whole tree and every `stride`-th query row. Blocks run on a
+    thread pool, one block per thread (the oracle itself is single-threaded; ctypes releases
+    the GIL). The sample's wall time is scaled to all query rows of the listed blocks, and
+    the value is queries of those blocks per extrapolated second."""
+    from concurrent.futures import ThreadPoolExecutor
+    from oracle import oracle as orc
+    from tree_routed_sparse_b200 import synth
+
+    orc.lib()
+    if inp is None:
+        inp = synth.make_inputs(wl, "cpu")
+    if blocks is None:
+        blocks = [(b, h) for b in range(wl.batch) for h in range(wl.heads)]
+    rows = np.arange(0, wl.nq, max(1, min(stride, wl.nq)), dtype=np.int32)
+    Vbits = inp["V"].view(torch.int16).numpy().view(np.uint16)
+    W = None if inp["W"] is None else inp["W"].numpy()
+
+    def run(bh):
+        b, h = bh
+        K = inp["K"][b, h].numpy()
+        Q = inp["Q"][b, h].numpy()
+        bo = None if inp["budget_override"] is None else inp["budget_override"][b, h].numpy()
+        t0 = time.perf_counter()
+        nodes = orc.build_tree(K)
+        t1 = time.perf_counter()
+        orc.forward(Q, K, Vbits[b, h], nodes, W, bo, q_start=wl.q_start, window=wl.window,
+                    max_keys=wl.max_keys, rows=rows)
+        t2 = time.perf_counter()
+        return t1 - t0, t2 - t1
+
+    threads = max(1, min(os.cpu_count() or 1, len(blocks)))
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(threads) as ex:
+        res = list(ex.map(run, blocks))
+    wall = time.perf_counter() - t0
+    t_tree = sum(r[0] for r in res)
+    t_route = sum(r[1] for r in res)
+    scale = wl.nq / len(rows)
+    est_wall = wall * (t_tree + t_route * scale) / (t_tree + t_route)
+    total_q = len(blocks) * wl.nq
+    return {"value": total_q / est_wall, "unit": "queries/s", "cores": threads,
+            "kind": "oracle",
+            "sample": (f"{describe(wl)}; {len(blocks)} (b,h) blocks: each whole tree plus "
+                       f"every {max(1, min(stride, wl.nq))}-th query row ({len(rows)} of "
+                       f"{wl.nq}), time scaled to all rows; {threads} threads, one block per "
+                       f"thread; sample wall {wall:.2f} s"),
+            "sample_wall_s": wall}
+
+
+# ------------------------------------------------------------------ the GPU arm
+
+def run_alhr(args, dist, rank, world):
+    from tree_routed_sparse_b200 import alhr, metrics, synth
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = synth.WORKLOADS[args.workload].replace(seed=synth.WORKLOADS[args.workload].seed + rank)
+    vb = max(-wl.qk_lo, wl.qk_hi)
+    inp = synth.make_inputs(wl, dev)
+    Q, K, V, W, bo = inp["Q"], inp["K"], inp["V"], inp["W"], inp["budget_override"]
+    nodes = torch.empty((wl.batch, wl.heads, wl.n - 1, wl.d), dtype=torch.int32, device=dev)
+    out = torch.empty((wl.batch, wl.heads, wl.nq, wl.d), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    kw = dict(q_start=wl.q_start, window=wl.window, max_keys=wl.max_keys,
+              score_bits=wl.score_bits, value_bound=vb)
+
+    def step():
+        alhr.build_tree(K, nodes, value_bound=vb)
+        alhr.forward(Q, K, V, nodes, W=W, budget_override=bo, out=out, **kw)
+
+    # one untimed run with every output: counts for the byte model
+    alhr.build_tree(K, nodes, value_bound=vb)
+    full = alhr.forward(Q, K, V, nodes, W=W, budget_override=bo, want_count=True,
+                        want_expansions=True, want_budget=True, **kw)
+    torch.cuda.synchronize()
+    pos = np.broadcast_to(np.arange(wl.q_start, wl.q_start + wl.nq), (wl.bh, wl.nq))
+    fwd_bytes = metrics.forward_bytes(pos, wl.d, wl.window, full["count"].cpu().numpy(),
+                                      full["expansions"].cpu().numpy(),
+                                      full["budget"].cpu().numpy(), wl.predictor, wl.max_keys)
+    tree_bytes = metrics.tree_bytes(wl.bh, wl.n, wl.d)
+    mean_keys = float(full["count"].float().mean())
+    mean_budget = float(full["budget"].float().mean())
+    del full
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    barrier(dist)
+    torch.cuda.synchronize()
+    sampler.start()
+    wall0 = time.perf_counter()
+    for s in range(args.steps):
+        flush.fill_(s & 0xFF)
+        ev[s][0].record(stream)
+        alhr.build_tree(K, nodes, value_bound=vb)
+        ev[s][1].record(stream)
+        alhr.forward(Q, K, V, nodes, W=W, budget_override=bo, out=out, **kw)
+        ev[s][2].record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    barrier(dist)
+    clocks = sampler.stop()
+    t_tree = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_fwd = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    t_step = t_tree + t_fwd
+    t_job = max_over_ranks(dist, t_step)
+    queries = wl.bh * wl.nq
+    value = world * queries * args.steps / t_job
+
+    # end to end through the public API, host buffers: H2D of the step's inputs from pinned
+    # memory, tree + forward, D2H of the output, all inside the timed region
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in inp.items()}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = out_host.numel() * out_host.element_size()
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    dW = None if W is None else torch.empty_like(W)
+    dbo = None if bo is None else torch.empty_like(bo)
+
+    def e2e_step():
+        dQ.copy_(host["Q"], non_blocking=True)
+        dK.copy_(host["K"], non_blocking=True)
+        dV.copy_(host["V"], non_blocking=True)
+        if dW is not None:
+            dW.copy_(host["W"], non_blocking=True)
+        if dbo is not None:
+            dbo.copy_(host["budget_override"], non_blocking=True)
+        alhr.build_tree(dK, nodes, value_bound=vb)
+        alhr.forward(dQ, dK, dV, nodes, W=dW, budget_override=dbo, out=out, **kw)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    assert torch.equal(out_host, out.cpu())
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.e2e_steps)]
+    barrier(dist)
+    torch.cuda.synchronize()
+    for s in range(args.e2e_steps):
+        flush.fill_(s & 0xFF)
+        e2e_ev[s][0].record(stream)
+        e2e_step()
+        e2e_ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(dist)
+    t_e2e = max_over_ranks(dist, sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / 1e3)
+    e2e_value = world * queries * args.e2e_steps / t_e2e
+
+    if rank != 0:
+        return None
+
+    peaks = {}
+    try:
+        with open(os.path.join(HERE, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except OSError:
+        pass
+    peak = float(peaks.get("hbm_gbs", 6650.0))
+    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    fwd_launch_s = t_fwd / args.steps
+    achieved = fwd_bytes / fwd_launch_s / 1e9
+    traffic = profiled_traffic(args.workload)
+    tree_launches = math.ceil(int(math.log2(wl.n)) / 7)
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "queries/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": t_job / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int32",
+        "data": "synthetic (seeded SplitMix64; random int8 predictor weights, no trained model)",
+        "config": {
+            "workload": describe(wl),
+            "queries_per_step_per_gpu": queries,
+            "step": "alhr_build_tree + alhr_forward (fused budget, window, descent, attention)",
+            "l2": "flushed by a 512 MiB write before every timed step (not timed)",
+            "parallelism": f"{world} independent replica(s), one per GPU, no collective",
+            "score_bits": 32 if alhr.score_bits(alhr.make_dims(Q, K, **kw)) == 32 else 64,
+            "mean_keys_per_query": mean_keys,
+            "mean_budget": mean_budget,
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "query_kernel (fused alhr_forward)",
+            "achieved": achieved,
+            "peak": peak,
+            "unit": "GB/s",
+            "frac": achieved / peak,
+            "peak_source": f"{peak_src} hbm_gbs",
+            "algorithmic_bytes_per_launch": fwd_bytes,
+            "launch_ms": fwd_launch_s * 1e3,
+            "traffic": traffic,
+            "note": ("algorithmic bytes count every row the path reads as if from DRAM; the "
+                     "working set of one step (tree, keys, values) is smaller than L2, so "
+                     "repeat reads of upper tree levels are served by L2 and achieved can "
+                     "exceed the DRAM peak; traffic is the DRAM bytes ncu measured"),
+        },
+        "stages_ms": {"tree_build": t_tree / args.steps * 1e3,
+                      "forward": t_fwd / args.steps * 1e3,
+                      "tree_build_GBps": tree_bytes / (t_tree / args.steps) / 1e9},
+        "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * (tree_launches + 1),
+        "clocks": clocks,
+        "wall_s_timed_region": wall,
+    }
+    return line
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary, if that
+    summary was taken on the kernel source as it is now; else None."""
+    path = os.path.join(HERE, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(workload)
+    except (OSError, ValueError):
+        return None
+    if not rec:
+        return None
+    from tree_routed_sparse_b200 import build
+    if rec.get("source_hash") != build._hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        # the oracle on the host cores; under torchrun only rank 0 works
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        if rank != 0:
+            return
+        from tree_routed_sparse_b200 import synth
+        wl = synth.WORKLOADS[args.workload]
+        inp = synth.make_inputs(wl, "cpu")
+        all_blocks = [(b, h) for b in range(wl.batch) for h in range(wl.heads)]
+        # one step = one (b,h) block (whole tree, every stride-th query row), round robin
+        pick = lambda k: [all_blocks[j % len(all_blocks)] for j in range(k)]
+        if args.warmup:
+            oracle_sample(wl, args.ref_stride, pick(args.warmup), inp)
+        r = oracle_sample(wl, args.ref_stride, pick(args.steps), inp)
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": r["value"], "unit": "queries/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": wl.nq / r["value"] * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64",
+            "data": "synthetic", "config": {"workload": describe(wl),
+                                            "step": "one (b,h) block of the workload"},
+            "cpu_baseline": {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")},
+            "e2e": {"value": r["value"], "unit": "queries/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }))
+        return
+
+    dist, rank, world = dist_setup(args.gpus)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    from tree_routed_sparse_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(dist)
+    line = run_alhr(args, dist, rank, world)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            from tree_routed_sparse_b200 import synth
+            cb = oracle_sample(synth.WORKLOADS[args.workload], args.cpu_sample_stride)
+            line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        print(json.dumps(line))
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

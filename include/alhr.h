@@ -47,6 +47,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define ALHR_API __attribute__((visibility("default")))
+#else
+#define ALHR_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -62,6 +68,7 @@ typedef enum {
 /* Bits OR-ed into the optional device word *dev_err. */
 #define ALHR_DEVERR_BUDGET_LOW  0x1u /* a budget < 1 was read; it was treated as 1          */
 #define ALHR_DEVERR_VALUE_RANGE 0x2u /* a Q or K value had |value| > value_bound            */
+#define ALHR_DEVERR_INDEX       0x4u /* alhr_attend: an idx entry outside [0, i] was skipped */
 
 /* Problem sizes, shared by every entry point. */
 typedef struct {
@@ -78,23 +85,23 @@ typedef struct {
 } alhr_dims;
 
 /* Number of tree rows per (b,h): n - 1. Returns 0 when n is not a power of two in [2, 2^20]. */
-size_t alhr_tree_rows(int32_t n);
+ALHR_API size_t alhr_tree_rows(int32_t n);
 
 /* Row offset of tree level `level` (1 <= level <= log2 n) inside one (b,h) block of `nodes`:
  * level l holds n >> l rows starting at row n - (n >> (l-1)); row j of level l is the sum of
  * keys [j*2^l, (j+1)*2^l). Level 0 (the keys themselves) is K and is not stored.
  * Returns (size_t)-1 for an invalid pair. */
-size_t alhr_tree_level_offset(int32_t n, int32_t level);
+ALHR_API size_t alhr_tree_level_offset(int32_t n, int32_t level);
 
 /* Score width the kernels will use for these sizes (32 or 64), or a negative alhr_status
  * (-ALHR_ERR_...) when the sizes are invalid or score_bits = 32 cannot be exact. */
-int32_t alhr_score_bits(const alhr_dims* dims);
+ALHR_API int32_t alhr_score_bits(const alhr_dims* dims);
 
 /* Human-readable name of a status code (static storage, never NULL). */
-const char* alhr_status_string(int32_t status);
+ALHR_API const char* alhr_status_string(int32_t status);
 
 /* Build identification (static storage): target architecture and library version. */
-const char* alhr_build_info(void);
+ALHR_API const char* alhr_build_info(void);
 
 /*
  * alhr_build_tree -- the static key tree [README §Inference stage, first paragraph: the tree
@@ -108,7 +115,7 @@ const char* alhr_build_info(void);
  *   nodes   device, int32 [batch][heads][n-1][d], fully overwritten
  *   dev_err device uint32 or NULL; ALHR_DEVERR_VALUE_RANGE if some |K| > value_bound
  */
-alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, int32_t* nodes,
+ALHR_API alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, int32_t* nodes,
                             uint32_t* dev_err, void* stream);
 
 /*
@@ -125,7 +132,7 @@ alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, int32_t* nod
  *   budget       device int32 [batch][heads][nq], overwritten
  *   dev_err      as above (ALHR_DEVERR_VALUE_RANGE for |q| > value_bound)
  */
-alhr_status alhr_predict_budget(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
+ALHR_API alhr_status alhr_predict_budget(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
                                 const int32_t* nodes, const int8_t* W, int32_t* budget,
                                 uint32_t* dev_err, void* stream);
 
@@ -147,7 +154,7 @@ alhr_status alhr_predict_budget(const alhr_dims* dims, const int8_t* Q, const in
  *   expansions device int32 [..][2] or NULL: {level >= 2 nodes expanded, level-1 nodes expanded}
  *   dev_err    as above (ALHR_DEVERR_BUDGET_LOW, ALHR_DEVERR_VALUE_RANGE)
  */
-alhr_status alhr_route(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
+ALHR_API alhr_status alhr_route(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
                        const int32_t* nodes, const int32_t* budget, int32_t* idx, int32_t* count,
                        int32_t* expansions, uint32_t* dev_err, void* stream);
 
@@ -157,11 +164,11 @@ alhr_status alhr_route(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
  *
  * out_i = sum_j softmax_j(s) V[j] over j in idx[0..count), s_j = (q_i . K[j]) / sqrt(d), with the
  * integer dot product exact and the softmax and sum in fp32. A query with count <= 0 gets a
- * zero row. Entries of idx outside [0, i] are not read (they are skipped).
+ * zero row. Entries of idx outside [0, i] are skipped (not read) and flag ALHR_DEVERR_INDEX.
  *   Q, K, V, idx, count  device inputs (layouts above)
  *   out                  device float [batch][heads][nq][d], overwritten
  */
-alhr_status alhr_attend(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
+ALHR_API alhr_status alhr_attend(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
                         const uint16_t* V, const int32_t* idx, const int32_t* count, float* out,
                         uint32_t* dev_err, void* stream);
 
@@ -177,7 +184,7 @@ alhr_status alhr_attend(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
  *                    clamp to >= 1)
  * Results equal alhr_predict_budget + alhr_route + alhr_attend on the same inputs.
  */
-alhr_status alhr_forward(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
+ALHR_API alhr_status alhr_forward(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
                          const uint16_t* V, const int32_t* nodes, const int8_t* W,
                          const int32_t* budget_override, float* out, int32_t* idx,
                          int32_t* count, int32_t* expansions, int32_t* budget_out,

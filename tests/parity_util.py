@@ -1,0 +1,43 @@
+"""Helpers shared by the GPU parity tests: run the oracle on the same seeded inputs."""
+import numpy as np
+import torch
+
+from oracle import oracle as orc
+
+
+def v_bits(V: torch.Tensor) -> np.ndarray:
+    return V.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def oracle_slice(inp_cpu: dict, wl, b: int, h: int, rows=None, nodes=None) -> dict:
+    """Oracle results for the (b, h) block of a workload's inputs (host tensors)."""
+    K = inp_cpu["K"][b, h].numpy()
+    Q = inp_cpu["Q"][b, h].numpy()
+    V = v_bits(inp_cpu["V"][b, h])
+    if nodes is None:
+        nodes = orc.build_tree(K)
+    W = None if inp_cpu["W"] is None else inp_cpu["W"].numpy()
+    bo = None if inp_cpu["budget_override"] is None else inp_cpu["budget_override"][b, h].numpy()
+    res = orc.forward(Q, K, V, nodes, W, bo, q_start=wl.q_start, window=wl.window,
+                      max_keys=wl.max_keys, rows=rows)
+    res["nodes"] = nodes
+    return res
+
+
+def compare_rows(gpu: dict, ref: dict, b: int, h: int, rows, tol=1e-3, what=""):
+    """Bit-exact idx/count/expansions/budget and |out - oracle| <= tol on the given rows."""
+    rows = np.asarray(rows)
+    for key in ("idx", "count", "expansions", "budget"):
+        if key in gpu:
+            g = gpu[key][b, h].cpu().numpy()[rows]
+            r = ref[key][rows]
+            if not np.array_equal(g, r):
+                bad = np.nonzero((g != r).reshape(len(rows), -1).any(1))[0][:5]
+                raise AssertionError(f"{what} {key} differs at rows {rows[bad].tolist()}:\n"
+                                     f"gpu {g[bad].tolist()}\noracle {r[bad].tolist()}")
+    if "out" in gpu:
+        g = gpu["out"][b, h].cpu().numpy()[rows].astype(np.float64)
+        err = np.abs(g - ref["out"][rows]).max() if len(rows) else 0.0
+        assert err <= tol, f"{what} max |out - oracle| = {err:.3e} > {tol}"
+        return float(err)
+    return 0.0

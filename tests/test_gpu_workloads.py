@@ -1,0 +1,95 @@
+"""Parity at the benchmark table's full sizes, in the benchmark's launch configuration.
+
+Each workload runs once exactly as the benchmark times it (tree build, then the fused forward
+with only `out` requested) and once with every optional output; `out` must be identical between
+the two. Sampled (b, h) blocks are then checked against the oracle on sampled query rows that
+include the first positions, the last positions (the ragged end of the grid) and a stride in
+between: tree sums, budgets, index sets, counts and expansions bit-exact, outputs within 1e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as orc
+from parity_util import compare_rows, oracle_slice
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def alhr():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from tree_routed_sparse_b200 import build
+    build.build()
+    from tree_routed_sparse_b200 import alhr as A
+    A.lib()
+    return A
+
+
+def _sample_rows(nq, rng, k=40):
+    if nq <= 3 * k:
+        return np.arange(nq)
+    mid = rng.choice(np.arange(k, nq - k), size=k, replace=False)
+    return np.unique(np.r_[np.arange(k // 2), mid, np.arange(nq - k // 2, nq)])
+
+
+def _slice_inputs(inp, wl, b, h):
+    """Host copies of one (b, h) block (plus W / budget), as oracle_slice expects."""
+    cut = lambda t: None if t is None else t[b:b + 1, h:h + 1].cpu()
+    return dict(Q=cut(inp["Q"]), K=cut(inp["K"]), V=cut(inp["V"]),
+                W=None if inp["W"] is None else inp["W"].cpu(),
+                budget_override=cut(inp["budget_override"]))
+
+
+@pytest.mark.parametrize("name,blocks", [
+    ("tiny_prefill_n1024", [(0, 0)]),
+    ("prefill_b4h8_n4096", [(0, 0), (3, 7)]),
+    ("prefill_b2h8_n16384", [(0, 3), (1, 7)]),
+    ("recall_b2h4_n16384_d128", [(0, 0), (1, 3)]),
+    ("decode_s64h8_n262144_d128", [(0, 0), (5, 1), (17, 2), (31, 3), (40, 4), (50, 5),
+                                   (62, 6), (63, 7)]),
+])
+def test_workload_parity(alhr, name, blocks):
+    from tree_routed_sparse_b200 import synth
+    wl = synth.WORKLOADS[name]
+    need = wl.bh * wl.n * wl.d * (1 + 2 + 4) + wl.bh * wl.nq * wl.d * 5
+    free, _ = torch.cuda.mem_get_info()
+    if need > free - (2 << 30):
+        pytest.skip(f"{name} needs {need / 2**30:.1f} GiB, {free / 2**30:.1f} GiB free")
+    inp = synth.make_inputs(wl, "cuda")
+    vb = max(-wl.qk_lo, wl.qk_hi)
+    kw = dict(q_start=wl.q_start, window=wl.window, max_keys=wl.max_keys,
+              score_bits=wl.score_bits, value_bound=vb)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    # the benchmark's configuration
+    nodes = alhr.build_tree(inp["K"], value_bound=vb, dev_err=err)
+    bench_out = alhr.forward(inp["Q"], inp["K"], inp["V"], nodes, W=inp["W"],
+                             budget_override=inp["budget_override"], dev_err=err, **kw)["out"]
+    full = alhr.forward(inp["Q"], inp["K"], inp["V"], nodes, W=inp["W"],
+                        budget_override=inp["budget_override"], want_idx=True, want_count=True,
+                        want_expansions=True, want_budget=True, dev_err=err, **kw)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(bench_out, full["out"])
+    rng = np.random.default_rng(0)
+    for b, h in blocks:
+        rows = _sample_rows(wl.nq, rng)
+        cpu = _slice_inputs(inp, wl, b, h)
+        ref = oracle_slice(cpu, wl, 0, 0, rows=rows)
+        assert np.array_equal(nodes[b, h].cpu().numpy(), ref["nodes"]), f"tree {b},{h}"
+        sub = {k: v[b:b + 1, h:h + 1].cpu() for k, v in full.items()}
+        compare_rows(sub, ref, 0, 0, rows, TOL, f"{name} b{b}h{h}")
+    if wl.plant_pairs:
+        # diagnostic only: how often the planted key lands in its query's selection
+        hits = 0
+        idx = full["idx"].cpu()
+        for b in range(wl.batch):
+            p, u = synth.plant_positions(wl, b)
+            sel = idx[b][:, u]  # [H, P, max_keys]
+            hits += int((sel == p.view(1, -1, 1).to(torch.int32)).any(-1).sum())
+        print(f"recall@selection {hits / (wl.batch * wl.heads * wl.plant_pairs):.3f}")
+    del inp, nodes, full, bench_out
+    torch.cuda.empty_cache()

@@ -1,0 +1,198 @@
+"""Thin ctypes binding of libalhr.so (the C ABI declared in include/alhr.h).
+
+Argument marshalling only: shapes are read from the torch tensors, outputs are allocated with
+torch on the inputs' device, raw pointers and the current CUDA stream are passed to the C entry
+points, and a non-OK status raises AlhrError. Every step of the path runs in the library's CUDA
+kernels; there is no fallback of any kind. Loading fails loudly when the library has not been
+built (python -m tree_routed_sparse_b200.build).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_lib", "libalhr.so")
+
+ALHR_OK = 0
+STATUS = {0: "ALHR_OK", 1: "ALHR_ERR_INVALID_ARG", 2: "ALHR_ERR_UNSUPPORTED",
+          3: "ALHR_ERR_OVERFLOW", 4: "ALHR_ERR_CUDA"}
+DEVERR_BUDGET_LOW = 0x1
+DEVERR_VALUE_RANGE = 0x2
+DEVERR_INDEX = 0x4
+
+EXPORTS = ["alhr_tree_rows", "alhr_tree_level_offset", "alhr_score_bits",
+           "alhr_status_string", "alhr_build_info", "alhr_build_tree", "alhr_predict_budget",
+           "alhr_route", "alhr_attend", "alhr_forward"]
+
+
+class AlhrError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_int32) for f in
+                ("batch", "heads", "n", "d", "q_start", "nq", "window", "max_keys",
+                 "score_bits", "value_bound")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library with argument types set. Raises if it was never built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libalhr.so is not built ({LIB_PATH}); run "
+                               "`python -m tree_routed_sparse_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        DP = ctypes.POINTER(Dims)
+        L.alhr_tree_rows.argtypes, L.alhr_tree_rows.restype = [I32], SZ
+        L.alhr_tree_level_offset.argtypes, L.alhr_tree_level_offset.restype = [I32, I32], SZ
+        L.alhr_score_bits.argtypes, L.alhr_score_bits.restype = [DP], I32
+        L.alhr_status_string.argtypes, L.alhr_status_string.restype = [I32], ctypes.c_char_p
+        L.alhr_build_info.argtypes, L.alhr_build_info.restype = [], ctypes.c_char_p
+        L.alhr_build_tree.argtypes = [DP, P, P, P, P]
+        L.alhr_predict_budget.argtypes = [DP, P, P, P, P, P, P, P]
+        L.alhr_route.argtypes = [DP, P, P, P, P, P, P, P, P, P]
+        L.alhr_attend.argtypes = [DP, P, P, P, P, P, P, P, P]
+        L.alhr_forward.argtypes = [DP, P, P, P, P, P, P, P, P, P, P, P, P, P]
+        for f in ("alhr_build_tree", "alhr_predict_budget", "alhr_route", "alhr_attend",
+                  "alhr_forward"):
+            getattr(L, f).restype = I32
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != ALHR_OK:
+        raise AlhrError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def make_dims(Q, K, q_start=0, window=16, max_keys=96, score_bits=0, value_bound=16) -> Dims:
+    B, H, n, d = K.shape
+    nq = 0 if Q is None else Q.shape[2]
+    return Dims(B, H, n, d, q_start, nq, window, max_keys, score_bits, value_bound)
+
+
+def _want(t, dtype, shape, name):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous {dtype} {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+
+
+def tree_rows(n: int) -> int:
+    return int(lib().alhr_tree_rows(n))
+
+
+def score_bits(dims: Dims) -> int:
+    return int(lib().alhr_score_bits(ctypes.byref(dims)))
+
+
+def build_tree(K: torch.Tensor, nodes: torch.Tensor | None = None, value_bound: int = 16,
+               dev_err: torch.Tensor | None = None) -> torch.Tensor:
+    """K int8 [B,H,n,d] -> level-major int32 tree [B,H,n-1,d]."""
+    B, H, n, d = K.shape
+    _want(K, torch.int8, (B, H, n, d), "K")
+    if nodes is None:
+        nodes = torch.empty((B, H, n - 1, d), dtype=torch.int32, device=K.device)
+    _want(nodes, torch.int32, (B, H, n - 1, d), "nodes")
+    dims = make_dims(None, K, value_bound=value_bound)
+    _check(lib().alhr_build_tree(ctypes.byref(dims), _ptr(K), _ptr(nodes), _ptr(dev_err),
+                                 _stream(K.device)), "alhr_build_tree")
+    return nodes
+
+
+def predict_budget(Q, K, nodes, W, q_start=0, window=16, max_keys=96, score_bits=0,
+                   value_bound=16, budget=None, dev_err=None) -> torch.Tensor:
+    dims = make_dims(Q, K, q_start, window, max_keys, score_bits, value_bound)
+    B, H, nq, d = Q.shape
+    if budget is None:
+        budget = torch.empty((B, H, nq), dtype=torch.int32, device=Q.device)
+    _want(Q, torch.int8, (B, H, nq, d), "Q")
+    _want(W, torch.int8, (32, 2 * d), "W")
+    _want(budget, torch.int32, (B, H, nq), "budget")
+    _check(lib().alhr_predict_budget(ctypes.byref(dims), _ptr(Q), _ptr(K), _ptr(nodes), _ptr(W),
+                                     _ptr(budget), _ptr(dev_err), _stream(Q.device)),
+           "alhr_predict_budget")
+    return budget
+
+
+def route(Q, K, nodes, budget, q_start=0, window=16, max_keys=96, score_bits=0,
+          value_bound=16, with_expansions=True, dev_err=None) -> dict:
+    dims = make_dims(Q, K, q_start, window, max_keys, score_bits, value_bound)
+    B, H, nq, d = Q.shape
+    _want(budget, torch.int32, (B, H, nq), "budget")
+    idx = torch.empty((B, H, nq, max_keys), dtype=torch.int32, device=Q.device)
+    count = torch.empty((B, H, nq), dtype=torch.int32, device=Q.device)
+    exp = (torch.empty((B, H, nq, 2), dtype=torch.int32, device=Q.device)
+           if with_expansions else None)
+    _check(lib().alhr_route(ctypes.byref(dims), _ptr(Q), _ptr(K), _ptr(nodes), _ptr(budget),
+                            _ptr(idx), _ptr(count), _ptr(exp), _ptr(dev_err), _stream(Q.device)),
+           "alhr_route")
+    return dict(idx=idx, count=count, expansions=exp)
+
+
+def attend(Q, K, V, idx, count, q_start=0, window=16, max_keys=96, value_bound=16,
+           out=None, dev_err=None) -> torch.Tensor:
+    dims = make_dims(Q, K, q_start, window, max_keys, 0, value_bound)
+    B, H, nq, d = Q.shape
+    _want(V, torch.bfloat16, K.shape, "V")
+    _want(idx, torch.int32, (B, H, nq, max_keys), "idx")
+    if out is None:
+        out = torch.empty((B, H, nq, d), dtype=torch.float32, device=Q.device)
+    _check(lib().alhr_attend(ctypes.byref(dims), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
+                             _ptr(count), _ptr(out), _ptr(dev_err), _stream(Q.device)),
+           "alhr_attend")
+    return out
+
+
+def forward(Q, K, V, nodes, W=None, budget_override=None, q_start=0, window=16, max_keys=96,
+            score_bits=0, value_bound=16, out=None, want_idx=False, want_count=False,
+            want_expansions=False, want_budget=False, dev_err=None) -> dict:
+    """The fused path. Returns a dict with `out` and the optional outputs asked for."""
+    dims = make_dims(Q, K, q_start, window, max_keys, score_bits, value_bound)
+    B, H, nq, d = Q.shape
+    dev = Q.device
+    _want(Q, torch.int8, (B, H, nq, d), "Q")
+    _want(K, torch.int8, (B, H, K.shape[2], d), "K")
+    _want(V, torch.bfloat16, K.shape, "V")
+    _want(nodes, torch.int32, (B, H, K.shape[2] - 1, d), "nodes")
+    if W is not None:
+        _want(W, torch.int8, (32, 2 * d), "W")
+    if budget_override is not None:
+        _want(budget_override, torch.int32, (B, H, nq), "budget_override")
+    if out is None:
+        out = torch.empty((B, H, nq, d), dtype=torch.float32, device=dev)
+    res = dict(out=out)
+    mk = lambda shape: torch.empty(shape, dtype=torch.int32, device=dev)
+    if want_idx:
+        res["idx"] = mk((B, H, nq, max_keys))
+    if want_count:
+        res["count"] = mk((B, H, nq))
+    if want_expansions:
+        res["expansions"] = mk((B, H, nq, 2))
+    if want_budget:
+        res["budget"] = mk((B, H, nq))
+    _check(lib().alhr_forward(ctypes.byref(dims), _ptr(Q), _ptr(K), _ptr(V), _ptr(nodes),
+                              _ptr(W), _ptr(budget_override), _ptr(out), _ptr(res.get("idx")),
+                              _ptr(res.get("count")), _ptr(res.get("expansions")),
+                              _ptr(res.get("budget")), _ptr(dev_err), _stream(dev)),
+           "alhr_forward")
+    return res

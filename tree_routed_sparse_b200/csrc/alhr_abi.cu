@@ -1,0 +1,191 @@
+// alhr_abi.cu -- the C ABI of libalhr.so: argument checks, score-width choice, launches.
+//
+// Every entry point checks its arguments on the host before anything is launched and returns
+// a status; nothing is allocated and no state is kept between calls.
+#include <cmath>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/alhr.h"
+#include "alhr_device.cuh"
+#include "internal.h"
+
+namespace {
+
+bool pow2_in_range(int32_t n) { return n >= 2 && n <= (1 << 20) && (n & (n - 1)) == 0; }
+
+int log2_exact(int32_t n) {
+  int l = 0;
+  while ((int64_t(1) << l) < n) ++l;
+  return l;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int value_bound_of(const alhr_dims* d) { return d->value_bound == 0 ? 16 : d->value_bound; }
+
+// Sizes shared by every entry point.
+alhr_status check_common(const alhr_dims* d) {
+  if (!d) return ALHR_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->heads < 1) return ALHR_ERR_INVALID_ARG;
+  if (!pow2_in_range(d->n)) return ALHR_ERR_INVALID_ARG;
+  if (d->d != 64 && d->d != 128) return ALHR_ERR_UNSUPPORTED;
+  if (d->value_bound < 0 || d->value_bound > 127) return ALHR_ERR_INVALID_ARG;
+  return ALHR_OK;
+}
+
+alhr_status check_queries(const alhr_dims* d) {
+  const alhr_status s = check_common(d);
+  if (s != ALHR_OK) return s;
+  if (d->q_start < 0 || d->nq < 0 || int64_t(d->q_start) + d->nq > d->n) return ALHR_ERR_INVALID_ARG;
+  if (d->window < 1) return ALHR_ERR_INVALID_ARG;
+  if (d->window > 32) return ALHR_ERR_UNSUPPORTED;
+  if (d->max_keys < 1) return ALHR_ERR_INVALID_ARG;
+  if (d->max_keys > alhr::kMaxKeys) return ALHR_ERR_UNSUPPORTED;
+  if (d->score_bits != 0 && d->score_bits != 32 && d->score_bits != 64) return ALHR_ERR_INVALID_ARG;
+  return ALHR_OK;
+}
+
+// Largest |q . node| over every node a query can score: the biggest root of [0, i - w] has
+// level <= log2 n - 1, so |score| <= d * vb^2 * n/2 (and d * vb^2 for a key).
+int64_t score_bound(const alhr_dims* d) {
+  const int64_t vb = value_bound_of(d);
+  return int64_t(d->d) * vb * vb * (int64_t(d->n) / 2);
+}
+
+int resolve_bits(const alhr_dims* d, alhr_status* st) {
+  const bool fits32 = score_bound(d) <= int64_t(INT32_MAX);
+  *st = ALHR_OK;
+  if (d->score_bits == 32) {
+    if (!fits32) *st = ALHR_ERR_OVERFLOW;
+    return 32;
+  }
+  if (d->score_bits == 64) return 64;
+  return fits32 ? 32 : 64;
+}
+
+alhr::QueryArgs base_args(const alhr_dims* d) {
+  alhr::QueryArgs a{};
+  a.n = d->n;
+  a.L = log2_exact(d->n);
+  a.q_start = d->q_start;
+  a.nq = d->nq;
+  a.window = d->window;
+  a.max_keys = d->max_keys;
+  a.value_bound = value_bound_of(d);
+  a.num_queries = int64_t(d->batch) * d->heads * d->nq;
+  a.scale = float(1.0 / std::sqrt(double(d->d)));
+  return a;
+}
+
+alhr_status from_cuda(cudaError_t e) { return e == cudaSuccess ? ALHR_OK : ALHR_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t alhr_tree_rows(int32_t n) { return pow2_in_range(n) ? size_t(n) - 1 : 0; }
+
+size_t alhr_tree_level_offset(int32_t n, int32_t level) {
+  if (!pow2_in_range(n) || level < 1 || level > log2_exact(n)) return size_t(-1);
+  return size_t(n) - size_t(n >> (level - 1));
+}
+
+int32_t alhr_score_bits(const alhr_dims* d) {
+  alhr_status s = check_queries(d);
+  if (s != ALHR_OK) return -int32_t(s);
+  const int bits = resolve_bits(d, &s);
+  return s == ALHR_OK ? bits : -int32_t(s);
+}
+
+const char* alhr_status_string(int32_t status) {
+  switch (status) {
+    case ALHR_OK: return "ALHR_OK";
+    case ALHR_ERR_INVALID_ARG: return "ALHR_ERR_INVALID_ARG";
+    case ALHR_ERR_UNSUPPORTED: return "ALHR_ERR_UNSUPPORTED";
+    case ALHR_ERR_OVERFLOW: return "ALHR_ERR_OVERFLOW";
+    case ALHR_ERR_CUDA: return "ALHR_ERR_CUDA";
+    default: return "ALHR_ERR_UNKNOWN";
+  }
+}
+
+const char* alhr_build_info(void) { return "libalhr 0.1 sm_100a"; }
+
+alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, int32_t* nodes,
+                            uint32_t* dev_err, void* stream) {
+  const alhr_status s = check_common(dims);
+  if (s != ALHR_OK) return s;
+  if (!K || !nodes || !aligned16(K) || !aligned16(nodes)) return ALHR_ERR_INVALID_ARG;
+  const long long bh = (long long)dims->batch * dims->heads;
+  return from_cuda(alhr::launch_build_tree(K, nodes, bh, dims->n, dims->d, value_bound_of(dims),
+                                           dev_err, static_cast<cudaStream_t>(stream)));
+}
+
+alhr_status alhr_predict_budget(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
+                                const int32_t* nodes, const int8_t* W, int32_t* budget,
+                                uint32_t* dev_err, void* stream) {
+  alhr_status s = check_queries(dims);
+  if (s != ALHR_OK) return s;
+  const int bits = resolve_bits(dims, &s);
+  if (s != ALHR_OK) return s;
+  if (dims->nq == 0) return ALHR_OK;  // nothing to read or write
+  if (!Q || !K || !nodes || !W || !budget) return ALHR_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(nodes) || !aligned16(W)) return ALHR_ERR_INVALID_ARG;
+  alhr::QueryArgs a = base_args(dims);
+  a.Q = Q; a.K = K; a.nodes = nodes; a.W = W; a.budget_out = budget; a.dev_err = dev_err;
+  return from_cuda(alhr::launch_predict(a, dims->d, bits, static_cast<cudaStream_t>(stream)));
+}
+
+alhr_status alhr_route(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
+                       const int32_t* nodes, const int32_t* budget, int32_t* idx, int32_t* count,
+                       int32_t* expansions, uint32_t* dev_err, void* stream) {
+  alhr_status s = check_queries(dims);
+  if (s != ALHR_OK) return s;
+  const int bits = resolve_bits(dims, &s);
+  if (s != ALHR_OK) return s;
+  if (dims->nq == 0) return ALHR_OK;  // nothing to read or write
+  if (!Q || !K || !nodes || !budget || !idx || !count) return ALHR_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(nodes)) return ALHR_ERR_INVALID_ARG;
+  alhr::QueryArgs a = base_args(dims);
+  a.Q = Q; a.K = K; a.nodes = nodes; a.budget_in = budget;
+  a.idx_out = idx; a.count_out = count; a.exp_out = expansions; a.dev_err = dev_err;
+  return from_cuda(alhr::launch_route(a, dims->d, bits, static_cast<cudaStream_t>(stream)));
+}
+
+alhr_status alhr_attend(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
+                        const uint16_t* V, const int32_t* idx, const int32_t* count, float* out,
+                        uint32_t* dev_err, void* stream) {
+  const alhr_status s = check_queries(dims);
+  if (s != ALHR_OK) return s;
+  if (dims->nq == 0) return ALHR_OK;  // nothing to read or write
+  if (!Q || !K || !V || !idx || !count || !out) return ALHR_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return ALHR_ERR_INVALID_ARG;
+  alhr::QueryArgs a = base_args(dims);
+  a.Q = Q; a.K = K; a.V = V; a.idx_in = idx; a.count_in = count; a.out = out; a.dev_err = dev_err;
+  return from_cuda(alhr::launch_attend(a, dims->d, static_cast<cudaStream_t>(stream)));
+}
+
+alhr_status alhr_forward(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
+                         const uint16_t* V, const int32_t* nodes, const int8_t* W,
+                         const int32_t* budget_override, float* out, int32_t* idx,
+                         int32_t* count, int32_t* expansions, int32_t* budget_out,
+                         uint32_t* dev_err, void* stream) {
+  alhr_status s = check_queries(dims);
+  if (s != ALHR_OK) return s;
+  const int bits = resolve_bits(dims, &s);
+  if (s != ALHR_OK) return s;
+  if (dims->nq == 0) return ALHR_OK;  // nothing to read or write
+  if (!Q || !K || !V || !nodes || !out) return ALHR_ERR_INVALID_ARG;
+  if (!W && !budget_override) return ALHR_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(nodes) || !aligned16(out))
+    return ALHR_ERR_INVALID_ARG;
+  if (!budget_override && !aligned16(W)) return ALHR_ERR_INVALID_ARG;
+  alhr::QueryArgs a = base_args(dims);
+  a.Q = Q; a.K = K; a.V = V; a.nodes = nodes; a.W = W; a.budget_in = budget_override;
+  a.out = out; a.idx_out = idx; a.count_out = count; a.exp_out = expansions;
+  a.budget_out = budget_out; a.dev_err = dev_err;
+  return from_cuda(alhr::launch_forward(a, dims->d, bits, budget_override == nullptr,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,22 @@
+// internal.h -- launchers shared between the C ABI layer and the kernel files.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace alhr {
+
+struct QueryArgs;
+
+// Tree build: levels 1..log2 n of every (b,h) block (see tree_build.cu).
+cudaError_t launch_build_tree(const int8_t* K, int32_t* nodes, long long bh, int n, int d,
+                              int value_bound, uint32_t* dev_err, cudaStream_t st);
+
+// Warp-per-query kernels (see query_kernels.cu).
+cudaError_t launch_forward(const QueryArgs& a, int d, int score_bits, bool predict,
+                           cudaStream_t st);
+cudaError_t launch_route(const QueryArgs& a, int d, int score_bits, cudaStream_t st);
+cudaError_t launch_predict(const QueryArgs& a, int d, int score_bits, cudaStream_t st);
+cudaError_t launch_attend(const QueryArgs& a, int d, cudaStream_t st);
+
+}  // namespace alhr
