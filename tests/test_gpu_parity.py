@@ -200,7 +200,7 @@ def test_attend_skips_bad_indices(alhr, synth):
     out = alhr.attend(inp["Q"], inp["K"], inp["V"], idx, count, dev_err=err)
     torch.cuda.synchronize()
     assert int(err.item()) & alhr.DEVERR_INDEX
-    Q, K, V = (inp[k][0, 0].cpu().numpy() for k in "QKV")
+    Q, K = (inp[k][0, 0].cpu().numpy() for k in "QK")
     Vb = v_bits(inp["V"][0, 0])
     o = out[0, 0].cpu().numpy()
     assert np.all(o[0] == 0)
