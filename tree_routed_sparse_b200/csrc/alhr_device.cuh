@@ -1,10 +1,12 @@
 // alhr_device.cuh -- device building blocks of the warp-per-query ALHR path (sm_100a).
 //
-// One warp owns one query. Lane l owns dims [l*DPL, (l+1)*DPL) of every d-wide row (DPL = d/32),
-// so every row the warp reads is one coalesced access of d (keys), 2d (values) or 4d (tree
-// sums) bytes. Scores of up to R rows are finished together by a transposed butterfly (one
-// shuffle per row instead of five). The frontier and the candidates of the descent live in a
-// per-warp shared-memory buffer.
+// One warp owns one query. Rows are scored in "row groups": TPR = d/16 consecutive lanes share a
+// row and each lane holds 16 of its dims (dims 4*(sub + TPR*v) + e for v, e < 4, sub = lane %
+// TPR), so one warp pass scores RPI = 32/TPR rows (8 at d=64, 4 at d=128): a tree row (int32) is
+// four 16-byte loads and 16 multiply-adds per lane, a key row (int8) four 4-byte loads and four
+// dp4a per lane, and a row score costs log2(TPR) shuffles. The value rows of the final weighted
+// sum use the plain layout instead: lane l owns dims [l*d/32, (l+1)*d/32) of every value row.
+// The frontier and the candidates of the descent live in a per-warp shared-memory buffer.
 #pragma once
 
 #include <cstdint>
@@ -18,13 +20,22 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kMaxKeys = 96;        // 32 budget classes x 3 keys
 constexpr int kMaxFrontier = 96;    // r <= max_keys - 1 nodes survive a step
 constexpr int kMaxCand = 192;       // a step offers at most 2 r candidates
-constexpr int kCandSlots = kMaxCand / 32;
 constexpr int kFrontSlots = kMaxFrontier / 32;
 constexpr int kWarps = 8;           // queries in flight per CTA
 
+template <int D>
+struct Lay {
+  static constexpr int TPR = D / 16;    // lanes per row in the row-group layout
+  static constexpr int RPI = 32 / TPR;  // rows per warp pass
+  static constexpr int DPL = D / 32;    // dims per lane in the value layout
+};
+
 // Node descriptor: (start << 5) | level; the node covers keys [start, start + 2^level).
+// Bits 29 and 30 are free (start < 2^20) and carry flags in the phase-one row list.
+constexpr int kFlagRoot = 1 << 29;  // the row is a root of the descent forest
+constexpr int kFlagG = 1 << 30;     // the row is a block of the causal sum G_i
 __device__ __forceinline__ int desc_level(int desc) { return desc & 31; }
-__device__ __forceinline__ int desc_start(int desc) { return desc >> 5; }
+__device__ __forceinline__ int desc_start(int desc) { return (desc >> 5) & 0xFFFFF; }
 __device__ __forceinline__ int make_desc(int start, int level) { return (start << 5) | level; }
 
 // First row of tree level `level` (>= 1) in the level-major layout of one (b,h).
@@ -52,41 +63,75 @@ struct QueryArgs {
   uint32_t* dev_err;
 };
 
-// ------------------------------------------------------------------ per-lane row loads
+__device__ __forceinline__ int sx8(int w, int byte) { return (w << (24 - 8 * byte)) >> 24; }
 
-// DPL int8 values of a key row (or a query row) at lane `lane`, sign-extended.
-template <int DPL>
-__device__ __forceinline__ void load_i8(const int8_t* row, int lane, int (&v)[DPL]) {
-  if constexpr (DPL == 2) {
-    const int t = __ldg(reinterpret_cast<const short*>(row) + lane);
-    v[0] = (t << 24) >> 24;
-    v[1] = (t << 16) >> 24;
-  } else {
-    const int t = __ldg(reinterpret_cast<const int*>(row) + lane);
-    v[0] = (t << 24) >> 24;
-    v[1] = (t << 16) >> 24;
-    v[2] = (t << 8) >> 24;
-    v[3] = t >> 24;
+// The query in the row-group layout: packed words (for dp4a on key rows) and the same 16
+// values sign-extended (for tree rows).
+struct RowQ {
+  int qp[4];
+  int qn[16];
+};
+
+template <int D>
+__device__ __forceinline__ void load_rowq(const int8_t* qrow, int sub, RowQ& q) {
+  constexpr int TPR = Lay<D>::TPR;
+  const int* p = reinterpret_cast<const int*>(qrow) + sub;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    q.qp[v] = __ldg(p + TPR * v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) q.qn[4 * v + e] = sx8(q.qp[v], e);
   }
 }
 
-// DPL int32 values of a tree row at lane `lane`.
-template <int DPL>
-__device__ __forceinline__ void load_i32(const int32_t* row, int lane, int (&v)[DPL]) {
-  if constexpr (DPL == 2) {
-    const int2 t = __ldg(reinterpret_cast<const int2*>(row) + lane);
-    v[0] = t.x;
-    v[1] = t.y;
-  } else {
-    const int4 t = __ldg(reinterpret_cast<const int4*>(row) + lane);
-    v[0] = t.x;
-    v[1] = t.y;
-    v[2] = t.z;
-    v[3] = t.w;
+// A tree row (int32) in the row-group layout.
+template <int D>
+__device__ __forceinline__ void ld_tree(const int32_t* row, int sub, int (&x)[16]) {
+  constexpr int TPR = Lay<D>::TPR;
+  const int4* p = reinterpret_cast<const int4*>(row) + sub;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const int4 t = __ldg(p + TPR * v);
+    x[4 * v + 0] = t.x;
+    x[4 * v + 1] = t.y;
+    x[4 * v + 2] = t.z;
+    x[4 * v + 3] = t.w;
   }
 }
 
-// DPL bf16 values of a value row at lane `lane`, as floats (bf16 -> f32 is exact).
+// A key row (int8) in the row-group layout, as packed words.
+template <int D>
+__device__ __forceinline__ void ld_key(const int8_t* row, int sub, int (&xp)[4]) {
+  constexpr int TPR = Lay<D>::TPR;
+  const int* p = reinterpret_cast<const int*>(row) + sub;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) xp[v] = __ldg(p + TPR * v);
+}
+
+template <typename S>
+__device__ __forceinline__ S dot_tree(const RowQ& q, const int (&x)[16]) {
+  S s = 0;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) s += S(q.qn[j]) * S(x[j]);
+  return s;
+}
+
+__device__ __forceinline__ int dot_key(const RowQ& q, const int (&xp)[4]) {
+  int s = 0;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) s = __dp4a(xp[v], q.qp[v], s);
+  return s;
+}
+
+// Sum over the TPR lanes of a row group (every lane of the group gets the sum).
+template <typename S, int TPR>
+__device__ __forceinline__ S group_sum(S s) {
+#pragma unroll
+  for (int off = 1; off < TPR; off *= 2) s += __shfl_xor_sync(kFull, s, off);
+  return s;
+}
+
+// DPL bf16 values of a value row in the value layout, as floats (bf16 -> f32 is exact).
 template <int DPL>
 __device__ __forceinline__ void load_bf16(const uint16_t* row, int lane, float (&v)[DPL]) {
   if constexpr (DPL == 2) {
@@ -102,44 +147,6 @@ __device__ __forceinline__ void load_bf16(const uint16_t* row, int lane, float (
   }
 }
 
-// Row (level, j) of one head: a key row (level 0) or a stored tree sum (level >= 1).
-template <int DPL>
-__device__ __forceinline__ void load_node(const int8_t* Kh, const int32_t* Nh, int n, int level,
-                                          int j, int lane, int (&v)[DPL]) {
-  constexpr int D = 32 * DPL;
-  if (level == 0) {
-    load_i8<DPL>(Kh + (long long)j * D, lane, v);
-  } else {
-    load_i32<DPL>(Nh + (level_row(n, level) + j) * D, lane, v);
-  }
-}
-
-template <typename S, int DPL>
-__device__ __forceinline__ S lane_dot(const int (&q)[DPL], const int (&v)[DPL]) {
-  S s = 0;
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) s += S(q[e]) * S(v[e]);
-  return s;
-}
-
-// Transposed butterfly: lane x returns the warp-wide sum of v[x % R].
-template <typename S, int R>
-__device__ __forceinline__ S transpose_reduce(S (&v)[R], int lane) {
-#pragma unroll
-  for (int h = R / 2; h >= 1; h /= 2) {
-    const bool up = (lane & h) != 0;
-#pragma unroll
-    for (int j = 0; j < h; ++j) {
-      const S keep = up ? v[j + h] : v[j];
-      const S send = up ? v[j] : v[j + h];
-      v[j] = keep + __shfl_xor_sync(kFull, send, h);
-    }
-  }
-#pragma unroll
-  for (int off = R; off < 32; off *= 2) v[0] += __shfl_xor_sync(kFull, v[0], off);
-  return v[0];
-}
-
 template <typename S>
 __device__ __forceinline__ S warp_min(S x) {
 #pragma unroll
@@ -149,6 +156,8 @@ __device__ __forceinline__ S warp_min(S x) {
   }
   return x;
 }
+template <>
+__device__ __forceinline__ int warp_min<int>(int x) { return __reduce_min_sync(kFull, x); }
 
 template <typename S>
 __device__ __forceinline__ S warp_max(S x) {
@@ -159,6 +168,8 @@ __device__ __forceinline__ S warp_max(S x) {
   }
   return x;
 }
+template <>
+__device__ __forceinline__ int warp_max<int>(int x) { return __reduce_max_sync(kFull, x); }
 
 __device__ __forceinline__ float warp_maxf(float x) {
 #pragma unroll
@@ -171,8 +182,6 @@ __device__ __forceinline__ float warp_sumf(float x) {
   for (int off = 16; off >= 1; off /= 2) x += __shfl_xor_sync(kFull, x, off);
   return x;
 }
-
-__device__ __forceinline__ int warp_count(bool p) { return __popc(__ballot_sync(kFull, p)); }
 
 __device__ __forceinline__ unsigned lanemask_lt(int lane) { return (1u << lane) - 1u; }
 
@@ -193,59 +202,58 @@ struct ScoreLimits<long long> {
   static constexpr long long highest = 9223372036854775807LL;
 };
 
-// Per-warp scratch of the descent (shared memory).
+// Per-warp scratch of one query (shared memory).
 template <typename S>
 struct WarpBuf {
-  int cdesc[kMaxCand];
+  int cdesc[kMaxCand];       // frontier / candidates
   S cscore[kMaxCand];
-  int xdesc[kMaxFrontier];
+  int xdesc[kMaxFrontier];   // nodes expanded this step
   S xscore[kMaxFrontier];
+  int plist[32];             // phase-one row list (causal-sum blocks and roots)
+  int winsc[32];             // scores of the window keys
 };
 
 // ------------------------------------------------------------------ top-r selection
 //
-// Keeps, among the C candidates in buf (C > r), the r with the largest score, ties to the lower
-// start, and packs them into buf[0, r). Exact: the r-th largest score T is found by bisection on
-// the integer score, then the candidates tied at T are cut by bisection on their start.
-template <typename S>
-__device__ __forceinline__ void select_top_r(WarpBuf<S>& B, int C, int r, int lane) {
+// Keeps, among the C candidates (r < C <= 32*NS), the r with the largest score, ties to the
+// lower start, and packs them into the front of the buffer. Exact: the r-th largest score T is
+// found by bisection on the integer score; candidates tied at T are then cut by bisection on
+// their start position (starts are distinct).
+template <typename S, int NS>
+__device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int lane) {
   constexpr S kLow = ScoreLimits<S>::lowest;
-  S sc[kCandSlots];
-  int ds[kCandSlots];
-  __syncwarp();
+  S sc[NS];
+  int ds[NS];
 #pragma unroll
-  for (int s = 0; s < kCandSlots; ++s) {
+  for (int s = 0; s < NS; ++s) {
     const int e = lane + 32 * s;
     const bool ok = e < C;
     sc[s] = ok ? B.cscore[e] : kLow;
     ds[s] = ok ? B.cdesc[e] : 0;
   }
-  S lo, hi;
-  {
-    S mn = ScoreLimits<S>::highest, mx = kLow;
+  S mn = ScoreLimits<S>::highest, mx = kLow;
 #pragma unroll
-    for (int s = 0; s < kCandSlots; ++s) {
-      if (sc[s] != kLow) {
-        mn = sc[s] < mn ? sc[s] : mn;
-        mx = sc[s] > mx ? sc[s] : mx;
-      }
+  for (int s = 0; s < NS; ++s) {
+    if (sc[s] != kLow) {
+      mn = sc[s] < mn ? sc[s] : mn;
+      mx = sc[s] > mx ? sc[s] : mx;
     }
-    lo = warp_min<S>(mn);
-    hi = warp_max<S>(mx);
   }
+  S lo = warp_min<S>(mn);
+  S hi = warp_max<S>(mx);
   // largest T with #{score >= T} >= r
   for (int guard = 0; guard < 70 && lo < hi; ++guard) {
     const S mid = S((long long)lo + (((long long)hi - (long long)lo + 1) >> 1));
     int c = 0;
 #pragma unroll
-    for (int s = 0; s < kCandSlots; ++s) c += sc[s] >= mid ? 1 : 0;
+    for (int s = 0; s < NS; ++s) c += sc[s] >= mid ? 1 : 0;
     c = __reduce_add_sync(kFull, c);
     if (c >= r) lo = mid; else hi = mid - 1;
   }
   const S T = lo;
   int gt = 0, eq = 0;
 #pragma unroll
-  for (int s = 0; s < kCandSlots; ++s) {
+  for (int s = 0; s < NS; ++s) {
     gt += sc[s] > T ? 1 : 0;
     eq += sc[s] == T ? 1 : 0;
   }
@@ -255,12 +263,12 @@ __device__ __forceinline__ void select_top_r(WarpBuf<S>& B, int C, int r, int la
   int U = 0x7fffffff;
   if (need < eq) {
     // smallest U with #{score == T and start <= U} >= need
-    int lo2 = 0, hi2 = 0x7fffffff;
-    for (int guard = 0; guard < 34 && lo2 < hi2; ++guard) {
+    int lo2 = 0, hi2 = 1 << 20;
+    for (int guard = 0; guard < 24 && lo2 < hi2; ++guard) {
       const int mid = lo2 + ((hi2 - lo2) >> 1);
       int c = 0;
 #pragma unroll
-      for (int s = 0; s < kCandSlots; ++s) c += (sc[s] == T && desc_start(ds[s]) <= mid) ? 1 : 0;
+      for (int s = 0; s < NS; ++s) c += (sc[s] == T && desc_start(ds[s]) <= mid) ? 1 : 0;
       c = __reduce_add_sync(kFull, c);
       if (c >= need) hi2 = mid; else lo2 = mid + 1;
     }
@@ -269,7 +277,7 @@ __device__ __forceinline__ void select_top_r(WarpBuf<S>& B, int C, int r, int la
   __syncwarp();
   int base = 0;
 #pragma unroll
-  for (int s = 0; s < kCandSlots; ++s) {
+  for (int s = 0; s < NS; ++s) {
     const bool keep = sc[s] != kLow && (sc[s] > T || (sc[s] == T && desc_start(ds[s]) <= U));
     const unsigned bal = __ballot_sync(kFull, keep);
     if (keep) {
@@ -280,6 +288,15 @@ __device__ __forceinline__ void select_top_r(WarpBuf<S>& B, int C, int r, int la
     base += __popc(bal);
   }
   __syncwarp();
+}
+
+template <typename S>
+__device__ __forceinline__ void select_top_r(WarpBuf<S>& B, int C, int r, int lane) {
+  __syncwarp();
+  if (C <= 64) select_top_r_ns<S, 2>(B, C, r, lane);
+  else if (C <= 96) select_top_r_ns<S, 3>(B, C, r, lane);
+  else if (C <= 128) select_top_r_ns<S, 4>(B, C, r, lane);
+  else select_top_r_ns<S, 6>(B, C, r, lane);
 }
 
 }  // namespace alhr

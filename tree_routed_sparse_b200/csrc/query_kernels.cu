@@ -5,17 +5,18 @@
 // window first, then a budget-limited descent of the past-only forest, then exact attention
 // over the selected keys.
 //
-// Per query (one warp):
-//   1. q, the window rows i, i-1, ..., i-w+1 (key rows: scores for attention, and G_i) and the
-//      roots of [0, i-w] (tree rows: first frontier, and G_i) -- G_i = roots + window costs no
-//      extra bytes;
-//   2. budget: predictor logits over 32 classes from W in shared memory (int64, ties -> lower
-//      class), or the given budget;
-//   3. descent: every step reads only the LEFT child of each expanded node; the right child's
-//      score is parent - left (exact in integers), so a step costs one row per expansion;
-//      keep-the-best-r is an exact bisection on the integer score (select_top_r);
-//   4. routed leaves keep the scores computed during the descent, so their key rows are never
-//      read again; attention gathers only the value rows.
+// Per query (one warp, rows scored in row groups, see alhr_device.cuh):
+//   1. causal sum: G_i = sum of keys [0, i] is the sum of the tree rows of the binary
+//      decomposition of [0, i+1). Its largest blocks are also the largest roots of the descent
+//      forest of [0, i-w] (both decompositions share every block above the highest bit where
+//      i+1 and i-w+1 differ), so their scores are taken in the same pass;
+//   2. budget: logits over 32 classes from W in shared memory (int64, ties -> lower class), or
+//      the given budget;
+//   3. the remaining roots, then the descent: each step reads only the LEFT child of every
+//      expanded node (the right child's score is parent - left, exact in integers) and keeps the
+//      best r by an exact integer bisection (select_top_r);
+//   4. attention: the selected window keys are scored, routed keys keep the scores of the
+//      descent (their key rows are not read again), and the value rows are gathered.
 #include <cuda_runtime.h>
 
 #include "alhr_device.cuh"
@@ -25,22 +26,56 @@ namespace alhr {
 
 enum Mode : int { kForwardPredict = 0, kForwardOverride = 1, kRouteOnly = 2, kPredictOnly = 3 };
 
-template <typename S, int DPL, int MODE>
-__global__ void __launch_bounds__(kWarps * 32) query_kernel(const QueryArgs a) {
-  constexpr int D = 32 * DPL;
+// Writes the two children of expanded node x (descriptor pd, score ps; left score `left`).
+template <typename S>
+__device__ __forceinline__ void put_children(WarpBuf<S>& B, int nl, int x, int pd, S ps, S left) {
+  const int cl = desc_level(pd) - 1;
+  const int st = desc_start(pd);
+  B.cdesc[nl + 2 * x] = make_desc(st, cl);
+  B.cscore[nl + 2 * x] = left;
+  B.cdesc[nl + 2 * x + 1] = make_desc(st + (1 << cl), cl);
+  B.cscore[nl + 2 * x + 1] = ps - left;
+}
+
+// Dynamic shared memory of a query kernel: the predictor weights (the G half widened to
+// int32, then the q half as packed int8 words) followed by one WarpBuf per warp.
+template <typename S, int D, int MODE>
+struct QuerySmem {
+  static constexpr bool kUsesW = (MODE == kForwardPredict || MODE == kPredictOnly);
+  static constexpr size_t w_bytes = kUsesW ? size_t(32 * D + 32 * D / 4) * 4 : 0;
+  static constexpr size_t bytes = w_bytes + kWarps * sizeof(WarpBuf<S>);
+};
+
+constexpr int kMinBlocksPerSM = 3;
+
+template <typename S, int D, int MODE>
+__global__ void __launch_bounds__(kWarps * 32, kMinBlocksPerSM) query_kernel(const QueryArgs a) {
+  constexpr int TPR = Lay<D>::TPR;
+  constexpr int RPI = Lay<D>::RPI;
+  constexpr int DPL = Lay<D>::DPL;
+  constexpr int U = 2;  // tree rows per group per pass (loads in flight)
   constexpr bool kUsesW = (MODE == kForwardPredict || MODE == kPredictOnly);
   constexpr bool kDescend = (MODE != kPredictOnly);
   constexpr bool kAttend = (MODE == kForwardPredict || MODE == kForwardOverride);
-  constexpr int RB = (DPL == 2) ? 32 : 16;  // rows per expansion batch (64 registers of rows)
 
-  __shared__ __align__(16) int8_t sW[kUsesW ? 64 * D : 16];
-  __shared__ WarpBuf<S> wbuf[kWarps];
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  int* sWg = reinterpret_cast<int*>(smem_raw);
+  int* sWq = sWg + 32 * D;
+  WarpBuf<S>* wbuf = reinterpret_cast<WarpBuf<S>*>(smem_raw + QuerySmem<S, D, MODE>::w_bytes);
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  const int grp = lane / TPR;
+  const int sub = lane % TPR;
   if constexpr (kUsesW) {
-    for (int k = threadIdx.x; k < 64 * D / 16; k += blockDim.x)
-      reinterpret_cast<int4*>(sW)[k] = __ldg(reinterpret_cast<const int4*>(a.W) + k);
+    for (int k = threadIdx.x; k < 32 * D / 4; k += blockDim.x) {
+      const int c = k / (D / 4), m = k - c * (D / 4);
+      sWq[k] = __ldg(reinterpret_cast<const int*>(a.W + c * 2 * D) + m);
+    }
+    for (int k = threadIdx.x; k < 32 * D; k += blockDim.x) {
+      const int c = k / D, t = k - c * D;
+      sWg[k] = a.W[c * 2 * D + D + t];
+    }
     __syncthreads();
   }
   WarpBuf<S>& B = wbuf[warp];
@@ -48,24 +83,30 @@ __global__ void __launch_bounds__(kWarps * 32) query_kernel(const QueryArgs a) {
   const int w = a.window;
   const long long stride = (long long)gridDim.x * kWarps;
 
-  for (long long g = (long long)blockIdx.x * kWarps + warp; g < a.num_queries; g += stride) {
-    const long long bh = g / a.nq;
-    const int i = a.q_start + int(g - bh * a.nq);
+  for (long long qi = (long long)blockIdx.x * kWarps + warp; qi < a.num_queries; qi += stride) {
+    const long long bh = qi / a.nq;
+    const int i = a.q_start + int(qi - bh * a.nq);
     const int8_t* Kh = a.K + bh * (long long)n * D;
     const int32_t* Nh = a.nodes + bh * (long long)(n - 1) * D;
 
-    int qv[DPL];
-    load_i8<DPL>(a.Q + g * D, lane, qv);
+    RowQ q;
+    load_rowq<D>(a.Q + qi * D, sub, q);
     {
       bool bad = false;
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) bad |= (qv[e] > a.value_bound) | (qv[e] < -a.value_bound);
+      for (int j = 0; j < 16; ++j) bad |= (q.qn[j] > a.value_bound) | (q.qn[j] < -a.value_bound);
       if (__any_sync(kFull, bad) && lane == 0) flag(a.dev_err, ALHR_DEVERR_VALUE_RANGE);
     }
 
     const int nwin = min(w, i + 1);  // keys of the window
     const int M = i - w + 1;         // keys before the window: [0, M)
-    const int nr = M > 0 ? __popc(M) : 0;
+    const unsigned Mu = M > 0 ? unsigned(M) : 0u;
+    const unsigned A = unsigned(i + 1);
+    // highest bit where i+1 and i-w+1 differ; the blocks above it are shared by the causal-sum
+    // decomposition and the descent forest
+    const int p = kUsesW ? (M > 0 ? 31 - __clz(A ^ Mu) : 31) : 31;
+    const unsigned low_mask = p >= 31 ? 0xffffffffu : ((2u << p) - 1u);
+    const int n_common = __popc(Mu & ~low_mask);
 
     int budget = 0, b_eff = 0, nsel_win = 0, r = 0;
     auto settle = [&](int bud) {
@@ -78,201 +119,210 @@ __global__ void __launch_bounds__(kWarps * 32) query_kernel(const QueryArgs a) {
       nsel_win = min(b_eff, nwin);
       r = b_eff - nsel_win;
     };
-    if constexpr (!kUsesW) settle(__ldg(a.budget_in + g));
+    if constexpr (!kUsesW) settle(__ldg(a.budget_in + qi));
 
-    int G[DPL];
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) G[e] = 0;
-
-    // ---- window rows: lane x ends with the score of key i - x. The predictor needs every
-    // window key (G_i); with a given budget only the selected ones are read.
-    S win_score = 0;
-    if constexpr (kUsesW || kAttend) {
-      const int nload = kUsesW ? nwin : nsel_win;
-      for (int c0 = 0; c0 < nload; c0 += 16) {
-        int v[16][DPL];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          if (c0 + k < nload) {
-            load_i8<DPL>(Kh + (long long)(i - c0 - k) * D, lane, v[k]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) v[k][e] = 0;
-          }
-        }
-        S part[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          part[k] = lane_dot<S, DPL>(qv, v[k]);
-          if constexpr (kUsesW) {
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) G[e] += v[k][e];
-          }
-        }
-        const S res = transpose_reduce<S, 16>(part, lane);
-        if ((lane >> 4) == (c0 >> 4)) win_score = res;
-      }
-    }
-
-    // ---- roots of [0, M), largest first: lane k ends with root k
-    S root_score = 0;
-    int root_desc = 0;
-    const bool load_roots = kUsesW || (r > 0 && M > 0);
-    if (load_roots) {
-      int rest = M;
-      for (int c0 = 0; c0 < nr; c0 += 16) {
-        int v[16][DPL];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          if (c0 + k < nr) {
-            const int lvl = 31 - __clz(rest);
-            rest ^= 1 << lvl;
-            const int start = M & ~((2 << lvl) - 1);
-            if (lane == c0 + k) root_desc = make_desc(start, lvl);
-            load_node<DPL>(Kh, Nh, n, lvl, start >> lvl, lane, v[k]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) v[k][e] = 0;
-          }
-        }
-        S part[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          part[k] = lane_dot<S, DPL>(qv, v[k]);
-          if constexpr (kUsesW) {
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) G[e] += v[k][e];
-          }
-        }
-        const S res = transpose_reduce<S, 16>(part, lane);
-        if ((lane >> 4) == (c0 >> 4)) root_score = res;
-      }
-    }
-
-    // ---- budget predictor: logit_c = W[c][:d] . q + W[c][d:] . G_i, argmax, ties -> lower c
+    // ---- 1. causal sum G_i over the blocks of [0, i+1) (and the shared roots' scores)
     if constexpr (kUsesW) {
-      long long logit = 0;
+      int G[16];
 #pragma unroll
-      for (int c0 = 0; c0 < 32; c0 += 16) {
-        long long part[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int8_t* wr = sW + (c0 + k) * 2 * D;
-          int wq[DPL], wg[DPL];
-          if constexpr (DPL == 2) {
-            const int tq = reinterpret_cast<const short*>(wr)[lane];
-            const int tg = reinterpret_cast<const short*>(wr + D)[lane];
-            wq[0] = (tq << 24) >> 24; wq[1] = (tq << 16) >> 24;
-            wg[0] = (tg << 24) >> 24; wg[1] = (tg << 16) >> 24;
-          } else {
-            const int tq = reinterpret_cast<const int*>(wr)[lane];
-            const int tg = reinterpret_cast<const int*>(wr + D)[lane];
-            wq[0] = (tq << 24) >> 24; wq[1] = (tq << 16) >> 24;
-            wq[2] = (tq << 8) >> 24;  wq[3] = tq >> 24;
-            wg[0] = (tg << 24) >> 24; wg[1] = (tg << 16) >> 24;
-            wg[2] = (tg << 8) >> 24;  wg[3] = tg >> 24;
-          }
-          long long s = 0;
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) s += (long long)(wq[e] * qv[e]) + (long long)wg[e] * G[e];
-          part[k] = s;
-        }
-        const long long res = transpose_reduce<long long, 16>(part, lane);
-        if ((lane >> 4) == (c0 >> 4)) logit = res;
+      for (int j = 0; j < 16; ++j) G[j] = 0;
+      const int nA = __popc(A);
+      __syncwarp();
+      if ((A >> lane) & 1u) {
+        const int b = lane;
+        const int rank = __popc(A >> b) - 1;
+        const int start = int((A >> b) << b) - (1 << b);
+        B.plist[rank] = make_desc(start, b) | kFlagG | ((M > 0 && b > p) ? kFlagRoot : 0);
       }
-      // largest logit, then lowest class: pack (logit, 31 - class) and take the maximum
-      const long long key = warp_max<long long>(logit * 32 + (31 - lane));
-      const int cls = 31 - int(key & 31);
-      settle(3 * (cls + 1));
+      __syncwarp();
+      for (int base = 0; base < nA; base += RPI) {
+        const int k = base + grp;
+        const bool active = k < nA;
+        const int pd = active ? B.plist[k] : 0;
+        const int lvl = desc_level(pd);
+        const int st = desc_start(pd);
+        S sc = 0;
+        if (active) {
+          if (lvl > 0) {
+            int x[16];
+            ld_tree<D>(Nh + (level_row(n, lvl) + (st >> lvl)) * D, sub, x);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) G[j] += x[j];
+            sc = dot_tree<S>(q, x);
+          } else {
+            int xp[4];
+            ld_key<D>(Kh + (long long)st * D, sub, xp);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) G[4 * v + e] += sx8(xp[v], e);
+            sc = S(dot_key(q, xp));
+          }
+        }
+        sc = group_sum<S, TPR>(sc);
+        if (active && sub == 0 && (pd & kFlagRoot)) {
+          B.cdesc[k] = pd & ~(kFlagRoot | kFlagG);  // common roots are the first ones
+          B.cscore[k] = sc;
+        }
+      }
+#pragma unroll
+      for (int off = TPR; off < 32; off *= 2)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) G[j] += __shfl_xor_sync(kFull, G[j], off);
+
+      // ---- 2. budget predictor: group grp scores classes grp, grp+RPI, ...
+      long long best = ScoreLimits<long long>::lowest;
+#pragma unroll
+      for (int k = 0; k < 32 / RPI; ++k) {
+        const int c = grp + RPI * k;
+        int sq = 0;
+        long long sg = 0;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int m = sub + TPR * v;  // word index of dims 4m .. 4m+3
+          sq = __dp4a(sWq[c * (D / 4) + m], q.qp[v], sq);
+          const int4 wg = *reinterpret_cast<const int4*>(sWg + c * D + 4 * m);
+          sg += (long long)wg.x * G[4 * v] + (long long)wg.y * G[4 * v + 1] +
+                (long long)wg.z * G[4 * v + 2] + (long long)wg.w * G[4 * v + 3];
+        }
+        const long long logit = group_sum<long long, TPR>(sg + sq);
+        // largest logit, then lowest class: pack (logit, 31 - class)
+        const long long key = logit * 32 + (31 - c);
+        best = key > best ? key : best;
+      }
+#pragma unroll
+      for (int off = TPR; off < 32; off *= 2) {
+        const long long o = __shfl_xor_sync(kFull, best, off);
+        best = o > best ? o : best;
+      }
+      settle(3 * (31 - int(best & 31) + 1));
     }
 
     if constexpr (MODE == kPredictOnly) {
-      if (lane == 0) a.budget_out[g] = budget;
+      if (lane == 0) a.budget_out[qi] = budget;
       continue;
     }
 
-    // ---- descent of the past-only forest
+    // ---- 3. descent of the past-only forest
     int nf = 0, exp_hi = 0, exp_l1 = 0;
-    if (kDescend && r > 0 && M > 0) {
+    if (kDescend && r > 0) {  // r > 0 implies i >= w, i.e. M > 0
+      // roots not yet scored: the blocks of [0, M) below the shared ones
+      const unsigned rest = Mu & low_mask;
+      const int nB = __popc(rest);
       __syncwarp();
-      if (lane < nr) {
-        B.cdesc[lane] = root_desc;
-        B.cscore[lane] = root_score;
+      if ((rest >> lane) & 1u) {
+        const int b = lane;
+        B.plist[__popc(rest >> b) - 1] = make_desc(int((Mu >> b) << b) - (1 << b), b);
       }
-      nf = nr;
+      __syncwarp();
+      for (int base = 0; base < nB; base += RPI) {
+        const int k = base + grp;
+        const bool active = k < nB;
+        const int pd = active ? B.plist[k] : 0;
+        const int lvl = desc_level(pd);
+        const int st = desc_start(pd);
+        S sc = 0;
+        if (active) {
+          if (lvl > 0) {
+            int x[16];
+            ld_tree<D>(Nh + (level_row(n, lvl) + (st >> lvl)) * D, sub, x);
+            sc = dot_tree<S>(q, x);
+          } else {
+            int xp[4];
+            ld_key<D>(Kh + (long long)st * D, sub, xp);
+            sc = S(dot_key(q, xp));
+          }
+        }
+        sc = group_sum<S, TPR>(sc);
+        if (active && sub == 0) {
+          B.cdesc[n_common + k] = pd;
+          B.cscore[n_common + k] = sc;
+        }
+      }
+      nf = __popc(Mu);
+
       for (int step = 0; step < 32; ++step) {
         __syncwarp();
         int fd[kFrontSlots];
         S fs[kFrontSlots];
-        bool inner[kFrontSlots], leaf[kFrontSlots];
-        int nx = 0, nl = 0, nhi = 0;
-        unsigned bi[kFrontSlots], bl[kFrontSlots];
+        bool hi[kFrontSlots], l1[kFrontSlots], leaf[kFrontSlots];
+        unsigned bh_[kFrontSlots], b1_[kFrontSlots], bl_[kFrontSlots];
+        int nhi = 0, nl1 = 0, nl = 0;
 #pragma unroll
         for (int s = 0; s < kFrontSlots; ++s) {
           const int e = lane + 32 * s;
           const bool ok = e < nf;
           fd[s] = ok ? B.cdesc[e] : 0;
           fs[s] = ok ? B.cscore[e] : S(0);
-          inner[s] = ok && desc_level(fd[s]) > 0;
-          leaf[s] = ok && !inner[s];
-          bi[s] = __ballot_sync(kFull, inner[s]);
-          bl[s] = __ballot_sync(kFull, leaf[s]);
-          nx += __popc(bi[s]);
-          nl += __popc(bl[s]);
-          nhi += warp_count(inner[s] && desc_level(fd[s]) >= 2);
+          const int lv = desc_level(fd[s]);
+          hi[s] = ok && lv >= 2;
+          l1[s] = ok && lv == 1;
+          leaf[s] = ok && lv == 0;
+          bh_[s] = __ballot_sync(kFull, hi[s]);
+          b1_[s] = __ballot_sync(kFull, l1[s]);
+          bl_[s] = __ballot_sync(kFull, leaf[s]);
+          nhi += __popc(bh_[s]);
+          nl1 += __popc(b1_[s]);
+          nl += __popc(bl_[s]);
         }
+        const int nx = nhi + nl1;
         if (nx == 0) break;
         exp_hi += nhi;
-        exp_l1 += nx - nhi;
+        exp_l1 += nl1;
         __syncwarp();
         {
-          int xo = 0, lo = 0;
+          const unsigned below = lanemask_lt(lane);
+          int oh = 0, o1 = nhi, ol = 0;
 #pragma unroll
           for (int s = 0; s < kFrontSlots; ++s) {
-            const unsigned below = lanemask_lt(lane);
-            if (inner[s]) {
-              const int pos = xo + __popc(bi[s] & below);
+            if (hi[s] || l1[s]) {
+              const int pos = hi[s] ? oh + __popc(bh_[s] & below) : o1 + __popc(b1_[s] & below);
               B.xdesc[pos] = fd[s];
               B.xscore[pos] = fs[s];
             }
             if (leaf[s]) {
-              const int pos = lo + __popc(bl[s] & below);
+              const int pos = ol + __popc(bl_[s] & below);
               B.cdesc[pos] = fd[s];
               B.cscore[pos] = fs[s];
             }
-            xo += __popc(bi[s]);
-            lo += __popc(bl[s]);
+            oh += __popc(bh_[s]);
+            o1 += __popc(b1_[s]);
+            ol += __popc(bl_[s]);
           }
         }
         __syncwarp();
-        for (int base = 0; base < nx; base += RB) {
-          int v[RB][DPL];
+        // left children that are tree rows: U rows per group in flight
+        for (int base = 0; base < nhi; base += U * RPI) {
+          int x[U][16];
+          int pd[U];
 #pragma unroll
-          for (int k = 0; k < RB; ++k) {
-            if (base + k < nx) {
-              const int pd = B.xdesc[base + k];
-              const int cl = desc_level(pd) - 1;
-              load_node<DPL>(Kh, Nh, n, cl, desc_start(pd) >> cl, lane, v[k]);
+          for (int u = 0; u < U; ++u) {
+            const int xi = base + u * RPI + grp;
+            pd[u] = xi < nhi ? B.xdesc[xi] : 0;
+            if (xi < nhi) {
+              const int cl = desc_level(pd[u]) - 1;
+              ld_tree<D>(Nh + (level_row(n, cl) + (desc_start(pd[u]) >> cl)) * D, sub, x[u]);
             } else {
 #pragma unroll
-              for (int e = 0; e < DPL; ++e) v[k][e] = 0;
+              for (int j = 0; j < 16; ++j) x[u][j] = 0;
             }
           }
-          S part[RB];
 #pragma unroll
-          for (int k = 0; k < RB; ++k) part[k] = lane_dot<S, DPL>(qv, v[k]);
-          const S left = transpose_reduce<S, RB>(part, lane);
-          const int x = base + lane;
-          if (lane < RB && x < nx) {
-            const int pd = B.xdesc[x];
-            const S ps = B.xscore[x];
-            const int cl = desc_level(pd) - 1;
-            const int st = desc_start(pd);
-            B.cdesc[nl + 2 * x] = make_desc(st, cl);
-            B.cscore[nl + 2 * x] = left;
-            B.cdesc[nl + 2 * x + 1] = make_desc(st + (1 << cl), cl);
-            B.cscore[nl + 2 * x + 1] = ps - left;
+          for (int u = 0; u < U; ++u) {
+            const int xi = base + u * RPI + grp;
+            const S left = group_sum<S, TPR>(dot_tree<S>(q, x[u]));
+            if (xi < nhi && sub == 0) put_children<S>(B, nl, xi, pd[u], B.xscore[xi], left);
           }
+        }
+        // left children that are keys
+        for (int base = nhi; base < nx; base += RPI) {
+          const int xi = base + grp;
+          const bool active = xi < nx;
+          const int pd = active ? B.xdesc[xi] : 0;
+          int xp[4] = {0, 0, 0, 0};
+          if (active) ld_key<D>(Kh + (long long)desc_start(pd) * D, sub, xp);
+          const S left = S(group_sum<int, TPR>(dot_key(q, xp)));
+          if (active && sub == 0) put_children<S>(B, nl, xi, pd, B.xscore[xi], left);
         }
         const int C = nl + 2 * nx;
         if (C > r) {
@@ -280,22 +330,32 @@ __global__ void __launch_bounds__(kWarps * 32) query_kernel(const QueryArgs a) {
           nf = r;
         } else {
           nf = C;
-          __syncwarp();
         }
+      }
+    }
+
+    // ---- window key scores (attention only needs the selected ones)
+    if constexpr (kAttend) {
+      for (int base = 0; base < nsel_win; base += RPI) {
+        const int x = base + grp;
+        int xp[4] = {0, 0, 0, 0};
+        if (x < nsel_win) ld_key<D>(Kh + (long long)(i - x) * D, sub, xp);
+        const int s = group_sum<int, TPR>(dot_key(q, xp));
+        if (x < nsel_win && sub == 0) B.winsc[x] = s;
       }
     }
     __syncwarp();
 
     // ---- optional outputs of the route
     const int count = nsel_win + nf;
-    if (a.count_out && lane == 0) a.count_out[g] = count;
+    if (a.count_out && lane == 0) a.count_out[qi] = count;
     if (a.exp_out && lane == 0) {
-      a.exp_out[2 * g] = exp_hi;
-      a.exp_out[2 * g + 1] = exp_l1;
+      a.exp_out[2 * qi] = exp_hi;
+      a.exp_out[2 * qi + 1] = exp_l1;
     }
-    if (a.budget_out && lane == 0) a.budget_out[g] = budget;
+    if (a.budget_out && lane == 0) a.budget_out[qi] = budget;
     if (a.idx_out) {
-      int32_t* io = a.idx_out + g * a.max_keys;
+      int32_t* io = a.idx_out + qi * a.max_keys;
 #pragma unroll
       for (int s = 0; s < kFrontSlots; ++s) {
         const int e = lane + 32 * s;
@@ -307,13 +367,13 @@ __global__ void __launch_bounds__(kWarps * 32) query_kernel(const QueryArgs a) {
         }
       }
       if (lane < nsel_win) io[nf + nsel_win - 1 - lane] = i - lane;
-      for (int p = count + lane; p < a.max_keys; p += 32) io[p] = -1;
+      for (int pp = count + lane; pp < a.max_keys; pp += 32) io[pp] = -1;
     }
 
-    // ---- exact attention over window + routed keys
+    // ---- 4. exact attention over window + routed keys
     if constexpr (kAttend) {
       const float scale = a.scale;
-      const float sw = lane < nsel_win ? float(win_score) * scale : -INFINITY;
+      const float sw = lane < nsel_win ? float(B.winsc[lane]) * scale : -INFINITY;
       float sr[kFrontSlots];
       int kr[kFrontSlots];
 #pragma unroll
@@ -361,7 +421,7 @@ __global__ void __launch_bounds__(kWarps * 32) query_kernel(const QueryArgs a) {
         }
       }
       const float inv = 1.f / den;
-      float* o = a.out + g * D + lane * DPL;
+      float* o = a.out + qi * D + lane * DPL;
       if constexpr (DPL == 2) {
         *reinterpret_cast<float2*>(o) = make_float2(acc[0] * inv, acc[1] * inv);
       } else {
@@ -372,64 +432,56 @@ __global__ void __launch_bounds__(kWarps * 32) query_kernel(const QueryArgs a) {
   }
 }
 
-// Exact attention over a given selection (idx, count): key rows for the scores, value rows for
-// the sum. Entries outside [0, i] are skipped and flagged.
-template <int DPL>
+// Exact attention over a given selection (idx, count): key rows for the scores (row groups),
+// value rows for the sum. Entries outside [0, i] are skipped and flagged.
+template <int D>
 __global__ void __launch_bounds__(kWarps * 32) attend_kernel(const QueryArgs a) {
-  constexpr int D = 32 * DPL;
-  constexpr int RB = (DPL == 2) ? 32 : 16;
+  constexpr int TPR = Lay<D>::TPR;
+  constexpr int RPI = Lay<D>::RPI;
+  constexpr int DPL = Lay<D>::DPL;
+  __shared__ WarpBuf<int> wbuf[kWarps];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  const int grp = lane / TPR;
+  const int sub = lane % TPR;
+  WarpBuf<int>& B = wbuf[warp];
   const int n = a.n;
   const long long stride = (long long)gridDim.x * kWarps;
-  for (long long g = (long long)blockIdx.x * kWarps + warp; g < a.num_queries; g += stride) {
-    const long long bh = g / a.nq;
-    const int i = a.q_start + int(g - bh * a.nq);
+  for (long long qi = (long long)blockIdx.x * kWarps + warp; qi < a.num_queries; qi += stride) {
+    const long long bh = qi / a.nq;
+    const int i = a.q_start + int(qi - bh * a.nq);
     const int8_t* Kh = a.K + bh * (long long)n * D;
     const uint16_t* Vh = a.V + bh * (long long)n * D;
-    int qv[DPL];
-    load_i8<DPL>(a.Q + g * D, lane, qv);
-    const int cnt = min(__ldg(a.count_in + g), a.max_keys);
-    float* o = a.out + g * D + lane * DPL;
+    RowQ q;
+    load_rowq<D>(a.Q + qi * D, sub, q);
+    const int cnt = max(0, min(__ldg(a.count_in + qi), a.max_keys));
     int key[kFrontSlots];
     bool ok[kFrontSlots];
     bool bad = false;
+    __syncwarp();
 #pragma unroll
     for (int s = 0; s < kFrontSlots; ++s) {
       const int e = lane + 32 * s;
-      key[s] = e < cnt ? __ldg(a.idx_in + g * a.max_keys + e) : -1;
+      key[s] = e < cnt ? __ldg(a.idx_in + qi * a.max_keys + e) : -1;
       ok[s] = e < cnt && key[s] >= 0 && key[s] <= i;
       bad |= e < cnt && !ok[s];
+      if (e < cnt) B.cdesc[e] = ok[s] ? key[s] : -1;
     }
     if (__any_sync(kFull, bad) && lane == 0) flag(a.dev_err, ALHR_DEVERR_INDEX);
+    __syncwarp();
+    for (int base = 0; base < cnt; base += RPI) {
+      const int x = base + grp;
+      const int kk = x < cnt ? B.cdesc[x] : -1;
+      int xp[4] = {0, 0, 0, 0};
+      if (kk >= 0) ld_key<D>(Kh + (long long)kk * D, sub, xp);
+      const int s = group_sum<int, TPR>(dot_key(q, xp));
+      if (x < cnt && sub == 0) B.cscore[x] = s;
+    }
+    __syncwarp();
     float sc[kFrontSlots];
 #pragma unroll
-    for (int s = 0; s < kFrontSlots; ++s) {
-      sc[s] = -INFINITY;
-#pragma unroll
-      for (int h = 0; h < 32 / RB; ++h) {
-        const int base = 32 * s + RB * h;
-        if (base < cnt) {
-          int v[RB][DPL];
-#pragma unroll
-          for (int k = 0; k < RB; ++k) {
-            const int kk = __shfl_sync(kFull, key[s], RB * h + k);
-            const bool okk = __shfl_sync(kFull, ok[s], RB * h + k);
-            if (okk) {
-              load_i8<DPL>(Kh + (long long)kk * D, lane, v[k]);
-            } else {
-#pragma unroll
-              for (int e = 0; e < DPL; ++e) v[k][e] = 0;
-            }
-          }
-          int part[RB];
-#pragma unroll
-          for (int k = 0; k < RB; ++k) part[k] = lane_dot<int, DPL>(qv, v[k]);
-          const int res = transpose_reduce<int, RB>(part, lane);
-          if (lane / RB == h && ok[s]) sc[s] = float(res) * a.scale;
-        }
-      }
-    }
+    for (int s = 0; s < kFrontSlots; ++s)
+      sc[s] = ok[s] ? float(B.cscore[lane + 32 * s]) * a.scale : -INFINITY;
     float m = -INFINITY;
 #pragma unroll
     for (int s = 0; s < kFrontSlots; ++s) m = fmaxf(m, sc[s]);
@@ -461,6 +513,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(const QueryArgs a) 
       }
     }
     const float inv = den > 0.f ? 1.f / den : 0.f;
+    float* o = a.out + qi * D + lane * DPL;
     if constexpr (DPL == 2) {
       *reinterpret_cast<float2*>(o) = make_float2(acc[0] * inv, acc[1] * inv);
     } else {
@@ -474,51 +527,60 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(const QueryArgs a) 
 
 namespace {
 
-struct Occ {
-  int sms = 0;
-  int per_sm[20] = {0};
-};
+constexpr int kOccSlots = 20;
 
+// Grid size of a persistent launch: the resident CTAs of every SM, capped by the work. The
+// per-device occupancy (and the opt-in to more than 48 KB of dynamic shared memory) is
+// computed once per device and kernel.
 template <typename KernelT>
-int blocks_for(KernelT kernel, int slot, long long queries) {
+int blocks_for(KernelT kernel, int slot, size_t smem, long long queries, cudaError_t* err) {
   static thread_local int cached_dev = -1;
-  static thread_local Occ occ;
+  static thread_local int sms = 0;
+  static thread_local int per_sm[kOccSlots] = {0};
+  *err = cudaSuccess;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev != cached_dev) {
-    occ = Occ{};
-    cudaDeviceGetAttribute(&occ.sms, cudaDevAttrMultiProcessorCount, dev);
+    for (int k = 0; k < kOccSlots; ++k) per_sm[k] = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     cached_dev = dev;
   }
-  if (occ.per_sm[slot] == 0) {
+  if (per_sm[slot] == 0) {
+    if (smem > 48 * 1024) {
+      *err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      if (*err != cudaSuccess) return 0;
+    }
     int b = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, kWarps * 32, 0);
-    occ.per_sm[slot] = b > 0 ? b : 1;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, kWarps * 32, smem);
+    per_sm[slot] = b > 0 ? b : 1;
   }
   const long long need = (queries + kWarps - 1) / kWarps;
-  const long long cap = (long long)occ.sms * occ.per_sm[slot];
+  const long long cap = (long long)sms * per_sm[slot];
   return int(need < cap ? need : cap);
 }
 
-template <typename S, int DPL, int MODE>
+template <typename S, int D, int MODE>
 cudaError_t launch_query(const QueryArgs& a, cudaStream_t st) {
-  constexpr int slot = (MODE * 2 + (DPL == 4 ? 1 : 0)) * 2 + (sizeof(S) == 8 ? 1 : 0);
+  constexpr int slot = (MODE * 2 + (D == 128 ? 1 : 0)) * 2 + (sizeof(S) == 8 ? 1 : 0);
   static_assert(slot < 16, "occupancy cache slot");
-  auto kern = query_kernel<S, DPL, MODE>;
-  const int blocks = blocks_for(kern, slot, a.num_queries);
+  constexpr size_t smem = QuerySmem<S, D, MODE>::bytes;
+  auto kern = query_kernel<S, D, MODE>;
+  cudaError_t err;
+  const int blocks = blocks_for(kern, slot, smem, a.num_queries, &err);
+  if (err != cudaSuccess) return err;
   if (blocks <= 0) return cudaSuccess;
-  kern<<<blocks, kWarps * 32, 0, st>>>(a);
+  kern<<<blocks, kWarps * 32, smem, st>>>(a);
   return cudaGetLastError();
 }
 
 template <int MODE>
 cudaError_t dispatch_query(const QueryArgs& a, int d, int score_bits, cudaStream_t st) {
   if (d == 64) {
-    return score_bits == 32 ? launch_query<int, 2, MODE>(a, st)
-                            : launch_query<long long, 2, MODE>(a, st);
+    return score_bits == 32 ? launch_query<int, 64, MODE>(a, st)
+                            : launch_query<long long, 64, MODE>(a, st);
   }
-  return score_bits == 32 ? launch_query<int, 4, MODE>(a, st)
-                          : launch_query<long long, 4, MODE>(a, st);
+  return score_bits == 32 ? launch_query<int, 128, MODE>(a, st)
+                          : launch_query<long long, 128, MODE>(a, st);
 }
 
 }  // namespace
@@ -538,12 +600,15 @@ cudaError_t launch_predict(const QueryArgs& a, int d, int score_bits, cudaStream
 }
 
 cudaError_t launch_attend(const QueryArgs& a, int d, cudaStream_t st) {
+  cudaError_t err;
   if (d == 64) {
-    const int blocks = blocks_for(attend_kernel<2>, 16, a.num_queries);
-    attend_kernel<2><<<blocks, kWarps * 32, 0, st>>>(a);
+    const int blocks = blocks_for(attend_kernel<64>, 16, 0, a.num_queries, &err);
+    if (err != cudaSuccess) return err;
+    attend_kernel<64><<<blocks, kWarps * 32, 0, st>>>(a);
   } else {
-    const int blocks = blocks_for(attend_kernel<4>, 17, a.num_queries);
-    attend_kernel<4><<<blocks, kWarps * 32, 0, st>>>(a);
+    const int blocks = blocks_for(attend_kernel<128>, 17, 0, a.num_queries, &err);
+    if (err != cudaSuccess) return err;
+    attend_kernel<128><<<blocks, kWarps * 32, 0, st>>>(a);
   }
   return cudaGetLastError();
 }

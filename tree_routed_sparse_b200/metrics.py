@@ -1,33 +1,41 @@
 """Algorithmic byte model of the ALHR inference path (what the algorithm must touch).
 
-Per query of the fused forward (one (b,h) with head dimension d, window w):
-  q row                     d bytes
-  window key rows           nwin * d, nwin = min(w, i+1) with the predictor (G_i needs them
-                            all), else the selected window keys only
-  roots of [0, i-w]         4d per tree root, d for a key root; read with the predictor (G_i)
-                            or when the descent runs
-  descent                   exp_hi * 4d + exp_l1 * d: one left-child row per expansion (the
-                            right child's score is parent - left)
-  value rows                count * 2d (bf16)
-  output row                4d (fp32)
-plus the predictor weights 64 d once per launch. Routed keys' score rows are not re-read.
-The tree build touches K once and writes every tree row once: n d + (n-1) 4d per (b,h).
-These counts come from the run's own outputs (count, expansions), which match the oracle's
-bit for bit, so the byte total is exact for the run.
+Per query at position i of the fused forward (head dimension d, window w, M = i - w + 1 keys
+before the window, rowB(level) = d for a key row and 4d for a tree row):
+  q row                         d
+  causal sum G_i (predictor)    the tree rows of the binary decomposition of [0, i+1)
+  remaining descent roots       the blocks of [0, M) not shared with that decomposition (all of
+                                them without the predictor), only when the descent runs (r > 0)
+  selected window keys          nsel_win * d
+  descent                       exp_hi * 4d + exp_l1 * d: one left-child row per expansion (the
+                                right child's score is parent - left)
+  value rows                    count * 2d (bf16)
+  output row                    4d (fp32)
+plus the predictor weights (64 d) once per launch. Routed keys' rows are not re-read.
+The tree build reads K once and writes every tree row once: n d + (n-1) 4d per (b,h).
+The counts come from the run's own outputs (count, expansions, budget), which match the
+oracle's bit for bit, so the byte total is exact for the run.
 """
 from __future__ import annotations
 
 import numpy as np
 
 
-def root_row_bytes(m: np.ndarray, d: int) -> np.ndarray:
-    """Bytes of the roots of [0, m) for each m (0 where m <= 0)."""
-    m = np.maximum(np.asarray(m, dtype=np.int64), 0)
-    total = np.zeros_like(m)
+def _rows_bytes(bits: np.ndarray, d: int) -> np.ndarray:
+    """Sum of rowB over the set bits of each value (bit b = a block of level b)."""
+    bits = np.asarray(bits, dtype=np.int64)
+    total = np.zeros_like(bits)
     for b in range(0, 40):
-        bit = (m >> b) & 1
-        total += bit * (d if b == 0 else 4 * d)
+        total += ((bits >> b) & 1) * (d if b == 0 else 4 * d)
     return total
+
+
+def _highest_bit(x: np.ndarray) -> np.ndarray:
+    x = np.asarray(x, dtype=np.int64)
+    out = np.full(x.shape, -1, dtype=np.int64)
+    for b in range(0, 40):
+        out = np.where((x >> b) & 1, b, out)
+    return out
 
 
 def forward_bytes(positions, d: int, window: int, count, expansions, budget,
@@ -43,12 +51,18 @@ def forward_bytes(positions, d: int, window: int, count, expansions, budget,
     b_eff = np.minimum(np.minimum(np.maximum(budget, 1), i + 1), max_keys)
     nsel_win = np.minimum(b_eff, nwin)
     r = b_eff - nsel_win
-    m = i - window + 1
-    win_rows = nwin if predictor else nsel_win
-    roots = root_row_bytes(m, d)
-    if not predictor:
-        roots = np.where(r > 0, roots, 0)
-    per_q = (d + win_rows * d + roots + exp[:, 0] * 4 * d + exp[:, 1] * d
+    A = i + 1
+    M = np.maximum(i - window + 1, 0)
+    if predictor:
+        p = np.where(M > 0, _highest_bit(A ^ M), 62)
+        low = (np.int64(2) << np.minimum(p, 61)) - 1
+        g_rows = _rows_bytes(A, d)
+        rest = M & low
+    else:
+        g_rows = np.zeros_like(i)
+        rest = M
+    root_rows = np.where(r > 0, _rows_bytes(rest, d), 0)
+    per_q = (d + g_rows + root_rows + nsel_win * d + exp[:, 0] * 4 * d + exp[:, 1] * d
              + count * 2 * d + 4 * d)
     return int(per_q.sum()) + (64 * d if predictor else 0)
 
