@@ -241,27 +241,39 @@ __device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int
   }
   S lo = warp_min<S>(mn);
   S hi = warp_max<S>(mx);
-  // largest T with #{score >= T} >= r
+  // Bisection for the largest T with #{score >= T} >= r. It stops as soon as a midpoint has
+  // exactly r candidates at or above it: that set is the top r (nothing at or above the
+  // midpoint is left out, so no tie can straddle the cut), which takes about log2(C) probes
+  // instead of log2(score range).
+  bool exact = false;
   for (int guard = 0; guard < 70 && lo < hi; ++guard) {
     const S mid = S((long long)lo + (((long long)hi - (long long)lo + 1) >> 1));
     int c = 0;
 #pragma unroll
     for (int s = 0; s < NS; ++s) c += sc[s] >= mid ? 1 : 0;
     c = __reduce_add_sync(kFull, c);
-    if (c >= r) lo = mid; else hi = mid - 1;
+    if (c == r) {
+      lo = mid;
+      exact = true;
+      break;
+    }
+    if (c > r) lo = mid; else hi = mid - 1;
   }
   const S T = lo;
-  int gt = 0, eq = 0;
+  int need = 0, eq = 0;
+  if (!exact) {
+    int gt = 0;
 #pragma unroll
-  for (int s = 0; s < NS; ++s) {
-    gt += sc[s] > T ? 1 : 0;
-    eq += sc[s] == T ? 1 : 0;
+    for (int s = 0; s < NS; ++s) {
+      gt += sc[s] > T ? 1 : 0;
+      eq += sc[s] == T ? 1 : 0;
+    }
+    gt = __reduce_add_sync(kFull, gt);
+    eq = __reduce_add_sync(kFull, eq);
+    need = r - gt;
   }
-  gt = __reduce_add_sync(kFull, gt);
-  eq = __reduce_add_sync(kFull, eq);
-  const int need = r - gt;
   int U = 0x7fffffff;
-  if (need < eq) {
+  if (!exact && need < eq) {
     // smallest U with #{score == T and start <= U} >= need
     int lo2 = 0, hi2 = 1 << 20;
     for (int guard = 0; guard < 24 && lo2 < hi2; ++guard) {

@@ -38,29 +38,43 @@ __device__ __forceinline__ void put_children(WarpBuf<S>& B, int nl, int x, int p
 }
 
 // Dynamic shared memory of a query kernel: the predictor weights (the G half widened to
-// int32, then the q half as packed int8 words) followed by one WarpBuf per warp.
+// int32, then the q half as packed int8 words; rows padded so that the row groups, which read
+// different classes at once, hit different banks) followed by one WarpBuf per warp.
+template <int D>
+struct WLayout {
+  static constexpr int g_stride = D + 16;     // ints per class row of the G half
+  static constexpr int q_stride = D / 4 + 4;  // words per class row of the q half
+};
 template <typename S, int D, int MODE>
 struct QuerySmem {
   static constexpr bool kUsesW = (MODE == kForwardPredict || MODE == kPredictOnly);
-  static constexpr size_t w_bytes = kUsesW ? size_t(32 * D + 32 * D / 4) * 4 : 0;
+  static constexpr size_t w_bytes =
+      kUsesW ? size_t(32 * WLayout<D>::g_stride + 32 * WLayout<D>::q_stride) * 4 : 0;
   static constexpr size_t bytes = w_bytes + kWarps * sizeof(WarpBuf<S>);
 };
 
-constexpr int kMinBlocksPerSM = 3;
+// Register budget: int32 scores keep three CTAs (24 warps) per SM with two tree rows in flight
+// per row group; int64 scores need more registers, so two CTAs and one row in flight.
+template <typename S>
+constexpr int min_blocks_per_sm() { return sizeof(S) == 4 ? 3 : 2; }
+template <typename S, int D>
+constexpr int tree_rows_in_flight() { return (sizeof(S) == 4 && D == 64) ? 2 : 1; }
 
 template <typename S, int D, int MODE>
-__global__ void __launch_bounds__(kWarps * 32, kMinBlocksPerSM) query_kernel(const QueryArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_kernel(const QueryArgs a) {
   constexpr int TPR = Lay<D>::TPR;
   constexpr int RPI = Lay<D>::RPI;
   constexpr int DPL = Lay<D>::DPL;
-  constexpr int U = 2;  // tree rows per group per pass (loads in flight)
+  constexpr int U = tree_rows_in_flight<S, D>();  // tree rows per group per pass
   constexpr bool kUsesW = (MODE == kForwardPredict || MODE == kPredictOnly);
   constexpr bool kDescend = (MODE != kPredictOnly);
   constexpr bool kAttend = (MODE == kForwardPredict || MODE == kForwardOverride);
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  constexpr int GS = WLayout<D>::g_stride;
+  constexpr int QS = WLayout<D>::q_stride;
   int* sWg = reinterpret_cast<int*>(smem_raw);
-  int* sWq = sWg + 32 * D;
+  int* sWq = sWg + 32 * GS;
   WarpBuf<S>* wbuf = reinterpret_cast<WarpBuf<S>*>(smem_raw + QuerySmem<S, D, MODE>::w_bytes);
 
   const int lane = threadIdx.x & 31;
@@ -70,11 +84,11 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocksPerSM) query_kernel(con
   if constexpr (kUsesW) {
     for (int k = threadIdx.x; k < 32 * D / 4; k += blockDim.x) {
       const int c = k / (D / 4), m = k - c * (D / 4);
-      sWq[k] = __ldg(reinterpret_cast<const int*>(a.W + c * 2 * D) + m);
+      sWq[c * QS + m] = __ldg(reinterpret_cast<const int*>(a.W + c * 2 * D) + m);
     }
     for (int k = threadIdx.x; k < 32 * D; k += blockDim.x) {
       const int c = k / D, t = k - c * D;
-      sWg[k] = a.W[c * 2 * D + D + t];
+      sWg[c * GS + t] = a.W[c * 2 * D + D + t];
     }
     __syncthreads();
   }
@@ -180,8 +194,8 @@ __global__ void __launch_bounds__(kWarps * 32, kMinBlocksPerSM) query_kernel(con
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const int m = sub + TPR * v;  // word index of dims 4m .. 4m+3
-          sq = __dp4a(sWq[c * (D / 4) + m], q.qp[v], sq);
-          const int4 wg = *reinterpret_cast<const int4*>(sWg + c * D + 4 * m);
+          sq = __dp4a(sWq[c * QS + m], q.qp[v], sq);
+          const int4 wg = *reinterpret_cast<const int4*>(sWg + c * GS + 4 * m);
           sg += (long long)wg.x * G[4 * v] + (long long)wg.y * G[4 * v + 1] +
                 (long long)wg.z * G[4 * v + 2] + (long long)wg.w * G[4 * v + 3];
         }
