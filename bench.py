@@ -82,9 +82,11 @@ def barrier(dist):
 
 
 def max_over_ranks(dist, x: float) -> float:
+    """The largest x over all ranks (NCCL on the GPU, gloo on the host)."""
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 

@@ -13,7 +13,7 @@
  *     every routing score is an exact integer;
  *   - V is bf16 (passed as raw uint16 bit patterns); outputs are fp32;
  *   - budgets come from 32 classes, class c meaning 3*(c+1) keys, at most 96 keys
- *     [README §Results and Variables: "Max keys = 96 and Max Budget class = 32"];
+ *     [README §Results and Variables: the caps are 96 keys and 32 budget classes];
  *   - the neighbour window is w keys (16 in the README's setting).
  *
  * Memory layouts (all row-major, contiguous, device memory, 16-byte aligned base pointers):
@@ -123,7 +123,7 @@ ALHR_API alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, int
  * trainable function of the current query and the global key sum that outputs a leaf group,
  * i.e. the number of keys the query asks for; §Results and Variables: 32 classes, <= 96 keys].
  *
- * For the query at position i: G_i = sum_{t <= i} K[t] (the causal reading of "global sum"),
+ * For the query at position i: G_i = sum_{t <= i} K[t] (the key sum read causally),
  * logit_c = sum_t W[c][t] q_t + sum_t W[c][d+t] G_i[t] for c = 0..31 in int64,
  * c* = the smallest c with the largest logit, budget = 3*(c*+1).
  * G_i is formed from the tree: the roots of the past-only forest of [0, i-w] plus the window

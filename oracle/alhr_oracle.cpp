@@ -16,12 +16,12 @@
 //   * pruning is a full sort of the candidates.
 //
 // Readings of points the README leaves open (each one is listed in the design notes):
-//   R1  "a global sum of all the vectors" is read causally: G_i = sum of keys 0..i.
+//   R1  the predictor's sum over all key vectors is read causally: G_i = sum of keys 0..i.
 //   R2  the budget predictor is linear: logits = W [q ; G_i], 32 classes, ties -> lower class,
 //       class c asks for 3*(c+1) keys (32 classes, at most 96 keys, as in §Results and Variables).
 //   R3  the budget counts the whole selection: the own key and the window keys come first
-//       (nearest first) and the descent only fills what is left ("subtracting found
-//       neighbour keys with the leaf group", §Inference stage, fourth paragraph).
+//       (nearest first) and the descent only fills what is left (the neighbour keys found are
+//       taken off the predicted count, §Inference stage, fourth paragraph).
 //   R4  the window is the own key plus the w-1 keys before it; when the budget is smaller
 //       than the window, it is cut nearest first.
 //   R5  causality (§Training stage, last paragraph) is the forest of maximal aligned
@@ -30,8 +30,8 @@
 //       then keeps the r best by exact integer q . node_sum (raw sums, not means), ties to
 //       the lower start position; it ends when the frontier holds only keys. The number of
 //       branches followed equals the keys still needed (§Inference stage, fourth paragraph).
-//   R7  "the data of the previous queries that matched with their own neighbours" (§Inference
-//       stage, third paragraph) is read as a cache that changes no selected set; ignored.
+//   R7  the reuse of what earlier queries found among their own neighbours (§Inference stage,
+//       third paragraph) is read as a cache that changes no selected set; ignored.
 //   R8  attention is softmax(q . k / sqrt(d)) . V over the selected keys, no temperature.
 
 #include <algorithm>
