@@ -209,6 +209,8 @@ struct WarpBuf {
   S cscore[kMaxCand];
   int xdesc[kMaxFrontier];   // nodes expanded this step
   S xscore[kMaxFrontier];
+  int xrow[kMaxFrontier];    // element offset of each expanded node's left child row
+  S xleft[kMaxFrontier];     // score of that left child
   int plist[32];             // phase-one row list (causal-sum blocks and roots)
   int winsc[32];             // scores of the window keys
 };

@@ -60,6 +60,32 @@ constexpr int min_blocks_per_sm() { return sizeof(S) == 4 ? 3 : 2; }
 template <typename S, int D>
 constexpr int tree_rows_in_flight() { return (sizeof(S) == 4 && D == 64) ? 2 : 1; }
 
+// One pass over expanded nodes whose left child is a tree row: each row group loads US rows
+// (US in flight per lane) and leaves their scores in xleft.
+template <int US, typename S, int D>
+__device__ __forceinline__ void tree_child_pass(WarpBuf<S>& B, const int32_t* Nh, const RowQ& q,
+                                                int base, int end, int grp, int sub) {
+  constexpr int RPI = Lay<D>::RPI;
+  constexpr int TPR = Lay<D>::TPR;
+  int x[US][16];
+#pragma unroll
+  for (int u = 0; u < US; ++u) {
+    const int xi = base + u * RPI + grp;
+    if (xi < end) {
+      ld_tree<D>(Nh + B.xrow[xi], sub, x[u]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) x[u][j] = 0;
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < US; ++u) {
+    const int xi = base + u * RPI + grp;
+    const S left = group_sum<S, TPR>(dot_tree<S>(q, x[u]));
+    if (xi < end && sub == 0) B.xleft[xi] = left;
+  }
+}
+
 template <typename S, int D, int MODE>
 __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_kernel(const QueryArgs a) {
   constexpr int TPR = Lay<D>::TPR;
@@ -264,20 +290,26 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
         int nhi = 0, nl1 = 0, nl = 0;
 #pragma unroll
         for (int s = 0; s < kFrontSlots; ++s) {
-          const int e = lane + 32 * s;
-          const bool ok = e < nf;
-          fd[s] = ok ? B.cdesc[e] : 0;
-          fs[s] = ok ? B.cscore[e] : S(0);
-          const int lv = desc_level(fd[s]);
-          hi[s] = ok && lv >= 2;
-          l1[s] = ok && lv == 1;
-          leaf[s] = ok && lv == 0;
-          bh_[s] = __ballot_sync(kFull, hi[s]);
-          b1_[s] = __ballot_sync(kFull, l1[s]);
-          bl_[s] = __ballot_sync(kFull, leaf[s]);
-          nhi += __popc(bh_[s]);
-          nl1 += __popc(b1_[s]);
-          nl += __popc(bl_[s]);
+          hi[s] = l1[s] = leaf[s] = false;
+          bh_[s] = b1_[s] = bl_[s] = 0u;
+          fd[s] = 0;
+          fs[s] = S(0);
+          if (32 * s < nf) {  // warp-uniform: only the slots the frontier occupies
+            const int e = lane + 32 * s;
+            const bool ok = e < nf;
+            fd[s] = ok ? B.cdesc[e] : 0;
+            fs[s] = ok ? B.cscore[e] : S(0);
+            const int lv = desc_level(fd[s]);
+            hi[s] = ok && lv >= 2;
+            l1[s] = ok && lv == 1;
+            leaf[s] = ok && lv == 0;
+            bh_[s] = __ballot_sync(kFull, hi[s]);
+            b1_[s] = __ballot_sync(kFull, l1[s]);
+            bl_[s] = __ballot_sync(kFull, leaf[s]);
+            nhi += __popc(bh_[s]);
+            nl1 += __popc(b1_[s]);
+            nl += __popc(bl_[s]);
+          }
         }
         const int nx = nhi + nl1;
         if (nx == 0) break;
@@ -285,14 +317,19 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
         exp_l1 += nl1;
         __syncwarp();
         {
+          // leaves stay candidates; expanded nodes go to the x lists with their left child's
+          // row offset (computed once per node here, not once per lane in the passes)
           const unsigned below = lanemask_lt(lane);
           int oh = 0, o1 = nhi, ol = 0;
 #pragma unroll
           for (int s = 0; s < kFrontSlots; ++s) {
             if (hi[s] || l1[s]) {
               const int pos = hi[s] ? oh + __popc(bh_[s] & below) : o1 + __popc(b1_[s] & below);
+              const int cl = desc_level(fd[s]) - 1;
+              const int st = desc_start(fd[s]);
               B.xdesc[pos] = fd[s];
               B.xscore[pos] = fs[s];
+              B.xrow[pos] = hi[s] ? int(level_row(n, cl) + (st >> cl)) * D : st * D;
             }
             if (leaf[s]) {
               const int pos = ol + __popc(bl_[s] & below);
@@ -305,39 +342,28 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
           }
         }
         __syncwarp();
-        // left children that are tree rows: U rows per group in flight
-        for (int base = 0; base < nhi; base += U * RPI) {
-          int x[U][16];
-          int pd[U];
-#pragma unroll
-          for (int u = 0; u < U; ++u) {
-            const int xi = base + u * RPI + grp;
-            pd[u] = xi < nhi ? B.xdesc[xi] : 0;
-            if (xi < nhi) {
-              const int cl = desc_level(pd[u]) - 1;
-              ld_tree<D>(Nh + (level_row(n, cl) + (desc_start(pd[u]) >> cl)) * D, sub, x[u]);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 16; ++j) x[u][j] = 0;
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < U; ++u) {
-            const int xi = base + u * RPI + grp;
-            const S left = group_sum<S, TPR>(dot_tree<S>(q, x[u]));
-            if (xi < nhi && sub == 0) put_children<S>(B, nl, xi, pd[u], B.xscore[xi], left);
+        // left children that are tree rows: U rows per group in flight, one in a last short pass
+        for (int base = 0; base < nhi;) {
+          if (U > 1 && nhi - base > RPI) {
+            tree_child_pass<U, S, D>(B, Nh, q, base, nhi, grp, sub);
+            base += U * RPI;
+          } else {
+            tree_child_pass<1, S, D>(B, Nh, q, base, nhi, grp, sub);
+            base += RPI;
           }
         }
         // left children that are keys
         for (int base = nhi; base < nx; base += RPI) {
           const int xi = base + grp;
-          const bool active = xi < nx;
-          const int pd = active ? B.xdesc[xi] : 0;
           int xp[4] = {0, 0, 0, 0};
-          if (active) ld_key<D>(Kh + (long long)desc_start(pd) * D, sub, xp);
-          const S left = S(group_sum<int, TPR>(dot_key(q, xp)));
-          if (active && sub == 0) put_children<S>(B, nl, xi, pd, B.xscore[xi], left);
+          if (xi < nx) ld_key<D>(Kh + B.xrow[xi], sub, xp);
+          const int left = group_sum<int, TPR>(dot_key(q, xp));
+          if (xi < nx && sub == 0) B.xleft[xi] = S(left);
         }
+        __syncwarp();
+        // both children of every expanded node, one node per lane
+        for (int x0 = lane; x0 < nx; x0 += 32)
+          put_children<S>(B, nl, x0, B.xdesc[x0], B.xscore[x0], B.xleft[x0]);
         const int C = nl + 2 * nx;
         if (C > r) {
           select_top_r<S>(B, C, r, lane);
