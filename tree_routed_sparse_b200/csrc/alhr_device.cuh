@@ -147,6 +147,57 @@ __device__ __forceinline__ void load_bf16(const uint16_t* row, int lane, float (
   }
 }
 
+// The softmax-weighted sum of the selected value rows, in value groups: VPR = d/8 lanes share
+// a row (one 16-byte load of 8 bf16 per lane) and a warp pass covers KPP = 32/VPR rows, UV
+// passes in flight. Keys and weights come from shared memory (selk/selp). The groups' partial
+// sums are added by log2(KPP) shuffle stages and the first group writes the fp32 row, scaled
+// by inv (the reciprocal of the softmax denominator).
+template <int D, int UV>
+__device__ __forceinline__ void gather_values(const int* selk, const float* selp, int count,
+                                              float inv, const uint16_t* Vh, int lane,
+                                              float* out_row) {
+  constexpr int VPR = D / 8;
+  constexpr int KPP = 32 / VPR;
+  const int kg = lane / VPR;
+  const int vs = lane % VPR;
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  for (int base = 0; base < count; base += UV * KPP) {
+    uint4 raw[UV];
+    float p[UV];
+#pragma unroll
+    for (int u = 0; u < UV; ++u) {
+      const int k = base + u * KPP + kg;
+      if (k < count) {
+        raw[u] = __ldg(reinterpret_cast<const uint4*>(Vh + (long long)selk[k] * D) + vs);
+        p[u] = selp[k];
+      } else {
+        raw[u] = make_uint4(0u, 0u, 0u, 0u);
+        p[u] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UV; ++u) {
+      const unsigned w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc[2 * j] = fmaf(p[u], __uint_as_float(w[j] << 16), acc[2 * j]);
+        acc[2 * j + 1] = fmaf(p[u], __uint_as_float(w[j] & 0xffff0000u), acc[2 * j + 1]);
+      }
+    }
+  }
+#pragma unroll
+  for (int off = VPR; off < 32; off *= 2)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] += __shfl_xor_sync(kFull, acc[j], off);
+  if (lane < VPR) {
+    float4* o = reinterpret_cast<float4*>(out_row + 8 * vs);
+    o[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    o[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+  }
+}
+
 template <typename S>
 __device__ __forceinline__ S warp_min(S x) {
 #pragma unroll
@@ -211,6 +262,8 @@ struct WarpBuf {
   S xscore[kMaxFrontier];
   int xrow[kMaxFrontier];    // element offset of each expanded node's left child row
   S xleft[kMaxFrontier];     // score of that left child
+  int selk[kMaxKeys];        // the selected keys and their softmax weights
+  float selp[kMaxKeys];
   int plist[32];             // phase-one row list (causal-sum blocks and roots)
   int winsc[32];             // scores of the window keys
 };

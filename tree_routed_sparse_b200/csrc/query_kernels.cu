@@ -90,7 +90,6 @@ template <typename S, int D, int MODE>
 __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_kernel(const QueryArgs a) {
   constexpr int TPR = Lay<D>::TPR;
   constexpr int RPI = Lay<D>::RPI;
-  constexpr int DPL = Lay<D>::DPL;
   constexpr int U = tree_rows_in_flight<S, D>();  // tree rows per group per pass
   constexpr bool kUsesW = (MODE == kForwardPredict || MODE == kPredictOnly);
   constexpr bool kDescend = (MODE != kPredictOnly);
@@ -435,39 +434,22 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
         psum += pr[s];
       }
       const float den = warp_sumf(psum);
-      const uint16_t* Vh = a.V + bh * (long long)n * D;
-      float acc[DPL];
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-#pragma unroll 4
-      for (int x = 0; x < nsel_win; ++x) {
-        const float px = __shfl_sync(kFull, pw, x);
-        float v[DPL];
-        load_bf16<DPL>(Vh + (long long)(i - x) * D, lane, v);
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[e] = fmaf(px, v[e], acc[e]);
+      // stage keys and weights: window keys first, then the routed keys
+      if (lane < nsel_win) {
+        B.selk[lane] = i - lane;
+        B.selp[lane] = pw;
       }
 #pragma unroll
       for (int s = 0; s < kFrontSlots; ++s) {
-        const int cnt = min(32, nf - 32 * s);
-#pragma unroll 4
-        for (int x = 0; x < cnt; ++x) {
-          const float px = __shfl_sync(kFull, pr[s], x);
-          const int key = __shfl_sync(kFull, kr[s], x);
-          float v[DPL];
-          load_bf16<DPL>(Vh + (long long)key * D, lane, v);
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) acc[e] = fmaf(px, v[e], acc[e]);
+        const int e = lane + 32 * s;
+        if (e < nf) {
+          B.selk[nsel_win + e] = kr[s];
+          B.selp[nsel_win + e] = pr[s];
         }
       }
-      const float inv = 1.f / den;
-      float* o = a.out + qi * D + lane * DPL;
-      if constexpr (DPL == 2) {
-        *reinterpret_cast<float2*>(o) = make_float2(acc[0] * inv, acc[1] * inv);
-      } else {
-        *reinterpret_cast<float4*>(o) =
-            make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-      }
+      __syncwarp();
+      gather_values<D, 2>(B.selk, B.selp, nsel_win + nf, 1.f / den, a.V + bh * (long long)n * D,
+                          lane, a.out + qi * D);
     }
   }
 }
@@ -478,7 +460,6 @@ template <int D>
 __global__ void __launch_bounds__(kWarps * 32) attend_kernel(const QueryArgs a) {
   constexpr int TPR = Lay<D>::TPR;
   constexpr int RPI = Lay<D>::RPI;
-  constexpr int DPL = Lay<D>::DPL;
   __shared__ WarpBuf<int> wbuf[kWarps];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -534,32 +515,18 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(const QueryArgs a) 
       psum += pr[s];
     }
     const float den = warp_sumf(psum);
-    float acc[DPL];
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+    // skipped entries keep weight 0 and read row 0 of the head (always in bounds)
 #pragma unroll
     for (int s = 0; s < kFrontSlots; ++s) {
-      const int c = min(32, cnt - 32 * s);
-#pragma unroll 4
-      for (int x = 0; x < c; ++x) {
-        const float px = __shfl_sync(kFull, pr[s], x);
-        const int kk = __shfl_sync(kFull, key[s], x);
-        if (px != 0.f) {
-          float v[DPL];
-          load_bf16<DPL>(Vh + (long long)kk * D, lane, v);
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) acc[e] = fmaf(px, v[e], acc[e]);
-        }
+      const int e = lane + 32 * s;
+      if (e < cnt) {
+        B.selk[e] = ok[s] ? key[s] : 0;
+        B.selp[e] = pr[s];
       }
     }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    float* o = a.out + qi * D + lane * DPL;
-    if constexpr (DPL == 2) {
-      *reinterpret_cast<float2*>(o) = make_float2(acc[0] * inv, acc[1] * inv);
-    } else {
-      *reinterpret_cast<float4*>(o) =
-          make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-    }
+    __syncwarp();
+    gather_values<D, 2>(B.selk, B.selp, cnt, den > 0.f ? 1.f / den : 0.f, Vh, lane,
+                        a.out + qi * D);
   }
 }
 
