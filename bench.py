@@ -210,26 +210,28 @@ def run_alhr(args, dist, rank, world):
     vb = max(-wl.qk_lo, wl.qk_hi)
     inp = synth.make_inputs(wl, dev)
     Q, K, V, W, bo = inp["Q"], inp["K"], inp["V"], inp["W"], inp["budget_override"]
-    nodes = torch.empty((wl.batch, wl.heads, wl.n - 1, wl.d), dtype=torch.int32, device=dev)
+    tree = torch.empty((wl.batch, wl.heads, alhr.tree_bytes(wl.n, wl.d, vb)), dtype=torch.uint8,
+                       device=dev)
     out = torch.empty((wl.batch, wl.heads, wl.nq, wl.d), dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     kw = dict(q_start=wl.q_start, window=wl.window, max_keys=wl.max_keys,
               score_bits=wl.score_bits, value_bound=vb)
 
     def step():
-        alhr.build_tree(K, nodes, value_bound=vb)
-        alhr.forward(Q, K, V, nodes, W=W, budget_override=bo, out=out, **kw)
+        alhr.build_tree(K, tree, value_bound=vb)
+        alhr.forward(Q, K, V, tree, W=W, budget_override=bo, out=out, **kw)
 
     # one untimed run with every output: counts for the byte model
-    alhr.build_tree(K, nodes, value_bound=vb)
-    full = alhr.forward(Q, K, V, nodes, W=W, budget_override=bo, want_count=True,
+    alhr.build_tree(K, tree, value_bound=vb)
+    full = alhr.forward(Q, K, V, tree, W=W, budget_override=bo, want_count=True,
                         want_expansions=True, want_budget=True, **kw)
     torch.cuda.synchronize()
     pos = np.broadcast_to(np.arange(wl.q_start, wl.q_start + wl.nq), (wl.bh, wl.nq))
-    fwd_bytes = metrics.forward_bytes(pos, wl.d, wl.window, full["count"].cpu().numpy(),
+    fwd_bytes = metrics.forward_bytes(pos, wl.n, wl.d, wl.window, full["count"].cpu().numpy(),
                                       full["expansions"].cpu().numpy(),
-                                      full["budget"].cpu().numpy(), wl.predictor, wl.max_keys)
-    tree_bytes = metrics.tree_bytes(wl.bh, wl.n, wl.d)
+                                      full["budget"].cpu().numpy(), wl.predictor, wl.max_keys,
+                                      value_bound=vb)
+    tree_bytes = metrics.tree_bytes(wl.bh, wl.n, wl.d, vb)
     mean_keys = float(full["count"].float().mean())
     mean_budget = float(full["budget"].float().mean())
     del full
@@ -249,9 +251,9 @@ def run_alhr(args, dist, rank, world):
     for s in range(args.steps):
         flush.fill_(s & 0xFF)
         ev[s][0].record(stream)
-        alhr.build_tree(K, nodes, value_bound=vb)
+        alhr.build_tree(K, tree, value_bound=vb)
         ev[s][1].record(stream)
-        alhr.forward(Q, K, V, nodes, W=W, budget_override=bo, out=out, **kw)
+        alhr.forward(Q, K, V, tree, W=W, budget_override=bo, out=out, **kw)
         ev[s][2].record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
@@ -282,8 +284,8 @@ def run_alhr(args, dist, rank, world):
             dW.copy_(host["W"], non_blocking=True)
         if dbo is not None:
             dbo.copy_(host["budget_override"], non_blocking=True)
-        alhr.build_tree(dK, nodes, value_bound=vb)
-        alhr.forward(dQ, dK, dV, nodes, W=dW, budget_override=dbo, out=out, **kw)
+        alhr.build_tree(dK, tree, value_bound=vb)
+        alhr.forward(dQ, dK, dV, tree, W=dW, budget_override=dbo, out=out, **kw)
         out_host.copy_(out, non_blocking=True)
 
     for _ in range(3):

@@ -20,13 +20,25 @@
  *   Q      int8     [batch][heads][nq][d]        row t is the query at position q_start+t
  *   K      int8     [batch][heads][n][d]
  *   V      uint16   [batch][heads][n][d]         bf16 bit patterns
- *   nodes  int32    [batch][heads][n-1][d]       level-major tree (see alhr_tree_level_offset)
+ *   tree   bytes    [batch][heads][alhr_tree_bytes(n, d, value_bound)]  the key tree, see below
  *   W      int8     [32][2d]                     budget-predictor weights, shared by all heads
  *   budget int32    [batch][heads][nq]           keys asked for by each query (>= 1)
  *   idx    int32    [batch][heads][nq][max_keys] selected key positions, ascending, -1 padded
  *   count  int32    [batch][heads][nq]           number of valid entries of idx
- *   expansions int32 [batch][heads][nq][2]       {nodes of level >= 2 expanded, level-1 nodes expanded}
+ *   expansions int32 [batch][heads][nq][3]       {nodes of level >= 2 expanded, level-1 nodes
+ *                                                 expanded, expanded nodes whose children are
+ *                                                 32-bit tree rows (level >= wide_level + 1)}
  *   out    float    [batch][heads][nq][d]
+ *
+ * Tree layout (one block of alhr_tree_bytes(n, d, value_bound) bytes per (b,h), blocks
+ * consecutive): levels 1 .. log2 n in increasing order, level l holding n >> l rows; row j of
+ * level l is the exact sum of keys [j*2^l, (j+1)*2^l). At d = 128 a level whose sums are bounded
+ * by value_bound * 2^l <= 32767 is stored as int16 rows of 2d bytes ("narrow" levels 1 ..
+ * alhr_tree_narrow_levels); every other level (every level at d = 64) as int32 rows of 4d
+ * bytes. The byte offset of a
+ * level inside a block is alhr_tree_level_offset(). The layout depends on value_bound, so every
+ * call that reads a tree must pass the value_bound it was built with. alhr_tree_unpack expands
+ * a tree to plain int32 rows.
  *
  * Ownership: every pointer belongs to the caller. The library allocates no device memory and
  * keeps no state between calls; a call only reads its inputs and writes its outputs.
@@ -87,11 +99,18 @@ typedef struct {
 /* Number of tree rows per (b,h): n - 1. Returns 0 when n is not a power of two in [2, 2^20]. */
 ALHR_API size_t alhr_tree_rows(int32_t n);
 
-/* Row offset of tree level `level` (1 <= level <= log2 n) inside one (b,h) block of `nodes`:
- * level l holds n >> l rows starting at row n - (n >> (l-1)); row j of level l is the sum of
- * keys [j*2^l, (j+1)*2^l). Level 0 (the keys themselves) is K and is not stored.
- * Returns (size_t)-1 for an invalid pair. */
-ALHR_API size_t alhr_tree_level_offset(int32_t n, int32_t level);
+/* Number of narrow (int16) levels: at d = 128 the largest l with value_bound * 2^l <= 32767
+ * (value_bound 0 means 16), capped at log2 n; at d = 64 none (every level is int32: there the
+ * descent is bound by instruction issue, not by row bytes). -1 for invalid arguments. */
+ALHR_API int32_t alhr_tree_narrow_levels(int32_t n, int32_t d, int32_t value_bound);
+
+/* Bytes of one (b,h) block of the tree (a multiple of 128), or 0 for invalid arguments
+ * (n a power of two in [2, 2^20], d in {64, 128}, 0 <= value_bound <= 127). */
+ALHR_API size_t alhr_tree_bytes(int32_t n, int32_t d, int32_t value_bound);
+
+/* Byte offset of tree level `level` (1 <= level <= log2 n) inside one (b,h) block. Level 0 (the
+ * keys themselves) is K and is not stored. Returns (size_t)-1 for invalid arguments. */
+ALHR_API size_t alhr_tree_level_offset(int32_t n, int32_t d, int32_t value_bound, int32_t level);
 
 /* Score width the kernels will use for these sizes (32 or 64), or a negative alhr_status
  * (-ALHR_ERR_...) when the sizes are invalid or score_bits = 32 cannot be exact. */
@@ -108,15 +127,25 @@ ALHR_API const char* alhr_build_info(void);
  * is built on the key matrix and stored, once per layer; README opening paragraph: every
  * branch is indexed by the sum of all key vectors beneath it].
  *
- * For every (b,h) writes nodes(l, j) = sum_{t in [j*2^l, (j+1)*2^l)} K[t] for l = 1..log2 n,
- * exact in int32, level-major as described at alhr_tree_level_offset. Only dims->batch,
- * heads, n, d and value_bound are read.
+ * For every (b,h) writes node(l, j) = sum_{t in [j*2^l, (j+1)*2^l)} K[t] for l = 1..log2 n,
+ * exact, in the tree layout above. Only dims->batch, heads, n, d and value_bound are read.
  *   K       device, int8 [batch][heads][n][d], read only
- *   nodes   device, int32 [batch][heads][n-1][d], fully overwritten
- *   dev_err device uint32 or NULL; ALHR_DEVERR_VALUE_RANGE if some |K| > value_bound
+ *   tree    device, batch*heads*alhr_tree_bytes(n, d, value_bound) bytes, fully overwritten
+ *   dev_err device uint32 or NULL; ALHR_DEVERR_VALUE_RANGE if some |K| > value_bound (the
+ *           narrow levels are then not exact)
  */
-ALHR_API alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, int32_t* nodes,
-                            uint32_t* dev_err, void* stream);
+ALHR_API alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, void* tree,
+                                     uint32_t* dev_err, void* stream);
+
+/*
+ * alhr_tree_unpack -- the tree as plain int32 rows: nodes[b][h][r][:] for r in [0, n-1), level l
+ * at rows [n - (n >> (l-1)), n - (n >> l)) (level-major, level 1 first). Reads dims->batch,
+ * heads, n, d and value_bound.
+ *   tree   device, as written by alhr_build_tree with the same dims
+ *   nodes  device, int32 [batch][heads][n-1][d], fully overwritten
+ */
+ALHR_API alhr_status alhr_tree_unpack(const alhr_dims* dims, const void* tree, int32_t* nodes,
+                                      void* stream);
 
 /*
  * alhr_predict_budget -- the budget predictor [README §Inference stage, second paragraph: a
@@ -128,13 +157,13 @@ ALHR_API alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, int
  * c* = the smallest c with the largest logit, budget = 3*(c*+1).
  * G_i is formed from the tree: the roots of the past-only forest of [0, i-w] plus the window
  * keys (i-w, i].
- *   Q, K, nodes  device inputs (layouts above); W device int8 [32][2d]
+ *   Q, K, tree   device inputs (layouts above); W device int8 [32][2d]
  *   budget       device int32 [batch][heads][nq], overwritten
  *   dev_err      as above (ALHR_DEVERR_VALUE_RANGE for |q| > value_bound)
  */
 ALHR_API alhr_status alhr_predict_budget(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
-                                const int32_t* nodes, const int8_t* W, int32_t* budget,
-                                uint32_t* dev_err, void* stream);
+                                         const void* tree, const int8_t* W, int32_t* budget,
+                                         uint32_t* dev_err, void* stream);
 
 /*
  * alhr_route -- neighbour search plus budget-limited tree descent [README §Inference stage,
@@ -151,12 +180,13 @@ ALHR_API alhr_status alhr_predict_budget(const alhr_dims* dims, const int8_t* Q,
  *   The routed keys are the final frontier; the selection is window + routed.
  *   idx        device int32 [..][max_keys]: selection ascending, -1 padded (required)
  *   count      device int32: |selection| = min(B_eff, i+1) (required)
- *   expansions device int32 [..][2] or NULL: {level >= 2 nodes expanded, level-1 nodes expanded}
+ *   expansions device int32 [..][3] or NULL: the three expansion counters of the layout table
  *   dev_err    as above (ALHR_DEVERR_BUDGET_LOW, ALHR_DEVERR_VALUE_RANGE)
  */
 ALHR_API alhr_status alhr_route(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
-                       const int32_t* nodes, const int32_t* budget, int32_t* idx, int32_t* count,
-                       int32_t* expansions, uint32_t* dev_err, void* stream);
+                                const void* tree, const int32_t* budget, int32_t* idx,
+                                int32_t* count, int32_t* expansions, uint32_t* dev_err,
+                                void* stream);
 
 /*
  * alhr_attend -- exact attention over the selected keys [README §Inference stage, fifth
@@ -185,7 +215,7 @@ ALHR_API alhr_status alhr_attend(const alhr_dims* dims, const int8_t* Q, const i
  * Results equal alhr_predict_budget + alhr_route + alhr_attend on the same inputs.
  */
 ALHR_API alhr_status alhr_forward(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
-                         const uint16_t* V, const int32_t* nodes, const int8_t* W,
+                         const uint16_t* V, const void* tree, const int8_t* W,
                          const int32_t* budget_override, float* out, int32_t* idx,
                          int32_t* count, int32_t* expansions, int32_t* budget_out,
                          uint32_t* dev_err, void* stream);

@@ -136,11 +136,15 @@ int oracle_predict(int d, const int8_t* q, const int64_t* G, const int8_t* W, in
 
 // Neighbour search and budget-limited descent for the query q at position i with budget B,
 // readings R3..R7 [README §Inference stage, third and fourth paragraphs; §Training stage, last
-// paragraph]. Writes the selection ascending into sel (room for min(B, i+1, max_keys) entries)
-// and {nodes of level >= 2 expanded, level-1 nodes expanded} into expansions (nullable).
+// paragraph]. Writes the selection ascending into sel (room for min(B, i+1, max_keys) entries),
+// {nodes of level >= 2 expanded, level-1 nodes expanded} into expansions (nullable) and the
+// number of expanded nodes of each level l into by_level[l], l < 32 (nullable).
 // Returns the selection size min(B_eff, i+1) with B_eff = min(max(B,1), i+1, max_keys).
 int oracle_route(int n, int d, const int8_t* K, const int32_t* nodes, const int8_t* q, int i,
-                 int budget, int w, int max_keys, int32_t* sel, int32_t* expansions) {
+                 int budget, int w, int max_keys, int32_t* sel, int32_t* expansions,
+                 int32_t* by_level) {
+  if (by_level)
+    for (int l = 0; l < 32; ++l) by_level[l] = 0;
   int64_t b_eff = std::max(budget, 1);
   b_eff = std::min<int64_t>(b_eff, int64_t(i) + 1);
   b_eff = std::min<int64_t>(b_eff, max_keys);
@@ -175,6 +179,7 @@ int oracle_route(int n, int d, const int8_t* K, const int32_t* nodes, const int8
           continue;
         }
         if (nd.level >= 2) ++exp_hi; else ++exp_l1;
+        if (by_level) ++by_level[nd.level];
         const int cl = nd.level - 1;
         const int64_t left = nd.start, right = nd.start + (int64_t(1) << cl);
         cand.push_back({cl, left, node_score(n, d, K, nodes, q, cl, left)});
@@ -232,12 +237,13 @@ void oracle_attend(int d, const int8_t* q, const int8_t* K, const uint16_t* V,
 //   Q [nq][d], K [n][d], V [n][d], nodes [n-1][d] (this oracle's own tree), W [32][2d] or NULL,
 //   budget_override [nq] or NULL, rows: the query rows to compute (NULL = all nq rows).
 // Outputs (rows not listed are left untouched): out [nq][d], idx [nq][max_keys] (-1 padded),
-// count [nq], expansions [nq][2], budget_out [nq] (the budget used, after the clamp to >= 1).
+// count [nq], expansions [nq][2], budget_out [nq] (the budget used, after the clamp to >= 1),
+// by_level [nq][32] or NULL (expanded nodes per level).
 void oracle_forward(int n, int d, int q_start, int nq, int w, int max_keys, const int8_t* Q,
                     const int8_t* K, const uint16_t* V, const int32_t* nodes, const int8_t* W,
                     const int32_t* budget_override, const int32_t* rows, int n_rows,
                     double* out, int32_t* idx, int32_t* count, int32_t* expansions,
-                    int32_t* budget_out) {
+                    int32_t* budget_out, int32_t* by_level) {
   std::vector<int64_t> G(static_cast<size_t>(d));
   std::vector<int32_t> sel(static_cast<size_t>(std::max(max_keys, 1)));
   const int total = rows ? n_rows : nq;
@@ -253,7 +259,8 @@ void oracle_forward(int n, int d, int q_start, int nq, int w, int max_keys, cons
       budget = 3 * (oracle_predict(d, q, G.data(), W, nullptr) + 1);
     }
     const int c = oracle_route(n, d, K, nodes, q, i, budget, w, max_keys, sel.data(),
-                               expansions + int64_t(row) * 2);
+                               expansions + int64_t(row) * 2,
+                               by_level ? by_level + int64_t(row) * 32 : nullptr);
     oracle_attend(d, q, K, V, sel.data(), c, out + int64_t(row) * d);
     for (int s = 0; s < max_keys; ++s) idx[int64_t(row) * max_keys + s] = s < c ? sel[size_t(s)] : -1;
     count[row] = c;

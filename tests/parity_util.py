@@ -3,6 +3,29 @@ import numpy as np
 import torch
 
 from oracle import oracle as orc
+from tree_routed_sparse_b200 import metrics
+
+
+def decode_tree(block: np.ndarray, n: int, d: int, value_bound: int = 16) -> np.ndarray:
+    """One (b,h) block of the tree bytes -> level-major int32 rows [n-1, d], read with the
+    layout documented in include/alhr.h (levels in order; at d = 128 int16 rows for
+    value_bound * 2^l <= 32767, int32 otherwise), independently of the library's unpack kernel."""
+    block = np.ascontiguousarray(block, dtype=np.uint8)
+    narrow = metrics.narrow_levels(n, d, value_bound)
+    out = np.zeros((n - 1, d), dtype=np.int32)
+    off, row0 = 0, 0
+    for lev in range(1, n.bit_length()):
+        rows = n >> lev
+        if lev <= narrow:
+            part = block[off: off + rows * 2 * d].view(np.int16).reshape(rows, d)
+            off += rows * 2 * d
+        else:
+            part = block[off: off + rows * 4 * d].view(np.int32).reshape(rows, d)
+            off += rows * 4 * d
+        out[row0: row0 + rows] = part
+        row0 += rows
+    assert off == len(block)
+    return out
 
 
 def v_bits(V: torch.Tensor) -> np.ndarray:
@@ -21,6 +44,7 @@ def oracle_slice(inp_cpu: dict, wl, b: int, h: int, rows=None, nodes=None) -> di
     res = orc.forward(Q, K, V, nodes, W, bo, q_start=wl.q_start, window=wl.window,
                       max_keys=wl.max_keys, rows=rows)
     res["nodes"] = nodes
+    res["narrow"] = metrics.narrow_levels(wl.n, wl.d, max(-wl.qk_lo, wl.qk_hi))
     return res
 
 
@@ -31,6 +55,11 @@ def compare_rows(gpu: dict, ref: dict, b: int, h: int, rows, tol=1e-3, what=""):
         if key in gpu:
             g = gpu[key][b, h].cpu().numpy()[rows]
             r = ref[key][rows]
+            if key == "expansions":
+                # GPU: {level >= 2, level 1, children stored as int32 rows}; the oracle gives the
+                # first two and a per-level histogram for the third
+                wide = ref["by_level"][rows][:, ref["narrow"] + 2:].sum(1)
+                r = np.concatenate([r, wide[:, None]], axis=1).astype(np.int32)
             if not np.array_equal(g, r):
                 bad = np.nonzero((g != r).reshape(len(rows), -1).any(1))[0][:5]
                 raise AssertionError(f"{what} {key} differs at rows {rows[bad].tolist()}:\n"

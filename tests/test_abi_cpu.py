@@ -51,10 +51,40 @@ def test_tree_layout_helpers(A):
     L = A.lib()
     assert L.alhr_tree_rows(8) == 7 and L.alhr_tree_rows(1 << 20) == (1 << 20) - 1
     assert L.alhr_tree_rows(6) == 0 and L.alhr_tree_rows(1) == 0 and L.alhr_tree_rows(1 << 21) == 0
-    assert [L.alhr_tree_level_offset(8, l) for l in (1, 2, 3)] == [0, 4, 6]
-    assert L.alhr_tree_level_offset(8, 0) == 2**64 - 1
-    assert L.alhr_tree_level_offset(8, 4) == 2**64 - 1
+    # n = 8, d = 128, value_bound 16: every level narrow (int16 rows of 256 bytes); at d = 64
+    # every level is int32 (rows of 256 bytes too)
+    assert [L.alhr_tree_level_offset(8, 128, 16, l) for l in (1, 2, 3)] == [0, 4 * 256, 6 * 256]
+    assert [L.alhr_tree_level_offset(8, 64, 16, l) for l in (1, 2, 3)] == [0, 4 * 256, 6 * 256]
+    assert L.alhr_tree_level_offset(8, 64, 16, 0) == 2**64 - 1
+    assert L.alhr_tree_level_offset(8, 64, 16, 4) == 2**64 - 1
+    assert L.alhr_tree_level_offset(8, 96, 16, 1) == 2**64 - 1
+    assert L.alhr_tree_narrow_levels(16384, 128, 16) == 10
+    assert L.alhr_tree_narrow_levels(16384, 128, 0) == 10
+    assert L.alhr_tree_narrow_levels(16384, 64, 16) == 0
+    assert L.alhr_tree_narrow_levels(1024, 128, 127) == 8 and L.alhr_tree_narrow_levels(8, 128, 1) == 3
+    assert L.alhr_tree_narrow_levels(1000, 128, 16) == -1
+    assert L.alhr_tree_narrow_levels(8, 128, 128) == -1 and L.alhr_tree_narrow_levels(8, 32, 16) == -1
+    assert L.alhr_tree_bytes(6, 64, 16) == 0 and L.alhr_tree_bytes(8, 32, 16) == 0
     assert b"sm_100a" in L.alhr_build_info()
+
+
+@pytest.mark.parametrize("n,d,vb", [(16384, 64, 16), (262144, 128, 16), (1024, 128, 127),
+                                    (4096, 128, 3), (2, 64, 0), (2, 128, 0), (1 << 20, 128, 1)])
+def test_tree_layout_matches_documented_layout(A, n, d, vb):
+    """Level offsets and block size follow the layout of include/alhr.h (levels in order,
+    int16 rows up to the narrow level, int32 above), computed here independently."""
+    from tree_routed_sparse_b200 import metrics
+    L = A.lib()
+    narrow = (0 if d == 64 else
+              max([l for l in range(0, n.bit_length()) if (vb or 16) << l <= 32767]))
+    assert metrics.narrow_levels(n, d, vb) == narrow
+    assert L.alhr_tree_narrow_levels(n, d, vb) == narrow
+    off = 0
+    for lev in range(1, n.bit_length()):
+        assert L.alhr_tree_level_offset(n, d, vb, lev) == off
+        off += (n >> lev) * (2 * d if lev <= narrow else 4 * d)
+    assert L.alhr_tree_bytes(n, d, vb) == off == metrics.tree_block_bytes(n, d, vb)
+    assert off % 128 == 0
 
 
 def _dims(A, **kw):

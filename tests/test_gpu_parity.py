@@ -7,7 +7,7 @@ import pytest
 import torch
 
 from oracle import oracle as orc
-from parity_util import compare_rows, oracle_slice, v_bits
+from parity_util import compare_rows, decode_tree, oracle_slice, v_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -37,15 +37,17 @@ def _to(inp, device):
 
 def _run_forward(A, wl, inp, **kw):
     dev = inp["Q"].device
-    nodes = A.build_tree(inp["K"], value_bound=max(-wl.qk_lo, wl.qk_hi))
+    vb = max(-wl.qk_lo, wl.qk_hi)
+    tree = A.build_tree(inp["K"], value_bound=vb)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    res = A.forward(inp["Q"], inp["K"], inp["V"], nodes, W=inp["W"],
+    res = A.forward(inp["Q"], inp["K"], inp["V"], tree, W=inp["W"],
                     budget_override=inp["budget_override"], q_start=wl.q_start,
                     window=wl.window, max_keys=wl.max_keys, score_bits=wl.score_bits,
                     value_bound=max(-wl.qk_lo, wl.qk_hi), want_idx=True, want_count=True,
                     want_expansions=True, want_budget=True, dev_err=err, **kw)
     torch.cuda.synchronize()
-    res["nodes"] = nodes
+    res["tree"] = tree
+    res["nodes"] = A.tree_unpack(tree, wl.n, wl.d, vb)
     res["dev_err"] = int(err.item())
     return res
 
@@ -56,12 +58,32 @@ def _run_forward(A, wl, inp, **kw):
 @pytest.mark.parametrize("B,H,n,d", [(1, 1, 2, 64), (1, 1, 8, 128), (2, 3, 128, 64),
                                      (1, 2, 1024, 128), (2, 1, 4096, 64), (1, 1, 1 << 16, 64)])
 def test_tree_bit_exact(alhr, synth, B, H, n, d):
+    """Both the library's unpack and an independent host reading of the documented layout
+    give the oracle's sums."""
     K = synth.uniform_int8(7, synth.TID_K, (B, H, n, d), -16, 16, "cuda")
-    nodes = alhr.build_tree(K).cpu().numpy()
+    tree = alhr.build_tree(K)
+    nodes = alhr.tree_unpack(tree, n, d).cpu().numpy()
+    tb = tree.cpu().numpy()
     Kc = K.cpu().numpy()
     for b in range(B):
         for h in range(H):
-            assert np.array_equal(nodes[b, h], orc.build_tree(Kc[b, h])), (b, h)
+            ref = orc.build_tree(Kc[b, h])
+            assert np.array_equal(nodes[b, h], ref), (b, h)
+            assert np.array_equal(decode_tree(tb[b, h], n, d, 16), ref), (b, h)
+
+
+@pytest.mark.parametrize("vb,n,d", [(127, 1024, 128), (1, 4096, 128), (5, 8192, 64), (16, 2048, 128)])
+def test_tree_other_value_bounds(alhr, synth, vb, n, d):
+    """Other bounds move the int16/int32 boundary; sums stay exact at the extremes."""
+    K = synth.uniform_int8(11, synth.TID_K, (1, 2, n, d), -vb, vb, "cuda")
+    K[0, 1, : n // 2] = vb
+    tree = alhr.build_tree(K, value_bound=vb)
+    tb = tree.cpu().numpy()
+    nodes = alhr.tree_unpack(tree, n, d, vb).cpu().numpy()
+    for h in range(2):
+        ref = orc.build_tree(K[0, h].cpu().numpy())
+        assert np.array_equal(nodes[0, h], ref)
+        assert np.array_equal(decode_tree(tb[0, h], n, d, vb), ref)
 
 
 def test_tree_extremes_and_range_flag(alhr):
@@ -70,8 +92,9 @@ def test_tree_extremes_and_range_flag(alhr):
     K[0, 0, 1::2] = -16
     K[0, 0, :512] = 16
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    nodes = alhr.build_tree(K, dev_err=err)
+    tree = alhr.build_tree(K, dev_err=err)
     assert int(err.item()) == 0
+    nodes = alhr.tree_unpack(tree, n, d)
     assert np.array_equal(nodes[0, 0].cpu().numpy(), orc.build_tree(K[0, 0].cpu().numpy()))
     K[0, 0, 77, 5] = 17
     alhr.build_tree(K, value_bound=16, dev_err=err)
@@ -170,8 +193,8 @@ def test_unfused_path_matches_oracle_and_fused(alhr, synth, d, bits):
     inp = synth.make_inputs(wl, "cuda")
     fused = _run_forward(alhr, wl, inp)
     kw = dict(q_start=0, window=wl.window, max_keys=wl.max_keys, score_bits=bits)
-    budget = alhr.predict_budget(inp["Q"], inp["K"], fused["nodes"], inp["W"], **kw)
-    routed = alhr.route(inp["Q"], inp["K"], fused["nodes"], budget, **kw)
+    budget = alhr.predict_budget(inp["Q"], inp["K"], fused["tree"], inp["W"], **kw)
+    routed = alhr.route(inp["Q"], inp["K"], fused["tree"], budget, **kw)
     out = alhr.attend(inp["Q"], inp["K"], inp["V"], routed["idx"], routed["count"],
                       q_start=0, window=wl.window, max_keys=wl.max_keys)
     torch.cuda.synchronize()
@@ -213,9 +236,9 @@ def test_attend_skips_bad_indices(alhr, synth):
 def test_empty_and_invalid_calls(alhr, synth):
     wl = synth.WORKLOADS["tiny_prefill_n1024"].replace(n=64, nq=0)
     inp = synth.make_inputs(wl, "cuda")
-    nodes = alhr.build_tree(inp["K"])
-    res = alhr.forward(inp["Q"], inp["K"], inp["V"], nodes, budget_override=inp["budget_override"])
+    tree = alhr.build_tree(inp["K"])
+    res = alhr.forward(inp["Q"], inp["K"], inp["V"], tree, budget_override=inp["budget_override"])
     assert res["out"].numel() == 0
     with pytest.raises(alhr.AlhrError):
-        alhr.forward(inp["Q"], inp["K"], inp["V"], nodes, window=33,
+        alhr.forward(inp["Q"], inp["K"], inp["V"], tree, window=33,
                      budget_override=inp["budget_override"])

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 from oracle import oracle as orc
-from parity_util import compare_rows, oracle_slice
+from parity_util import compare_rows, decode_tree, oracle_slice
 
 pytestmark = pytest.mark.gpu
 
@@ -55,7 +55,7 @@ def _slice_inputs(inp, wl, b, h):
 def test_workload_parity(alhr, name, blocks):
     from tree_routed_sparse_b200 import synth
     wl = synth.WORKLOADS[name]
-    need = wl.bh * wl.n * wl.d * (1 + 2 + 4) + wl.bh * wl.nq * wl.d * 5
+    need = wl.bh * wl.n * wl.d * (1 + 2 + 4) + wl.bh * wl.nq * wl.d * 5  # K, V, tree <= 4d/row
     free, _ = torch.cuda.mem_get_info()
     if need > free - (2 << 30):
         pytest.skip(f"{name} needs {need / 2**30:.1f} GiB, {free / 2**30:.1f} GiB free")
@@ -65,10 +65,10 @@ def test_workload_parity(alhr, name, blocks):
               score_bits=wl.score_bits, value_bound=vb)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     # the benchmark's configuration
-    nodes = alhr.build_tree(inp["K"], value_bound=vb, dev_err=err)
-    bench_out = alhr.forward(inp["Q"], inp["K"], inp["V"], nodes, W=inp["W"],
+    tree = alhr.build_tree(inp["K"], value_bound=vb, dev_err=err)
+    bench_out = alhr.forward(inp["Q"], inp["K"], inp["V"], tree, W=inp["W"],
                              budget_override=inp["budget_override"], dev_err=err, **kw)["out"]
-    full = alhr.forward(inp["Q"], inp["K"], inp["V"], nodes, W=inp["W"],
+    full = alhr.forward(inp["Q"], inp["K"], inp["V"], tree, W=inp["W"],
                         budget_override=inp["budget_override"], want_idx=True, want_count=True,
                         want_expansions=True, want_budget=True, dev_err=err, **kw)
     torch.cuda.synchronize()
@@ -79,7 +79,8 @@ def test_workload_parity(alhr, name, blocks):
         rows = _sample_rows(wl.nq, rng)
         cpu = _slice_inputs(inp, wl, b, h)
         ref = oracle_slice(cpu, wl, 0, 0, rows=rows)
-        assert np.array_equal(nodes[b, h].cpu().numpy(), ref["nodes"]), f"tree {b},{h}"
+        got = decode_tree(tree[b, h].cpu().numpy(), wl.n, wl.d, vb)
+        assert np.array_equal(got, ref["nodes"]), f"tree {b},{h}"
         sub = {k: v[b:b + 1, h:h + 1].cpu() for k, v in full.items()}
         compare_rows(sub, ref, 0, 0, rows, TOL, f"{name} b{b}h{h}")
     if wl.plant_pairs:
@@ -91,5 +92,5 @@ def test_workload_parity(alhr, name, blocks):
             sel = idx[b][:, u]  # [H, P, max_keys]
             hits += int((sel == p.view(1, -1, 1).to(torch.int32)).any(-1).sum())
         print(f"recall@selection {hits / (wl.batch * wl.heads * wl.plant_pairs):.3f}")
-    del inp, nodes, full, bench_out
+    del inp, tree, full, bench_out
     torch.cuda.empty_cache()

@@ -376,3 +376,27 @@ def test_forward_budget_override_clamp_and_predictor():
                       rows=np.array([0, 1, 2], dtype=np.int32))
     assert res["budget"][:3].tolist() == [1, 1, 3]
     assert res["count"][:3].tolist() == [1, 1, 3]
+
+
+def test_expansions_by_level_add_up(golden_n8):
+    """The per-level histogram sums to the two counters; the wide-beam case expands every
+    internal node of the forest once, so level l holds the forest's level-l nodes."""
+    K = np.array(golden_n8["K"], dtype=np.int8)
+    nodes = orc.build_tree(K)
+    for case in golden_n8["routes"]:
+        sel, exp, lv = orc.route(K, nodes, np.array(case["q"], dtype=np.int8), case["i"],
+                                 case["budget"], golden_n8["window"], 96, by_level=True)
+        assert lv[0] == 0 and lv[2:].sum() == exp[0] and lv[1] == exp[1]
+    rng = _rng(77)
+    n, d, w = 256, 8, 5
+    K = _rand_qk(rng, (n, d))
+    nodes = orc.build_tree(K)
+    for i in [200, 255, 77]:
+        _, _, lv = orc.route(K, nodes, _rand_qk(rng, (d,)), i, n, w, n, by_level=True)
+        m = i - w + 1
+        expect = np.zeros(32, dtype=np.int64)
+        for b in range(1, 20):
+            if (m >> b) & 1:
+                for l in range(1, b + 1):
+                    expect[l] += 1 << (b - l)
+        assert lv.tolist() == expect.tolist()

@@ -23,9 +23,10 @@ DEVERR_BUDGET_LOW = 0x1
 DEVERR_VALUE_RANGE = 0x2
 DEVERR_INDEX = 0x4
 
-EXPORTS = ["alhr_tree_rows", "alhr_tree_level_offset", "alhr_score_bits",
-           "alhr_status_string", "alhr_build_info", "alhr_build_tree", "alhr_predict_budget",
-           "alhr_route", "alhr_attend", "alhr_forward"]
+EXPORTS = ["alhr_tree_rows", "alhr_tree_narrow_levels", "alhr_tree_bytes",
+           "alhr_tree_level_offset", "alhr_score_bits", "alhr_status_string", "alhr_build_info",
+           "alhr_build_tree", "alhr_tree_unpack", "alhr_predict_budget", "alhr_route",
+           "alhr_attend", "alhr_forward"]
 
 
 class AlhrError(RuntimeError):
@@ -54,17 +55,22 @@ def lib() -> ctypes.CDLL:
         P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
         DP = ctypes.POINTER(Dims)
         L.alhr_tree_rows.argtypes, L.alhr_tree_rows.restype = [I32], SZ
-        L.alhr_tree_level_offset.argtypes, L.alhr_tree_level_offset.restype = [I32, I32], SZ
+        L.alhr_tree_narrow_levels.argtypes = [I32, I32, I32]
+        L.alhr_tree_narrow_levels.restype = I32
+        L.alhr_tree_bytes.argtypes, L.alhr_tree_bytes.restype = [I32, I32, I32], SZ
+        L.alhr_tree_level_offset.argtypes = [I32, I32, I32, I32]
+        L.alhr_tree_level_offset.restype = SZ
         L.alhr_score_bits.argtypes, L.alhr_score_bits.restype = [DP], I32
         L.alhr_status_string.argtypes, L.alhr_status_string.restype = [I32], ctypes.c_char_p
         L.alhr_build_info.argtypes, L.alhr_build_info.restype = [], ctypes.c_char_p
         L.alhr_build_tree.argtypes = [DP, P, P, P, P]
+        L.alhr_tree_unpack.argtypes = [DP, P, P, P]
         L.alhr_predict_budget.argtypes = [DP, P, P, P, P, P, P, P]
         L.alhr_route.argtypes = [DP, P, P, P, P, P, P, P, P, P]
         L.alhr_attend.argtypes = [DP, P, P, P, P, P, P, P, P]
         L.alhr_forward.argtypes = [DP, P, P, P, P, P, P, P, P, P, P, P, P, P]
-        for f in ("alhr_build_tree", "alhr_predict_budget", "alhr_route", "alhr_attend",
-                  "alhr_forward"):
+        for f in ("alhr_build_tree", "alhr_tree_unpack", "alhr_predict_budget", "alhr_route",
+                  "alhr_attend", "alhr_forward"):
             getattr(L, f).restype = I32
         _lib = L
     return _lib
@@ -101,25 +107,51 @@ def tree_rows(n: int) -> int:
     return int(lib().alhr_tree_rows(n))
 
 
+def tree_bytes(n: int, d: int, value_bound: int = 16) -> int:
+    """Bytes of one (b,h) block of the tree."""
+    return int(lib().alhr_tree_bytes(n, d, value_bound))
+
+
+def tree_narrow_levels(n: int, d: int, value_bound: int = 16) -> int:
+    return int(lib().alhr_tree_narrow_levels(n, d, value_bound))
+
+
+def tree_level_offset(n: int, d: int, value_bound: int, level: int) -> int:
+    return int(lib().alhr_tree_level_offset(n, d, value_bound, level))
+
+
 def score_bits(dims: Dims) -> int:
     return int(lib().alhr_score_bits(ctypes.byref(dims)))
 
 
-def build_tree(K: torch.Tensor, nodes: torch.Tensor | None = None, value_bound: int = 16,
+def build_tree(K: torch.Tensor, tree: torch.Tensor | None = None, value_bound: int = 16,
                dev_err: torch.Tensor | None = None) -> torch.Tensor:
-    """K int8 [B,H,n,d] -> level-major int32 tree [B,H,n-1,d]."""
+    """K int8 [B,H,n,d] -> the tree, uint8 [B,H,tree_bytes(n,d,value_bound)] (the block
+    layout of include/alhr.h: int16 rows for the narrow levels, int32 above)."""
     B, H, n, d = K.shape
     _want(K, torch.int8, (B, H, n, d), "K")
-    if nodes is None:
-        nodes = torch.empty((B, H, n - 1, d), dtype=torch.int32, device=K.device)
-    _want(nodes, torch.int32, (B, H, n - 1, d), "nodes")
+    tb = tree_bytes(n, d, value_bound)
+    if tree is None:
+        tree = torch.empty((B, H, tb), dtype=torch.uint8, device=K.device)
+    _want(tree, torch.uint8, (B, H, tb), "tree")
     dims = make_dims(None, K, value_bound=value_bound)
-    _check(lib().alhr_build_tree(ctypes.byref(dims), _ptr(K), _ptr(nodes), _ptr(dev_err),
+    _check(lib().alhr_build_tree(ctypes.byref(dims), _ptr(K), _ptr(tree), _ptr(dev_err),
                                  _stream(K.device)), "alhr_build_tree")
+    return tree
+
+
+def tree_unpack(tree: torch.Tensor, n: int, d: int, value_bound: int = 16) -> torch.Tensor:
+    """The tree as plain level-major int32 rows [B,H,n-1,d] (alhr_tree_unpack)."""
+    B, H, tb = tree.shape
+    _want(tree, torch.uint8, (B, H, tree_bytes(n, d, value_bound)), "tree")
+    nodes = torch.empty((B, H, n - 1, d), dtype=torch.int32, device=tree.device)
+    dims = Dims(B, H, n, d, 0, 0, 16, 96, 0, value_bound)
+    _check(lib().alhr_tree_unpack(ctypes.byref(dims), _ptr(tree), _ptr(nodes),
+                                  _stream(tree.device)), "alhr_tree_unpack")
     return nodes
 
 
-def predict_budget(Q, K, nodes, W, q_start=0, window=16, max_keys=96, score_bits=0,
+def predict_budget(Q, K, tree, W, q_start=0, window=16, max_keys=96, score_bits=0,
                    value_bound=16, budget=None, dev_err=None) -> torch.Tensor:
     dims = make_dims(Q, K, q_start, window, max_keys, score_bits, value_bound)
     B, H, nq, d = Q.shape
@@ -128,22 +160,22 @@ def predict_budget(Q, K, nodes, W, q_start=0, window=16, max_keys=96, score_bits
     _want(Q, torch.int8, (B, H, nq, d), "Q")
     _want(W, torch.int8, (32, 2 * d), "W")
     _want(budget, torch.int32, (B, H, nq), "budget")
-    _check(lib().alhr_predict_budget(ctypes.byref(dims), _ptr(Q), _ptr(K), _ptr(nodes), _ptr(W),
+    _check(lib().alhr_predict_budget(ctypes.byref(dims), _ptr(Q), _ptr(K), _ptr(tree), _ptr(W),
                                      _ptr(budget), _ptr(dev_err), _stream(Q.device)),
            "alhr_predict_budget")
     return budget
 
 
-def route(Q, K, nodes, budget, q_start=0, window=16, max_keys=96, score_bits=0,
+def route(Q, K, tree, budget, q_start=0, window=16, max_keys=96, score_bits=0,
           value_bound=16, with_expansions=True, dev_err=None) -> dict:
     dims = make_dims(Q, K, q_start, window, max_keys, score_bits, value_bound)
     B, H, nq, d = Q.shape
     _want(budget, torch.int32, (B, H, nq), "budget")
     idx = torch.empty((B, H, nq, max_keys), dtype=torch.int32, device=Q.device)
     count = torch.empty((B, H, nq), dtype=torch.int32, device=Q.device)
-    exp = (torch.empty((B, H, nq, 2), dtype=torch.int32, device=Q.device)
+    exp = (torch.empty((B, H, nq, 3), dtype=torch.int32, device=Q.device)
            if with_expansions else None)
-    _check(lib().alhr_route(ctypes.byref(dims), _ptr(Q), _ptr(K), _ptr(nodes), _ptr(budget),
+    _check(lib().alhr_route(ctypes.byref(dims), _ptr(Q), _ptr(K), _ptr(tree), _ptr(budget),
                             _ptr(idx), _ptr(count), _ptr(exp), _ptr(dev_err), _stream(Q.device)),
            "alhr_route")
     return dict(idx=idx, count=count, expansions=exp)
@@ -163,7 +195,7 @@ def attend(Q, K, V, idx, count, q_start=0, window=16, max_keys=96, value_bound=1
     return out
 
 
-def forward(Q, K, V, nodes, W=None, budget_override=None, q_start=0, window=16, max_keys=96,
+def forward(Q, K, V, tree, W=None, budget_override=None, q_start=0, window=16, max_keys=96,
             score_bits=0, value_bound=16, out=None, want_idx=False, want_count=False,
             want_expansions=False, want_budget=False, dev_err=None) -> dict:
     """The fused path. Returns a dict with `out` and the optional outputs asked for."""
@@ -173,7 +205,7 @@ def forward(Q, K, V, nodes, W=None, budget_override=None, q_start=0, window=16, 
     _want(Q, torch.int8, (B, H, nq, d), "Q")
     _want(K, torch.int8, (B, H, K.shape[2], d), "K")
     _want(V, torch.bfloat16, K.shape, "V")
-    _want(nodes, torch.int32, (B, H, K.shape[2] - 1, d), "nodes")
+    _want(tree, torch.uint8, (B, H, tree_bytes(K.shape[2], d, value_bound)), "tree")
     if W is not None:
         _want(W, torch.int8, (32, 2 * d), "W")
     if budget_override is not None:
@@ -187,10 +219,10 @@ def forward(Q, K, V, nodes, W=None, budget_override=None, q_start=0, window=16, 
     if want_count:
         res["count"] = mk((B, H, nq))
     if want_expansions:
-        res["expansions"] = mk((B, H, nq, 2))
+        res["expansions"] = mk((B, H, nq, 3))
     if want_budget:
         res["budget"] = mk((B, H, nq))
-    _check(lib().alhr_forward(ctypes.byref(dims), _ptr(Q), _ptr(K), _ptr(V), _ptr(nodes),
+    _check(lib().alhr_forward(ctypes.byref(dims), _ptr(Q), _ptr(K), _ptr(V), _ptr(tree),
                               _ptr(W), _ptr(budget_override), _ptr(out), _ptr(res.get("idx")),
                               _ptr(res.get("count")), _ptr(res.get("expansions")),
                               _ptr(res.get("budget")), _ptr(dev_err), _stream(dev)),

@@ -75,6 +75,7 @@ alhr::QueryArgs base_args(const alhr_dims* d) {
   a.value_bound = value_bound_of(d);
   a.num_queries = int64_t(d->batch) * d->heads * d->nq;
   a.scale = float(1.0 / std::sqrt(double(d->d)));
+  a.tl = alhr::make_tree_layout(d->n, d->d, d->value_bound);
   return a;
 }
 
@@ -86,9 +87,21 @@ extern "C" {
 
 size_t alhr_tree_rows(int32_t n) { return pow2_in_range(n) ? size_t(n) - 1 : 0; }
 
-size_t alhr_tree_level_offset(int32_t n, int32_t level) {
-  if (!pow2_in_range(n) || level < 1 || level > log2_exact(n)) return size_t(-1);
-  return size_t(n) - size_t(n >> (level - 1));
+int32_t alhr_tree_narrow_levels(int32_t n, int32_t d, int32_t value_bound) {
+  if (!pow2_in_range(n) || (d != 64 && d != 128) || value_bound < 0 || value_bound > 127) return -1;
+  return alhr::make_tree_layout(n, d, value_bound).narrow;
+}
+
+size_t alhr_tree_bytes(int32_t n, int32_t d, int32_t value_bound) {
+  if (!pow2_in_range(n) || (d != 64 && d != 128) || value_bound < 0 || value_bound > 127) return 0;
+  return size_t(alhr::make_tree_layout(n, d, value_bound).block_bytes);
+}
+
+size_t alhr_tree_level_offset(int32_t n, int32_t d, int32_t value_bound, int32_t level) {
+  if (!pow2_in_range(n) || (d != 64 && d != 128) || value_bound < 0 || value_bound > 127 ||
+      level < 1 || level > log2_exact(n))
+    return size_t(-1);
+  return size_t(alhr::make_tree_layout(n, d, value_bound).level_off[level]);
 }
 
 int32_t alhr_score_bits(const alhr_dims* d) {
@@ -111,43 +124,56 @@ const char* alhr_status_string(int32_t status) {
 
 const char* alhr_build_info(void) { return "libalhr 0.1 sm_100a"; }
 
-alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, int32_t* nodes,
+alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, void* tree,
                             uint32_t* dev_err, void* stream) {
   const alhr_status s = check_common(dims);
   if (s != ALHR_OK) return s;
-  if (!K || !nodes || !aligned16(K) || !aligned16(nodes)) return ALHR_ERR_INVALID_ARG;
+  if (!K || !tree || !aligned16(K) || !aligned16(tree)) return ALHR_ERR_INVALID_ARG;
   const long long bh = (long long)dims->batch * dims->heads;
-  return from_cuda(alhr::launch_build_tree(K, nodes, bh, dims->n, dims->d, value_bound_of(dims),
-                                           dev_err, static_cast<cudaStream_t>(stream)));
+  const alhr::TreeLayout tl = alhr::make_tree_layout(dims->n, dims->d, dims->value_bound);
+  return from_cuda(alhr::launch_build_tree(K, static_cast<char*>(tree), tl, bh,
+                                           value_bound_of(dims), dev_err,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+alhr_status alhr_tree_unpack(const alhr_dims* dims, const void* tree, int32_t* nodes,
+                             void* stream) {
+  const alhr_status s = check_common(dims);
+  if (s != ALHR_OK) return s;
+  if (!tree || !nodes || !aligned16(tree) || !aligned16(nodes)) return ALHR_ERR_INVALID_ARG;
+  const long long bh = (long long)dims->batch * dims->heads;
+  const alhr::TreeLayout tl = alhr::make_tree_layout(dims->n, dims->d, dims->value_bound);
+  return from_cuda(alhr::launch_tree_unpack(static_cast<const char*>(tree), tl, bh, nodes,
+                                            static_cast<cudaStream_t>(stream)));
 }
 
 alhr_status alhr_predict_budget(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
-                                const int32_t* nodes, const int8_t* W, int32_t* budget,
+                                const void* tree, const int8_t* W, int32_t* budget,
                                 uint32_t* dev_err, void* stream) {
   alhr_status s = check_queries(dims);
   if (s != ALHR_OK) return s;
   const int bits = resolve_bits(dims, &s);
   if (s != ALHR_OK) return s;
   if (dims->nq == 0) return ALHR_OK;  // nothing to read or write
-  if (!Q || !K || !nodes || !W || !budget) return ALHR_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(nodes) || !aligned16(W)) return ALHR_ERR_INVALID_ARG;
+  if (!Q || !K || !tree || !W || !budget) return ALHR_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(tree) || !aligned16(W)) return ALHR_ERR_INVALID_ARG;
   alhr::QueryArgs a = base_args(dims);
-  a.Q = Q; a.K = K; a.nodes = nodes; a.W = W; a.budget_out = budget; a.dev_err = dev_err;
+  a.Q = Q; a.K = K; a.tree = static_cast<const char*>(tree); a.W = W; a.budget_out = budget; a.dev_err = dev_err;
   return from_cuda(alhr::launch_predict(a, dims->d, bits, static_cast<cudaStream_t>(stream)));
 }
 
 alhr_status alhr_route(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
-                       const int32_t* nodes, const int32_t* budget, int32_t* idx, int32_t* count,
+                       const void* tree, const int32_t* budget, int32_t* idx, int32_t* count,
                        int32_t* expansions, uint32_t* dev_err, void* stream) {
   alhr_status s = check_queries(dims);
   if (s != ALHR_OK) return s;
   const int bits = resolve_bits(dims, &s);
   if (s != ALHR_OK) return s;
   if (dims->nq == 0) return ALHR_OK;  // nothing to read or write
-  if (!Q || !K || !nodes || !budget || !idx || !count) return ALHR_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(nodes)) return ALHR_ERR_INVALID_ARG;
+  if (!Q || !K || !tree || !budget || !idx || !count) return ALHR_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(tree)) return ALHR_ERR_INVALID_ARG;
   alhr::QueryArgs a = base_args(dims);
-  a.Q = Q; a.K = K; a.nodes = nodes; a.budget_in = budget;
+  a.Q = Q; a.K = K; a.tree = static_cast<const char*>(tree); a.budget_in = budget;
   a.idx_out = idx; a.count_out = count; a.exp_out = expansions; a.dev_err = dev_err;
   return from_cuda(alhr::launch_route(a, dims->d, bits, static_cast<cudaStream_t>(stream)));
 }
@@ -166,7 +192,7 @@ alhr_status alhr_attend(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
 }
 
 alhr_status alhr_forward(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
-                         const uint16_t* V, const int32_t* nodes, const int8_t* W,
+                         const uint16_t* V, const void* tree, const int8_t* W,
                          const int32_t* budget_override, float* out, int32_t* idx,
                          int32_t* count, int32_t* expansions, int32_t* budget_out,
                          uint32_t* dev_err, void* stream) {
@@ -175,13 +201,14 @@ alhr_status alhr_forward(const alhr_dims* dims, const int8_t* Q, const int8_t* K
   const int bits = resolve_bits(dims, &s);
   if (s != ALHR_OK) return s;
   if (dims->nq == 0) return ALHR_OK;  // nothing to read or write
-  if (!Q || !K || !V || !nodes || !out) return ALHR_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !tree || !out) return ALHR_ERR_INVALID_ARG;
   if (!W && !budget_override) return ALHR_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(nodes) || !aligned16(out))
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(tree) || !aligned16(out))
     return ALHR_ERR_INVALID_ARG;
   if (!budget_override && !aligned16(W)) return ALHR_ERR_INVALID_ARG;
   alhr::QueryArgs a = base_args(dims);
-  a.Q = Q; a.K = K; a.V = V; a.nodes = nodes; a.W = W; a.budget_in = budget_override;
+  a.Q = Q; a.K = K; a.V = V; a.tree = static_cast<const char*>(tree); a.W = W;
+  a.budget_in = budget_override;
   a.out = out; a.idx_out = idx; a.count_out = count; a.exp_out = expansions;
   a.budget_out = budget_out; a.dev_err = dev_err;
   return from_cuda(alhr::launch_forward(a, dims->d, bits, budget_override == nullptr,

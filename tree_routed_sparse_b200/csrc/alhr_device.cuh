@@ -13,6 +13,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/alhr.h"
+#include "tree_layout.h"
 
 namespace alhr {
 
@@ -22,6 +23,9 @@ constexpr int kMaxFrontier = 96;    // r <= max_keys - 1 nodes survive a step
 constexpr int kMaxCand = 192;       // a step offers at most 2 r candidates
 constexpr int kFrontSlots = kMaxFrontier / 32;
 constexpr int kWarps = 8;           // queries in flight per CTA
+#ifndef ALHR_NARROW_DP2A
+#define ALHR_NARROW_DP2A 1
+#endif
 
 template <int D>
 struct Lay {
@@ -50,7 +54,8 @@ struct QueryArgs {
   const int8_t* Q;
   const int8_t* K;
   const uint16_t* V;
-  const int32_t* nodes;
+  const char* tree;          // key tree, one block of tl.block_bytes per (b,h)
+  TreeLayout tl;
   const int8_t* W;
   const int32_t* budget_in;  // budget override / route input (nullable)
   const int32_t* idx_in;     // attend input
@@ -65,11 +70,30 @@ struct QueryArgs {
 
 __device__ __forceinline__ int sx8(int w, int byte) { return (w << (24 - 8 * byte)) >> 24; }
 
-// The query in the row-group layout: packed words (for dp4a on key rows) and the same 16
-// values sign-extended (for tree rows).
+// Byte offset of row j of tree level l (>= 1) inside a block of the layout of tree_layout.h,
+// from scalars only (levels 1 .. l-1 hold n - (n >> (l-1)) rows, the first n - (n >> narrow) of
+// them int16 rows of 2d bytes, the rest int32 rows of 4d bytes).
+template <int D>
+__device__ __forceinline__ int tree_row_offset(int n, int narrow, int level, int j) {
+  const int before = n - (n >> (level - 1));
+  if (narrow == 0) return (before + j) * 4 * D;
+  const int nar = n - (n >> narrow);
+  const bool is_narrow = level <= narrow;
+  const int off = is_narrow ? before * 2 * D : nar * 2 * D + (before - nar) * 4 * D;
+  return off + j * (is_narrow ? 2 * D : 4 * D);
+}
+
+// The query in the row-group layouts. Key rows and int32 tree rows: lane `sub` of a group holds
+// dims 4m .. 4m+3 for m = sub + TPR*v, v < 4 (qp: packed words for dp4a, qn: the same 16 values
+// sign-extended for int32 multiply-adds). int16 tree rows: the lane holds dims 8c .. 8c+7 for
+// c = sub + TPR*v, v < 2 (qw: the matching packed words for dp2a).
 struct RowQ {
   int qp[4];
   int qn[16];
+  int qw[4];
+#if !ALHR_NARROW_DP2A
+  int qn16[16];
+#endif
 };
 
 template <int D>
@@ -82,11 +106,81 @@ __device__ __forceinline__ void load_rowq(const int8_t* qrow, int sub, RowQ& q) 
 #pragma unroll
     for (int e = 0; e < 4; ++e) q.qn[4 * v + e] = sx8(q.qp[v], e);
   }
+  const int2* p2 = reinterpret_cast<const int2*>(qrow) + sub;
+#pragma unroll
+  for (int v = 0; v < 2; ++v) {
+    const int2 t = __ldg(p2 + TPR * v);
+    q.qw[2 * v] = t.x;
+    q.qw[2 * v + 1] = t.y;
+#if !ALHR_NARROW_DP2A
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      q.qn16[8 * v + e] = sx8(t.x, e);
+      q.qn16[8 * v + 4 + e] = sx8(t.y, e);
+    }
+#endif
+  }
+}
+
+// An int16 tree row (2d bytes) in its row-group layout: two 16-byte loads per lane, 8 words of
+// two int16 each.
+template <int D>
+__device__ __forceinline__ void ld_tree16(const char* row, int sub, int (&w)[8]) {
+  constexpr int TPR = Lay<D>::TPR;
+  const int4* p = reinterpret_cast<const int4*>(row) + sub;
+#pragma unroll
+  for (int v = 0; v < 2; ++v) {
+    const int4 t = __ldg(p + TPR * v);
+    w[4 * v + 0] = t.x;
+    w[4 * v + 1] = t.y;
+    w[4 * v + 2] = t.z;
+    w[4 * v + 3] = t.w;
+  }
+}
+
+// q . row over the lane's 16 dims of an int16 row: 8 two-way int16 x int8 dot products.
+__device__ __forceinline__ int dot_tree16(const RowQ& q, const int (&w)[8]) {
+  int s = 0;
+#if ALHR_NARROW_DP2A
+  // two independent accumulator chains (the intrinsic is not reassociated by the compiler)
+  int t = 0;
+#pragma unroll
+  for (int v = 0; v < 2; ++v) {
+    s = __dp2a_lo(w[4 * v + 0], q.qw[2 * v], s);
+    t = __dp2a_hi(w[4 * v + 1], q.qw[2 * v], t);
+    s = __dp2a_lo(w[4 * v + 2], q.qw[2 * v + 1], s);
+    t = __dp2a_hi(w[4 * v + 3], q.qw[2 * v + 1], t);
+  }
+  s += t;
+#else
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    s += ((w[k] << 16) >> 16) * q.qn16[2 * k];
+    s += (w[k] >> 16) * q.qn16[2 * k + 1];
+  }
+#endif
+  return s;
+}
+
+// An int16 tree row read in the int32 row layout (dims 4m .. 4m+3, m = sub + TPR*v), widened;
+// used where rows of different widths are summed (the causal key sum).
+template <int D>
+__device__ __forceinline__ void ld_tree16_as32(const char* row, int sub, int (&x)[16]) {
+  constexpr int TPR = Lay<D>::TPR;
+  const uint2* p = reinterpret_cast<const uint2*>(row) + sub;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const uint2 t = __ldg(p + TPR * v);
+    x[4 * v + 0] = int(t.x << 16) >> 16;
+    x[4 * v + 1] = int(t.x) >> 16;
+    x[4 * v + 2] = int(t.y << 16) >> 16;
+    x[4 * v + 3] = int(t.y) >> 16;
+  }
 }
 
 // A tree row (int32) in the row-group layout.
 template <int D>
-__device__ __forceinline__ void ld_tree(const int32_t* row, int sub, int (&x)[16]) {
+__device__ __forceinline__ void ld_tree(const char* row, int sub, int (&x)[16]) {
   constexpr int TPR = Lay<D>::TPR;
   const int4* p = reinterpret_cast<const int4*>(row) + sub;
 #pragma unroll
@@ -260,7 +354,8 @@ struct WarpBuf {
   S cscore[kMaxCand];
   int xdesc[kMaxFrontier];   // nodes expanded this step
   S xscore[kMaxFrontier];
-  int xrow[kMaxFrontier];    // element offset of each expanded node's left child row
+  int xrow[kMaxFrontier];    // byte offset of each expanded node's left child row (tree
+                             // block or key rows of the head)
   S xleft[kMaxFrontier];     // score of that left child
   int selk[kMaxKeys];        // the selected keys and their softmax weights
   float selp[kMaxKeys];

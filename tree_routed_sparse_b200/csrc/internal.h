@@ -4,13 +4,18 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "tree_layout.h"
+
 namespace alhr {
 
 struct QueryArgs;
 
 // Tree build: levels 1..log2 n of every (b,h) block (see tree_build.cu).
-cudaError_t launch_build_tree(const int8_t* K, int32_t* nodes, long long bh, int n, int d,
+cudaError_t launch_build_tree(const int8_t* K, char* tree, const TreeLayout& tl, long long bh,
                               int value_bound, uint32_t* dev_err, cudaStream_t st);
+// The tree as plain int32 rows, level-major (see tree_build.cu).
+cudaError_t launch_tree_unpack(const char* tree, const TreeLayout& tl, long long bh,
+                               int32_t* nodes, cudaStream_t st);
 
 // Warp-per-query kernels (see query_kernels.cu).
 cudaError_t launch_forward(const QueryArgs& a, int d, int score_bits, bool predict,

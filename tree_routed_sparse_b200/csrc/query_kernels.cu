@@ -60,10 +60,10 @@ constexpr int min_blocks_per_sm() { return sizeof(S) == 4 ? 3 : 2; }
 template <typename S, int D>
 constexpr int tree_rows_in_flight() { return (sizeof(S) == 4 && D == 64) ? 2 : 1; }
 
-// One pass over expanded nodes whose left child is a tree row: each row group loads US rows
-// (US in flight per lane) and leaves their scores in xleft.
+// One pass over expanded nodes whose left child is an int32 tree row: each row group loads US
+// rows (US in flight per lane) and leaves their scores in xleft.
 template <int US, typename S, int D>
-__device__ __forceinline__ void tree_child_pass(WarpBuf<S>& B, const int32_t* Nh, const RowQ& q,
+__device__ __forceinline__ void tree_child_pass(WarpBuf<S>& B, const char* Th, const RowQ& q,
                                                 int base, int end, int grp, int sub) {
   constexpr int RPI = Lay<D>::RPI;
   constexpr int TPR = Lay<D>::TPR;
@@ -72,7 +72,7 @@ __device__ __forceinline__ void tree_child_pass(WarpBuf<S>& B, const int32_t* Nh
   for (int u = 0; u < US; ++u) {
     const int xi = base + u * RPI + grp;
     if (xi < end) {
-      ld_tree<D>(Nh + B.xrow[xi], sub, x[u]);
+      ld_tree<D>(Th + B.xrow[xi], sub, x[u]);
     } else {
 #pragma unroll
       for (int j = 0; j < 16; ++j) x[u][j] = 0;
@@ -86,6 +86,45 @@ __device__ __forceinline__ void tree_child_pass(WarpBuf<S>& B, const int32_t* Nh
   }
 }
 
+// One pass over expanded nodes whose left child is a tree row, the list ordered [int32 rows |
+// int16 rows] with `nw` int32 rows. Each row group takes US rows: the int16 rows' loads are
+// issued first, then the (few, upper-level) int32 rows are loaded and scored while those are in
+// flight, then the int16 rows are scored with two-way dp2a. Scores go to xleft.
+template <int US, typename S, int D>
+__device__ __forceinline__ void child_pass(WarpBuf<S>& B, const char* Th, const RowQ& q, int base,
+                                           int nw, int end, int grp, int sub) {
+  constexpr int RPI = Lay<D>::RPI;
+  constexpr int TPR = Lay<D>::TPR;
+  int w[US][8];
+#pragma unroll
+  for (int u = 0; u < US; ++u) {
+    const int xi = base + u * RPI + grp;
+    if (xi >= nw && xi < end) {
+      ld_tree16<D>(Th + B.xrow[xi], sub, w[u]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) w[u][j] = 0;
+    }
+  }
+  S wide[US];
+#pragma unroll
+  for (int u = 0; u < US; ++u) {
+    const int xi = base + u * RPI + grp;
+    wide[u] = 0;
+    if (xi < nw) {
+      int x[16];
+      ld_tree<D>(Th + B.xrow[xi], sub, x);
+      wide[u] = dot_tree<S>(q, x);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < US; ++u) {
+    const int xi = base + u * RPI + grp;
+    const S left = group_sum<S, TPR>(xi < nw ? wide[u] : S(dot_tree16(q, w[u])));
+    if (xi < end && sub == 0) B.xleft[xi] = left;
+  }
+}
+
 template <typename S, int D, int MODE>
 __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_kernel(const QueryArgs a) {
   constexpr int TPR = Lay<D>::TPR;
@@ -94,6 +133,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
   constexpr bool kUsesW = (MODE == kForwardPredict || MODE == kPredictOnly);
   constexpr bool kDescend = (MODE != kPredictOnly);
   constexpr bool kAttend = (MODE == kForwardPredict || MODE == kForwardOverride);
+  constexpr bool kNarrow = (D == 128);  // int16 tree levels exist (see tree_layout.h)
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
   constexpr int GS = WLayout<D>::g_stride;
@@ -120,13 +160,15 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
   WarpBuf<S>& B = wbuf[warp];
   const int n = a.n;
   const int w = a.window;
+  const long long tree_block = a.tl.block_bytes;
+  const int narrow = kNarrow ? a.tl.narrow : 0;  // int16 levels 1 .. narrow (d = 128 only)
   const long long stride = (long long)gridDim.x * kWarps;
 
   for (long long qi = (long long)blockIdx.x * kWarps + warp; qi < a.num_queries; qi += stride) {
     const long long bh = qi / a.nq;
     const int i = a.q_start + int(qi - bh * a.nq);
     const int8_t* Kh = a.K + bh * (long long)n * D;
-    const int32_t* Nh = a.nodes + bh * (long long)(n - 1) * D;
+    const char* Th = a.tree + bh * tree_block;
 
     RowQ q;
     load_rowq<D>(a.Q + qi * D, sub, q);
@@ -184,7 +226,9 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
         if (active) {
           if (lvl > 0) {
             int x[16];
-            ld_tree<D>(Nh + (level_row(n, lvl) + (st >> lvl)) * D, sub, x);
+            const char* row = Th + tree_row_offset<D>(n, narrow, lvl, st >> lvl);
+            if (kNarrow && lvl <= narrow) ld_tree16_as32<D>(row, sub, x);
+            else ld_tree<D>(row, sub, x);
 #pragma unroll
             for (int j = 0; j < 16; ++j) G[j] += x[j];
             sc = dot_tree<S>(q, x);
@@ -243,7 +287,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
     }
 
     // ---- 3. descent of the past-only forest
-    int nf = 0, exp_hi = 0, exp_l1 = 0;
+    int nf = 0, exp_hi = 0, exp_l1 = 0, exp_wide = 0;
     if (kDescend && r > 0) {  // r > 0 implies i >= w, i.e. M > 0
       // roots not yet scored: the blocks of [0, M) below the shared ones
       const unsigned rest = Mu & low_mask;
@@ -262,14 +306,18 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
         const int st = desc_start(pd);
         S sc = 0;
         if (active) {
-          if (lvl > 0) {
-            int x[16];
-            ld_tree<D>(Nh + (level_row(n, lvl) + (st >> lvl)) * D, sub, x);
-            sc = dot_tree<S>(q, x);
-          } else {
+          if (lvl == 0) {
             int xp[4];
             ld_key<D>(Kh + (long long)st * D, sub, xp);
             sc = S(dot_key(q, xp));
+          } else if (!kNarrow || lvl > narrow) {
+            int x[16];
+            ld_tree<D>(Th + tree_row_offset<D>(n, narrow, lvl, st >> lvl), sub, x);
+            sc = dot_tree<S>(q, x);
+          } else {
+            int w[8];
+            ld_tree16<D>(Th + tree_row_offset<D>(n, narrow, lvl, st >> lvl), sub, w);
+            sc = S(dot_tree16(q, w));
           }
         }
         sc = group_sum<S, TPR>(sc);
@@ -282,61 +330,68 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
 
       for (int step = 0; step < 32; ++step) {
         __syncwarp();
+        // classify the frontier: keys stay; nodes to expand by the width of their left child's
+        // row: int32 tree row (level - 1 > narrow), int16 tree row, or key (level 1)
         int fd[kFrontSlots];
         S fs[kFrontSlots];
-        bool hi[kFrontSlots], l1[kFrontSlots], leaf[kFrontSlots];
-        unsigned bh_[kFrontSlots], b1_[kFrontSlots], bl_[kFrontSlots];
-        int nhi = 0, nl1 = 0, nl = 0;
+        int cat[kFrontSlots];  // 0 none, 1 key, 2 wide child, 3 narrow child, 4 key child
+        unsigned bl_[kFrontSlots], bw_[kFrontSlots], bn_[kFrontSlots], bk_[kFrontSlots];
+        int nl = 0, nw = 0, nn = 0, nk = 0;
 #pragma unroll
         for (int s = 0; s < kFrontSlots; ++s) {
-          hi[s] = l1[s] = leaf[s] = false;
-          bh_[s] = b1_[s] = bl_[s] = 0u;
+          cat[s] = 0;
+          bl_[s] = bw_[s] = bn_[s] = bk_[s] = 0u;
           fd[s] = 0;
           fs[s] = S(0);
           if (32 * s < nf) {  // warp-uniform: only the slots the frontier occupies
             const int e = lane + 32 * s;
-            const bool ok = e < nf;
-            fd[s] = ok ? B.cdesc[e] : 0;
-            fs[s] = ok ? B.cscore[e] : S(0);
-            const int lv = desc_level(fd[s]);
-            hi[s] = ok && lv >= 2;
-            l1[s] = ok && lv == 1;
-            leaf[s] = ok && lv == 0;
-            bh_[s] = __ballot_sync(kFull, hi[s]);
-            b1_[s] = __ballot_sync(kFull, l1[s]);
-            bl_[s] = __ballot_sync(kFull, leaf[s]);
-            nhi += __popc(bh_[s]);
-            nl1 += __popc(b1_[s]);
+            if (e < nf) {
+              fd[s] = B.cdesc[e];
+              fs[s] = B.cscore[e];
+              const int lv = desc_level(fd[s]);
+              cat[s] = lv == 0 ? 1 : (lv == 1 ? 4 : ((!kNarrow || lv - 1 > narrow) ? 2 : 3));
+            }
+            bl_[s] = __ballot_sync(kFull, cat[s] == 1);
+            bw_[s] = __ballot_sync(kFull, cat[s] == 2);
+            if constexpr (kNarrow) bn_[s] = __ballot_sync(kFull, cat[s] == 3);
+            bk_[s] = __ballot_sync(kFull, cat[s] == 4);
             nl += __popc(bl_[s]);
+            nw += __popc(bw_[s]);
+            nn += __popc(bn_[s]);
+            nk += __popc(bk_[s]);
           }
         }
-        const int nx = nhi + nl1;
+        const int nhi = nw + nn;  // tree-row children
+        const int nx = nhi + nk;
         if (nx == 0) break;
         exp_hi += nhi;
-        exp_l1 += nl1;
+        exp_l1 += nk;
+        exp_wide += nw;
         __syncwarp();
         {
-          // leaves stay candidates; expanded nodes go to the x lists with their left child's
-          // row offset (computed once per node here, not once per lane in the passes)
+          // keys stay candidates; expanded nodes go to the x lists ([wide | narrow | key]) with
+          // the byte offset of their left child's row, computed once per node here
           const unsigned below = lanemask_lt(lane);
-          int oh = 0, o1 = nhi, ol = 0;
+          int ow = 0, on = nw, ok = nhi, ol = 0;
 #pragma unroll
           for (int s = 0; s < kFrontSlots; ++s) {
-            if (hi[s] || l1[s]) {
-              const int pos = hi[s] ? oh + __popc(bh_[s] & below) : o1 + __popc(b1_[s] & below);
+            if (cat[s] >= 2) {
+              const int pos = cat[s] == 2 ? ow + __popc(bw_[s] & below)
+                                          : (cat[s] == 3 ? on + __popc(bn_[s] & below)
+                                                         : ok + __popc(bk_[s] & below));
               const int cl = desc_level(fd[s]) - 1;
               const int st = desc_start(fd[s]);
               B.xdesc[pos] = fd[s];
               B.xscore[pos] = fs[s];
-              B.xrow[pos] = hi[s] ? int(level_row(n, cl) + (st >> cl)) * D : st * D;
-            }
-            if (leaf[s]) {
+              B.xrow[pos] = cat[s] == 4 ? st * D : tree_row_offset<D>(n, narrow, cl, st >> cl);
+            } else if (cat[s] == 1) {
               const int pos = ol + __popc(bl_[s] & below);
               B.cdesc[pos] = fd[s];
               B.cscore[pos] = fs[s];
             }
-            oh += __popc(bh_[s]);
-            o1 += __popc(b1_[s]);
+            ow += __popc(bw_[s]);
+            on += __popc(bn_[s]);
+            ok += __popc(bk_[s]);
             ol += __popc(bl_[s]);
           }
         }
@@ -344,10 +399,12 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
         // left children that are tree rows: U rows per group in flight, one in a last short pass
         for (int base = 0; base < nhi;) {
           if (U > 1 && nhi - base > RPI) {
-            tree_child_pass<U, S, D>(B, Nh, q, base, nhi, grp, sub);
+            if constexpr (kNarrow) child_pass<U, S, D>(B, Th, q, base, nw, nhi, grp, sub);
+            else tree_child_pass<U, S, D>(B, Th, q, base, nhi, grp, sub);
             base += U * RPI;
           } else {
-            tree_child_pass<1, S, D>(B, Nh, q, base, nhi, grp, sub);
+            if constexpr (kNarrow) child_pass<1, S, D>(B, Th, q, base, nw, nhi, grp, sub);
+            else tree_child_pass<1, S, D>(B, Th, q, base, nhi, grp, sub);
             base += RPI;
           }
         }
@@ -389,8 +446,9 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
     const int count = nsel_win + nf;
     if (a.count_out && lane == 0) a.count_out[qi] = count;
     if (a.exp_out && lane == 0) {
-      a.exp_out[2 * qi] = exp_hi;
-      a.exp_out[2 * qi + 1] = exp_l1;
+      a.exp_out[3 * qi] = exp_hi;
+      a.exp_out[3 * qi + 1] = exp_l1;
+      a.exp_out[3 * qi + 2] = exp_wide;
     }
     if (a.budget_out && lane == 0) a.budget_out[qi] = budget;
     if (a.idx_out) {

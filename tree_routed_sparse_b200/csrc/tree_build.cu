@@ -6,11 +6,11 @@
 // stored.
 //
 // One CTA owns a chunk of 2^m consecutive rows of level `lin` (lin = 0: the int8 keys) of one
-// (b,h) and produces levels lin+1 .. lin+m of that chunk entirely in shared memory, so the keys
-// are read once and every tree row is written once (algorithmic bytes = K + tree). Rows are
-// moved with 16-byte vector accesses; a row of a level is contiguous with its neighbours, so
-// every warp store covers whole 32-byte sectors. Levels above the chunk height are produced by
-// further launches over the (much smaller) level-m rows.
+// (b,h) and produces levels lin+1 .. lin+m of that chunk entirely in shared memory (int32), so
+// the keys are read once and every tree row is written once (algorithmic bytes = K + tree).
+// Rows are written in the block layout of tree_layout.h: int16 for the narrow levels, int32
+// above. A level is contiguous, so the stores of a warp cover whole sectors. Levels above the
+// chunk height come from further launches over the (much smaller) level-(lin+m) rows.
 #include <cuda_runtime.h>
 
 #include "alhr_device.cuh"
@@ -23,18 +23,21 @@ namespace {
 constexpr int kTreeThreads = 256;
 constexpr int kChunkLog = 7;  // 128 input rows per CTA
 
-template <int D, bool kFromKeys>
+enum InKind : int { kFromKeys = 0, kFromNarrow = 1, kFromWide = 2 };
+
+template <int D, int IN>
 __global__ void __launch_bounds__(kTreeThreads)
-    tree_chunk_kernel(const int8_t* __restrict__ K, int32_t* __restrict__ nodes, int n, int lin,
-                      int m, int chunks_per_head, int value_bound, uint32_t* dev_err) {
+    tree_chunk_kernel(const int8_t* __restrict__ K, char* __restrict__ tree, const TreeLayout tl,
+                      int lin, int m, int chunks_per_head, int value_bound, uint32_t* dev_err) {
   extern __shared__ int4 smem4[];  // [2^m][D] int32
-  constexpr int Q4 = D / 4;                 // int4 per row
+  constexpr int Q4 = D / 4;        // int4 per row
   const long long bh = blockIdx.x / chunks_per_head;
   const int chunk = blockIdx.x - int(bh * chunks_per_head);
   const int rows = 1 << m;
-  int32_t* Nh = nodes + bh * (long long)(n - 1) * D;
+  const int n = tl.n;
+  char* Th = tree + bh * tl.block_bytes;
 
-  if constexpr (kFromKeys) {
+  if constexpr (IN == kFromKeys) {
     const int4* src = reinterpret_cast<const int4*>(K + (bh * n + (long long)chunk * rows) * D);
     bool bad = false;
     for (int k = threadIdx.x; k < rows * D / 16; k += kTreeThreads) {
@@ -52,8 +55,23 @@ __global__ void __launch_bounds__(kTreeThreads)
     }
     if (__syncthreads_or(bad) && threadIdx.x == 0 && dev_err)
       atomicOr(dev_err, ALHR_DEVERR_VALUE_RANGE);
+  } else if constexpr (IN == kFromNarrow) {
+    const int4* src = reinterpret_cast<const int4*>(Th + tl.level_off[lin] +
+                                                    (long long)chunk * rows * 2 * D);
+    for (int k = threadIdx.x; k < rows * D / 8; k += kTreeThreads) {
+      const int4 t = __ldg(src + k);  // 8 int16
+      const int wv[4] = {t.x, t.y, t.z, t.w};
+      int* dst = reinterpret_cast<int*>(smem4) + 8 * k;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        dst[2 * u] = (wv[u] << 16) >> 16;
+        dst[2 * u + 1] = wv[u] >> 16;
+      }
+    }
+    __syncthreads();
   } else {
-    const int4* src = reinterpret_cast<const int4*>(Nh + (level_row(n, lin) + (long long)chunk * rows) * D);
+    const int4* src = reinterpret_cast<const int4*>(Th + tl.level_off[lin] +
+                                                    (long long)chunk * rows * 4 * D);
     for (int k = threadIdx.x; k < rows * Q4; k += kTreeThreads) smem4[k] = __ldg(src + k);
     __syncthreads();
   }
@@ -61,9 +79,11 @@ __global__ void __launch_bounds__(kTreeThreads)
   // at most (rows/2) * Q4 outputs per level; per thread: rows*Q4/2/256
   constexpr int kMaxPer = ((1 << kChunkLog) / 2) * Q4 / kTreeThreads;
   for (int s = 1; s <= m; ++s) {
+    const int lv = lin + s;
     const int orows = rows >> s;
     const int total = orows * Q4;
-    int4* dst = reinterpret_cast<int4*>(Nh + (level_row(n, lin + s) + (long long)chunk * orows) * D);
+    const bool narrow = lv <= tl.narrow;
+    char* dst = Th + tl.level_off[lv] + (long long)chunk * orows * tl.row_bytes(lv);
     int4 res[kMaxPer > 0 ? kMaxPer : 1];
 #pragma unroll
     for (int u = 0; u < kMaxPer; ++u) {
@@ -73,7 +93,14 @@ __global__ void __launch_bounds__(kTreeThreads)
         const int4 a = smem4[(2 * row) * Q4 + col];
         const int4 b = smem4[(2 * row + 1) * Q4 + col];
         res[u] = make_int4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
-        dst[k] = res[u];
+        if (narrow) {
+          // exact: |sum| <= value_bound * 2^lv <= 32767 on a narrow level
+          const uint2 packed = make_uint2((unsigned(res[u].x) & 0xffffu) | (unsigned(res[u].y) << 16),
+                                          (unsigned(res[u].z) & 0xffffu) | (unsigned(res[u].w) << 16));
+          reinterpret_cast<uint2*>(dst)[k] = packed;
+        } else {
+          reinterpret_cast<int4*>(dst)[k] = res[u];
+        }
       }
     }
     __syncthreads();
@@ -86,21 +113,53 @@ __global__ void __launch_bounds__(kTreeThreads)
   }
 }
 
+// The tree as plain int32 rows: one thread per 4 values of an output row.
 template <int D>
-cudaError_t build_tree_d(const int8_t* K, int32_t* nodes, long long bh, int n, int value_bound,
-                         uint32_t* dev_err, cudaStream_t st) {
-  int L = 0;
-  while ((1 << L) < n) ++L;
+__global__ void __launch_bounds__(256)
+    tree_unpack_kernel(const char* __restrict__ tree, const TreeLayout tl, long long bh,
+                       int4* __restrict__ nodes) {
+  constexpr int Q4 = D / 4;
+  const int n = tl.n;
+  const long long per_block = (long long)(n - 1) * Q4;
+  const long long total = bh * per_block;
+  for (long long k = blockIdx.x * (long long)blockDim.x + threadIdx.x; k < total;
+       k += (long long)gridDim.x * blockDim.x) {
+    const long long b = k / per_block;
+    const long long rem = k - b * per_block;
+    const int r = int(rem / Q4), c = int(rem - (long long)r * Q4);
+    int l = 1;
+    while (l < tl.L && r >= n - (n >> l)) ++l;  // level l holds rows [n - (n>>(l-1)), n - (n>>l))
+    const int j = r - (n - (n >> (l - 1)));
+    const char* row = tree + b * tl.block_bytes + tl.level_off[l] + (long long)j * tl.row_bytes(l);
+    int4 v;
+    if (l <= tl.narrow) {
+      const uint2 p = __ldg(reinterpret_cast<const uint2*>(row) + c);
+      v = make_int4(int(p.x << 16) >> 16, int(p.x) >> 16, int(p.y << 16) >> 16, int(p.y) >> 16);
+    } else {
+      v = __ldg(reinterpret_cast<const int4*>(row) + c);
+    }
+    nodes[k] = v;
+  }
+}
+
+template <int D>
+cudaError_t build_tree_d(const int8_t* K, char* tree, const TreeLayout& tl, long long bh,
+                         int value_bound, uint32_t* dev_err, cudaStream_t st) {
+  const int L = tl.L;
+  const int n = tl.n;
   const size_t smem_max = size_t(1 << kChunkLog) * D * sizeof(int);
   // the opt-in above 48 KB of dynamic shared memory is a per-device function attribute
   static bool configured[128] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 128 || !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(tree_chunk_kernel<D, true>,
+    cudaError_t e = cudaFuncSetAttribute(tree_chunk_kernel<D, kFromKeys>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(tree_chunk_kernel<D, false>,
+      e = cudaFuncSetAttribute(tree_chunk_kernel<D, kFromNarrow>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(tree_chunk_kernel<D, kFromWide>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 128) configured[dev] = true;
@@ -113,11 +172,14 @@ cudaError_t build_tree_d(const int8_t* K, int32_t* nodes, long long bh, int n, i
     const size_t smem = size_t(1 << m) * D * sizeof(int);
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     if (lin == 0) {
-      tree_chunk_kernel<D, true><<<unsigned(grid), kTreeThreads, smem, st>>>(
-          K, nodes, n, lin, m, chunks, value_bound, dev_err);
+      tree_chunk_kernel<D, kFromKeys><<<unsigned(grid), kTreeThreads, smem, st>>>(
+          K, tree, tl, lin, m, chunks, value_bound, dev_err);
+    } else if (lin <= tl.narrow) {
+      tree_chunk_kernel<D, kFromNarrow><<<unsigned(grid), kTreeThreads, smem, st>>>(
+          K, tree, tl, lin, m, chunks, value_bound, dev_err);
     } else {
-      tree_chunk_kernel<D, false><<<unsigned(grid), kTreeThreads, smem, st>>>(
-          K, nodes, n, lin, m, chunks, value_bound, dev_err);
+      tree_chunk_kernel<D, kFromWide><<<unsigned(grid), kTreeThreads, smem, st>>>(
+          K, tree, tl, lin, m, chunks, value_bound, dev_err);
     }
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -128,10 +190,25 @@ cudaError_t build_tree_d(const int8_t* K, int32_t* nodes, long long bh, int n, i
 
 }  // namespace
 
-cudaError_t launch_build_tree(const int8_t* K, int32_t* nodes, long long bh, int n, int d,
+cudaError_t launch_build_tree(const int8_t* K, char* tree, const TreeLayout& tl, long long bh,
                               int value_bound, uint32_t* dev_err, cudaStream_t st) {
-  return d == 64 ? build_tree_d<64>(K, nodes, bh, n, value_bound, dev_err, st)
-                 : build_tree_d<128>(K, nodes, bh, n, value_bound, dev_err, st);
+  return tl.d == 64 ? build_tree_d<64>(K, tree, tl, bh, value_bound, dev_err, st)
+                    : build_tree_d<128>(K, tree, tl, bh, value_bound, dev_err, st);
+}
+
+cudaError_t launch_tree_unpack(const char* tree, const TreeLayout& tl, long long bh,
+                               int32_t* nodes, cudaStream_t st) {
+  const long long total = bh * (long long)(tl.n - 1) * (tl.d / 4);
+  long long blocks = (total + 255) / 256;
+  if (blocks > 148LL * 64) blocks = 148LL * 64;
+  if (blocks < 1) return cudaSuccess;
+  if (tl.d == 64)
+    tree_unpack_kernel<64><<<unsigned(blocks), 256, 0, st>>>(tree, tl, bh,
+                                                             reinterpret_cast<int4*>(nodes));
+  else
+    tree_unpack_kernel<128><<<unsigned(blocks), 256, 0, st>>>(tree, tl, bh,
+                                                              reinterpret_cast<int4*>(nodes));
+  return cudaGetLastError();
 }
 
 }  // namespace alhr

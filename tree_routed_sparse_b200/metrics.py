@@ -1,32 +1,53 @@
 """Algorithmic byte model of the ALHR inference path (what the algorithm must touch).
 
-Per query at position i of the fused forward (head dimension d, window w, M = i - w + 1 keys
-before the window, rowB(level) = d for a key row and 4d for a tree row):
+Row sizes: a key row d bytes, a tree row of a narrow level (at d = 128, value_bound * 2^l <=
+32767, stored as int16) 2d bytes, any other tree row 4d bytes. Per query at position i of the fused forward
+(window w, M = i - w + 1 keys before the window):
   q row                         d
   causal sum G_i (predictor)    the tree rows of the binary decomposition of [0, i+1)
   remaining descent roots       the blocks of [0, M) not shared with that decomposition (all of
                                 them without the predictor), only when the descent runs (r > 0)
   selected window keys          nsel_win * d
-  descent                       exp_hi * 4d + exp_l1 * d: one left-child row per expansion (the
-                                right child's score is parent - left)
+  descent                       one left-child row per expanded node (the right child's score
+                                is parent - left): exp_wide * 4d + (exp_hi - exp_wide) * 2d +
+                                exp_l1 * d
   value rows                    count * 2d (bf16)
   output row                    4d (fp32)
 plus the predictor weights (64 d) once per launch. Routed keys' rows are not re-read.
-The tree build reads K once and writes every tree row once: n d + (n-1) 4d per (b,h).
-The counts come from the run's own outputs (count, expansions, budget), which match the
-oracle's bit for bit, so the byte total is exact for the run.
+The tree build reads K once and writes every tree row once. The counters (count, the three
+expansion counters, budgets) come from the run's own outputs, which match the oracle's, so the
+byte total is exact for the run.
 """
 from __future__ import annotations
 
 import numpy as np
 
 
-def _rows_bytes(bits: np.ndarray, d: int) -> np.ndarray:
-    """Sum of rowB over the set bits of each value (bit b = a block of level b)."""
+def narrow_levels(n: int, d: int, value_bound: int = 16) -> int:
+    """At d = 128: the largest l with value_bound * 2^l <= 32767, capped at log2 n; at d = 64:
+    0 (every level int32)."""
+    if d != 128:
+        return 0
+    vb = 16 if value_bound == 0 else value_bound
+    L = int(n).bit_length() - 1
+    nl = 0
+    while nl < L and (vb << (nl + 1)) <= 32767:
+        nl += 1
+    return nl
+
+
+def row_bytes(level: int, d: int, narrow: int) -> int:
+    if level == 0:
+        return d
+    return 2 * d if level <= narrow else 4 * d
+
+
+def _rows_bytes(bits: np.ndarray, d: int, narrow: int) -> np.ndarray:
+    """Sum of row bytes over the set bits of each value (bit b = a block of level b)."""
     bits = np.asarray(bits, dtype=np.int64)
     total = np.zeros_like(bits)
     for b in range(0, 40):
-        total += ((bits >> b) & 1) * (d if b == 0 else 4 * d)
+        total += ((bits >> b) & 1) * row_bytes(b, d, narrow)
     return total
 
 
@@ -38,15 +59,17 @@ def _highest_bit(x: np.ndarray) -> np.ndarray:
     return out
 
 
-def forward_bytes(positions, d: int, window: int, count, expansions, budget,
-                  predictor: bool, max_keys: int = 96) -> int:
+def forward_bytes(positions, n: int, d: int, window: int, count, expansions, budget,
+                  predictor: bool, max_keys: int = 96, value_bound: int = 16) -> int:
     """Algorithmic bytes of one alhr_forward launch over the given queries.
 
-    positions: query positions i (any shape); count, budget: same shape; expansions: [..., 2]."""
+    positions: query positions i (any shape); count, budget: same shape; expansions: [..., 3]
+    (level >= 2 expanded, level 1 expanded, expanded with an int32 child row)."""
+    narrow = narrow_levels(n, d, value_bound)
     i = np.asarray(positions, dtype=np.int64).ravel()
     count = np.asarray(count, dtype=np.int64).ravel()
     budget = np.asarray(budget, dtype=np.int64).ravel()
-    exp = np.asarray(expansions, dtype=np.int64).reshape(-1, 2)
+    exp = np.asarray(expansions, dtype=np.int64).reshape(-1, 3)
     nwin = np.minimum(window, i + 1)
     b_eff = np.minimum(np.minimum(np.maximum(budget, 1), i + 1), max_keys)
     nsel_win = np.minimum(b_eff, nwin)
@@ -56,16 +79,23 @@ def forward_bytes(positions, d: int, window: int, count, expansions, budget,
     if predictor:
         p = np.where(M > 0, _highest_bit(A ^ M), 62)
         low = (np.int64(2) << np.minimum(p, 61)) - 1
-        g_rows = _rows_bytes(A, d)
+        g_rows = _rows_bytes(A, d, narrow)
         rest = M & low
     else:
         g_rows = np.zeros_like(i)
         rest = M
-    root_rows = np.where(r > 0, _rows_bytes(rest, d), 0)
-    per_q = (d + g_rows + root_rows + nsel_win * d + exp[:, 0] * 4 * d + exp[:, 1] * d
-             + count * 2 * d + 4 * d)
+    root_rows = np.where(r > 0, _rows_bytes(rest, d, narrow), 0)
+    descent = exp[:, 2] * 4 * d + (exp[:, 0] - exp[:, 2]) * 2 * d + exp[:, 1] * d
+    per_q = d + g_rows + root_rows + nsel_win * d + descent + count * 2 * d + 4 * d
     return int(per_q.sum()) + (64 * d if predictor else 0)
 
 
-def tree_bytes(bh: int, n: int, d: int) -> int:
-    return int(bh) * (n * d + (n - 1) * 4 * d)
+def tree_block_bytes(n: int, d: int, value_bound: int = 16) -> int:
+    narrow = narrow_levels(n, d, value_bound)
+    L = int(n).bit_length() - 1
+    return sum((n >> l) * row_bytes(l, d, narrow) for l in range(1, L + 1))
+
+
+def tree_bytes(bh: int, n: int, d: int, value_bound: int = 16) -> int:
+    """Algorithmic bytes of one tree build: K read once, every tree row written once."""
+    return int(bh) * (n * d + tree_block_bytes(n, d, value_bound))
