@@ -23,9 +23,6 @@ constexpr int kMaxFrontier = 96;    // r <= max_keys - 1 nodes survive a step
 constexpr int kMaxCand = 192;       // a step offers at most 2 r candidates
 constexpr int kFrontSlots = kMaxFrontier / 32;
 constexpr int kWarps = 8;           // queries in flight per CTA
-#ifndef ALHR_NARROW_DP2A
-#define ALHR_NARROW_DP2A 1
-#endif
 
 template <int D>
 struct Lay {
@@ -91,9 +88,6 @@ struct RowQ {
   int qp[4];
   int qn[16];
   int qw[4];
-#if !ALHR_NARROW_DP2A
-  int qn16[16];
-#endif
 };
 
 template <int D>
@@ -112,13 +106,6 @@ __device__ __forceinline__ void load_rowq(const int8_t* qrow, int sub, RowQ& q) 
     const int2 t = __ldg(p2 + TPR * v);
     q.qw[2 * v] = t.x;
     q.qw[2 * v + 1] = t.y;
-#if !ALHR_NARROW_DP2A
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      q.qn16[8 * v + e] = sx8(t.x, e);
-      q.qn16[8 * v + 4 + e] = sx8(t.y, e);
-    }
-#endif
   }
 }
 
@@ -141,7 +128,6 @@ __device__ __forceinline__ void ld_tree16(const char* row, int sub, int (&w)[8])
 // q . row over the lane's 16 dims of an int16 row: 8 two-way int16 x int8 dot products.
 __device__ __forceinline__ int dot_tree16(const RowQ& q, const int (&w)[8]) {
   int s = 0;
-#if ALHR_NARROW_DP2A
   // two independent accumulator chains (the intrinsic is not reassociated by the compiler)
   int t = 0;
 #pragma unroll
@@ -152,13 +138,6 @@ __device__ __forceinline__ int dot_tree16(const RowQ& q, const int (&w)[8]) {
     t = __dp2a_hi(w[4 * v + 3], q.qw[2 * v + 1], t);
   }
   s += t;
-#else
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    s += ((w[k] << 16) >> 16) * q.qn16[2 * k];
-    s += (w[k] >> 16) * q.qn16[2 * k + 1];
-  }
-#endif
   return s;
 }
 
@@ -364,6 +343,27 @@ struct WarpBuf {
 };
 
 // ------------------------------------------------------------------ top-r selection
+
+template <int NS>
+struct TieStarts {
+  int v[NS];  // start of each tied candidate of this lane, INT_MAX for the others
+};
+
+// Smallest U with #{tied candidates with start <= U} >= need (starts are distinct). Ties at the
+// threshold are rare, so this runs out of line and keeps the hot selection code small.
+template <int NS>
+__device__ __noinline__ int tie_cut(TieStarts<NS> ts, int need) {
+  int lo2 = 0, hi2 = 1 << 20;
+  for (int guard = 0; guard < 24 && lo2 < hi2; ++guard) {
+    const int mid = lo2 + ((hi2 - lo2) >> 1);
+    int c = 0;
+#pragma unroll
+    for (int s = 0; s < NS; ++s) c += ts.v[s] <= mid ? 1 : 0;
+    c = __reduce_add_sync(kFull, c);
+    if (c >= need) hi2 = mid; else lo2 = mid + 1;
+  }
+  return lo2;
+}
 //
 // Keeps, among the C candidates (r < C <= 32*NS), the r with the largest score, ties to the
 // lower start, and packs them into the front of the buffer. Exact: the r-th largest score T is
@@ -424,17 +424,10 @@ __device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int
   }
   int U = 0x7fffffff;
   if (!exact && need < eq) {
-    // smallest U with #{score == T and start <= U} >= need
-    int lo2 = 0, hi2 = 1 << 20;
-    for (int guard = 0; guard < 24 && lo2 < hi2; ++guard) {
-      const int mid = lo2 + ((hi2 - lo2) >> 1);
-      int c = 0;
+    TieStarts<NS> ts;
 #pragma unroll
-      for (int s = 0; s < NS; ++s) c += (sc[s] == T && desc_start(ds[s]) <= mid) ? 1 : 0;
-      c = __reduce_add_sync(kFull, c);
-      if (c >= need) hi2 = mid; else lo2 = mid + 1;
-    }
-    U = lo2;
+    for (int s = 0; s < NS; ++s) ts.v[s] = sc[s] == T ? desc_start(ds[s]) : 0x7fffffff;
+    U = tie_cut<NS>(ts, need);
   }
   __syncwarp();
   int base = 0;
@@ -455,9 +448,9 @@ __device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int
 template <typename S>
 __device__ __forceinline__ void select_top_r(WarpBuf<S>& B, int C, int r, int lane) {
   __syncwarp();
-  if (C <= 64) select_top_r_ns<S, 2>(B, C, r, lane);
-  else if (C <= 96) select_top_r_ns<S, 3>(B, C, r, lane);
-  else if (C <= 128) select_top_r_ns<S, 4>(B, C, r, lane);
+  // two instantiations only: the fused kernel is large enough that instruction-cache misses
+  // cost more than the spare slot comparisons (measured)
+  if (C <= 96) select_top_r_ns<S, 3>(B, C, r, lane);
   else select_top_r_ns<S, 6>(B, C, r, lane);
 }
 

@@ -125,6 +125,25 @@ __device__ __forceinline__ void child_pass(WarpBuf<S>& B, const char* Th, const 
   }
 }
 
+// The selection in ascending order, -1 padded: the routed keys (all below the window) sorted by
+// rank counting, then the window keys. Out of line: only the route outputs ask for it.
+template <typename S>
+__device__ __noinline__ void write_selection(const WarpBuf<S>& B, int nf, int nsel_win, int i,
+                                             int32_t* io, int max_keys, int lane) {
+#pragma unroll
+  for (int s = 0; s < kFrontSlots; ++s) {
+    const int e = lane + 32 * s;
+    if (e < nf) {
+      const int st = desc_start(B.cdesc[e]);
+      int rank = 0;
+      for (int f = 0; f < nf; ++f) rank += desc_start(B.cdesc[f]) < st ? 1 : 0;
+      io[rank] = st;
+    }
+  }
+  if (lane < nsel_win) io[nf + nsel_win - 1 - lane] = i - lane;
+  for (int pp = nf + nsel_win + lane; pp < max_keys; pp += 32) io[pp] = -1;
+}
+
 template <typename S, int D, int MODE>
 __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_kernel(const QueryArgs a) {
   constexpr int TPR = Lay<D>::TPR;
@@ -396,17 +415,11 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
           }
         }
         __syncwarp();
-        // left children that are tree rows: U rows per group in flight, one in a last short pass
-        for (int base = 0; base < nhi;) {
-          if (U > 1 && nhi - base > RPI) {
-            if constexpr (kNarrow) child_pass<U, S, D>(B, Th, q, base, nw, nhi, grp, sub);
-            else tree_child_pass<U, S, D>(B, Th, q, base, nhi, grp, sub);
-            base += U * RPI;
-          } else {
-            if constexpr (kNarrow) child_pass<1, S, D>(B, Th, q, base, nw, nhi, grp, sub);
-            else tree_child_pass<1, S, D>(B, Th, q, base, nhi, grp, sub);
-            base += RPI;
-          }
+        // left children that are tree rows: U rows per group in flight (a single pass body:
+        // a separate short tail pass measured slower through instruction-cache misses)
+        for (int base = 0; base < nhi; base += U * RPI) {
+          if constexpr (kNarrow) child_pass<U, S, D>(B, Th, q, base, nw, nhi, grp, sub);
+          else tree_child_pass<U, S, D>(B, Th, q, base, nhi, grp, sub);
         }
         // left children that are keys
         for (int base = nhi; base < nx; base += RPI) {
@@ -451,21 +464,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
       a.exp_out[3 * qi + 2] = exp_wide;
     }
     if (a.budget_out && lane == 0) a.budget_out[qi] = budget;
-    if (a.idx_out) {
-      int32_t* io = a.idx_out + qi * a.max_keys;
-#pragma unroll
-      for (int s = 0; s < kFrontSlots; ++s) {
-        const int e = lane + 32 * s;
-        if (e < nf) {
-          const int st = desc_start(B.cdesc[e]);
-          int rank = 0;
-          for (int f = 0; f < nf; ++f) rank += desc_start(B.cdesc[f]) < st ? 1 : 0;
-          io[rank] = st;
-        }
-      }
-      if (lane < nsel_win) io[nf + nsel_win - 1 - lane] = i - lane;
-      for (int pp = count + lane; pp < a.max_keys; pp += 32) io[pp] = -1;
-    }
+    if (a.idx_out) write_selection<S>(B, nf, nsel_win, i, a.idx_out + qi * a.max_keys, a.max_keys, lane);
 
     // ---- 4. exact attention over window + routed keys
     if constexpr (kAttend) {
