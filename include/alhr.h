@@ -123,6 +123,24 @@ ALHR_API const char* alhr_status_string(int32_t status);
 ALHR_API const char* alhr_build_info(void);
 
 /*
+ * Launch shape of the per-query kernels (alhr_forward, alhr_route, alhr_predict_budget), a
+ * process-wide setting. Trees, budgets, index sets, counts and expansions are identical in every
+ * mode; outputs may differ in the last bits of fp32 (another summation order of the value rows).
+ *   ALHR_LAUNCH_AUTO (default): latency shape when a launch has at most 8 queries per SM of the
+ *     device (decode and other small launches), throughput shape above.
+ *   ALHR_LAUNCH_THROUGHPUT: several CTAs per SM, one or two tree rows in flight per lane group.
+ *   ALHR_LAUNCH_LATENCY: one CTA per SM, up to eight rows in flight per lane group.
+ * alhr_set_launch_mode returns ALHR_ERR_INVALID_ARG (and changes nothing) for any other value.
+ */
+typedef enum {
+  ALHR_LAUNCH_AUTO = 0,
+  ALHR_LAUNCH_THROUGHPUT = 1,
+  ALHR_LAUNCH_LATENCY = 2
+} alhr_launch_mode;
+ALHR_API alhr_status alhr_set_launch_mode(int32_t mode);
+ALHR_API int32_t alhr_get_launch_mode(void);
+
+/*
  * alhr_build_tree -- the static key tree [README §Inference stage, first paragraph: the tree
  * is built on the key matrix and stored, once per layer; README opening paragraph: every
  * branch is indexed by the sum of all key vectors beneath it].

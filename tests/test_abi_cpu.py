@@ -68,6 +68,25 @@ def test_tree_layout_helpers(A):
     assert b"sm_100a" in L.alhr_build_info()
 
 
+def test_launch_mode_setting(A):
+    """The process-wide launch shape: default auto, the three documented values accepted,
+    anything else refused without changing the setting."""
+    L = A.lib()
+    assert A.get_launch_mode() == "auto"
+    try:
+        for name in ("latency", "throughput", "auto"):
+            A.set_launch_mode(name)
+            assert A.get_launch_mode() == name
+        A.set_launch_mode("latency")
+        for bad in (-1, 3, 1 << 30):
+            assert L.alhr_set_launch_mode(bad) == 1
+            assert A.get_launch_mode() == "latency"
+        with pytest.raises(ValueError):
+            A.set_launch_mode("fast")
+    finally:
+        A.set_launch_mode("auto")
+
+
 @pytest.mark.parametrize("n,d,vb", [(16384, 64, 16), (262144, 128, 16), (1024, 128, 127),
                                     (4096, 128, 3), (2, 64, 0), (2, 128, 0), (1 << 20, 128, 1)])
 def test_tree_layout_matches_documented_layout(A, n, d, vb):

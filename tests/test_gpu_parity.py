@@ -31,6 +31,15 @@ def synth():
     return S
 
 
+@pytest.fixture(params=["throughput", "latency"])
+def shape(request, alhr):
+    """Both launch shapes of the per-query kernels on the same small inputs (the automatic choice
+    would pick the latency shape for all of them)."""
+    alhr.set_launch_mode(request.param)
+    yield request.param
+    alhr.set_launch_mode("auto")
+
+
 def _to(inp, device):
     return {k: (None if v is None else v.to(device)) for k, v in inp.items()}
 
@@ -105,7 +114,7 @@ def test_tree_extremes_and_range_flag(alhr):
 # ------------------------------------------------------------------ fused forward, small cases
 
 
-def test_forward_tiny_prefill_all_queries(alhr, synth):
+def test_forward_tiny_prefill_all_queries(alhr, synth, shape):
     """1 x 1 x 1024, d=64, fixed budget min(i+1, 32): every query against the oracle."""
     wl = synth.WORKLOADS["tiny_prefill_n1024"]
     inp = synth.make_inputs(wl, "cuda")
@@ -121,7 +130,7 @@ def test_forward_tiny_prefill_all_queries(alhr, synth):
                                            (1024, 64, 1, 96, 32), (512, 64, 32, 96, 0),
                                            (256, 128, 5, 7, 0), (64, 64, 16, 96, 64),
                                            (2048, 128, 16, 50, 0)])
-def test_forward_predicted_budget_all_queries(alhr, synth, n, d, w, mk, bits):
+def test_forward_predicted_budget_all_queries(alhr, synth, n, d, w, mk, bits, shape):
     wl = synth.WORKLOADS["prefill_b4h8_n4096"].replace(
         batch=2, heads=2, n=n, d=d, nq=n, window=w, max_keys=mk, score_bits=bits, seed=n + d + w)
     inp = synth.make_inputs(wl, "cuda")
@@ -134,7 +143,7 @@ def test_forward_predicted_budget_all_queries(alhr, synth, n, d, w, mk, bits):
     assert res["dev_err"] == 0
 
 
-def test_forward_ties_everywhere(alhr, synth):
+def test_forward_ties_everywhere(alhr, synth, shape):
     """All keys equal: every candidate score ties, so only the lower-start rule decides."""
     wl = synth.WORKLOADS["prefill_b4h8_n4096"].replace(batch=1, heads=2, n=512, nq=512)
     inp = synth.make_inputs(wl, "cuda")
@@ -146,7 +155,7 @@ def test_forward_ties_everywhere(alhr, synth):
         compare_rows(res, oracle_slice(cpu, wl, 0, h), 0, h, np.arange(512), TOL, f"h{h}")
 
 
-def test_forward_extreme_values(alhr, synth):
+def test_forward_extreme_values(alhr, synth, shape):
     wl = synth.WORKLOADS["prefill_b4h8_n4096"].replace(batch=1, heads=1, n=4096, nq=4096,
                                                        score_bits=32)
     inp = synth.make_inputs(wl, "cuda")
@@ -158,7 +167,7 @@ def test_forward_extreme_values(alhr, synth):
     compare_rows(res, oracle_slice(cpu, wl, 0, 0, rows=rows), 0, 0, rows, TOL, "extreme")
 
 
-def test_forward_budget_override_edges(alhr, synth):
+def test_forward_budget_override_edges(alhr, synth, shape):
     """Budgets below 1 are clamped and flagged; budgets above max_keys are capped."""
     wl = synth.WORKLOADS["tiny_prefill_n1024"].replace(n=256, nq=256)
     inp = synth.make_inputs(wl, "cuda")
@@ -171,7 +180,7 @@ def test_forward_budget_override_edges(alhr, synth):
     assert res["dev_err"] & alhr.DEVERR_BUDGET_LOW
 
 
-def test_decode_style_queries(alhr, synth):
+def test_decode_style_queries(alhr, synth, shape):
     """q_start > 0: the last 7 positions of a 4096-key head, int64 scores, d = 128."""
     wl = synth.WORKLOADS["decode_s64h8_n262144_d128"].replace(batch=3, heads=2, n=4096,
                                                               q_start=4089, nq=7)
@@ -187,7 +196,7 @@ def test_decode_style_queries(alhr, synth):
 
 
 @pytest.mark.parametrize("d,bits", [(64, 0), (128, 64)])
-def test_unfused_path_matches_oracle_and_fused(alhr, synth, d, bits):
+def test_unfused_path_matches_oracle_and_fused(alhr, synth, d, bits, shape):
     wl = synth.WORKLOADS["prefill_b4h8_n4096"].replace(batch=1, heads=3, n=1024, nq=1024, d=d,
                                                        score_bits=bits)
     inp = synth.make_inputs(wl, "cuda")

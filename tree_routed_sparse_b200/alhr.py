@@ -22,11 +22,12 @@ STATUS = {0: "ALHR_OK", 1: "ALHR_ERR_INVALID_ARG", 2: "ALHR_ERR_UNSUPPORTED",
 DEVERR_BUDGET_LOW = 0x1
 DEVERR_VALUE_RANGE = 0x2
 DEVERR_INDEX = 0x4
+LAUNCH_MODES = {"auto": 0, "throughput": 1, "latency": 2}
 
 EXPORTS = ["alhr_tree_rows", "alhr_tree_narrow_levels", "alhr_tree_bytes",
            "alhr_tree_level_offset", "alhr_score_bits", "alhr_status_string", "alhr_build_info",
            "alhr_build_tree", "alhr_tree_unpack", "alhr_predict_budget", "alhr_route",
-           "alhr_attend", "alhr_forward"]
+           "alhr_attend", "alhr_forward", "alhr_set_launch_mode", "alhr_get_launch_mode"]
 
 
 class AlhrError(RuntimeError):
@@ -69,8 +70,10 @@ def lib() -> ctypes.CDLL:
         L.alhr_route.argtypes = [DP, P, P, P, P, P, P, P, P, P]
         L.alhr_attend.argtypes = [DP, P, P, P, P, P, P, P, P]
         L.alhr_forward.argtypes = [DP, P, P, P, P, P, P, P, P, P, P, P, P, P]
+        L.alhr_set_launch_mode.argtypes = [I32]
+        L.alhr_get_launch_mode.argtypes, L.alhr_get_launch_mode.restype = [], I32
         for f in ("alhr_build_tree", "alhr_tree_unpack", "alhr_predict_budget", "alhr_route",
-                  "alhr_attend", "alhr_forward"):
+                  "alhr_attend", "alhr_forward", "alhr_set_launch_mode"):
             getattr(L, f).restype = I32
         _lib = L
     return _lib
@@ -79,6 +82,18 @@ def lib() -> ctypes.CDLL:
 def _check(status: int, where: str):
     if status != ALHR_OK:
         raise AlhrError(status, where)
+
+
+def set_launch_mode(mode: str) -> None:
+    """Process-wide launch shape of the per-query kernels: "auto", "throughput" or "latency"."""
+    if mode not in LAUNCH_MODES:
+        raise ValueError(f"launch mode {mode!r}: one of {sorted(LAUNCH_MODES)}")
+    _check(lib().alhr_set_launch_mode(LAUNCH_MODES[mode]), "alhr_set_launch_mode")
+
+
+def get_launch_mode() -> str:
+    code = lib().alhr_get_launch_mode()
+    return {v: k for k, v in LAUNCH_MODES.items()}[code]
 
 
 def _ptr(t):

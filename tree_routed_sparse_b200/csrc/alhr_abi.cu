@@ -124,6 +124,15 @@ const char* alhr_status_string(int32_t status) {
 
 const char* alhr_build_info(void) { return "libalhr 0.1 sm_100a"; }
 
+alhr_status alhr_set_launch_mode(int32_t mode) {
+  if (mode != ALHR_LAUNCH_AUTO && mode != ALHR_LAUNCH_THROUGHPUT && mode != ALHR_LAUNCH_LATENCY)
+    return ALHR_ERR_INVALID_ARG;
+  alhr::set_query_launch_mode(mode);
+  return ALHR_OK;
+}
+
+int32_t alhr_get_launch_mode(void) { return alhr::query_launch_mode(); }
+
 alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, void* tree,
                             uint32_t* dev_err, void* stream) {
   const alhr_status s = check_common(dims);

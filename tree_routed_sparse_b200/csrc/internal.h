@@ -24,4 +24,8 @@ cudaError_t launch_route(const QueryArgs& a, int d, int score_bits, cudaStream_t
 cudaError_t launch_predict(const QueryArgs& a, int d, int score_bits, cudaStream_t st);
 cudaError_t launch_attend(const QueryArgs& a, int d, cudaStream_t st);
 
+// Process-wide launch shape of the per-query kernels: 0 auto, 1 throughput, 2 latency.
+void set_query_launch_mode(int mode);
+int query_launch_mode();
+
 }  // namespace alhr

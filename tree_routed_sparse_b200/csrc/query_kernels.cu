@@ -17,6 +17,7 @@
 //      best r by an exact integer bisection (select_top_r);
 //   4. attention: the selected window keys are scored, routed keys keep the scores of the
 //      descent (their key rows are not read again), and the value rows are gathered.
+#include <atomic>
 #include <cuda_runtime.h>
 
 #include "alhr_device.cuh"
@@ -78,6 +79,7 @@ __device__ __forceinline__ void tree_child_pass(WarpBuf<S>& B, const char* Th, c
       for (int j = 0; j < 16; ++j) x[u][j] = 0;
     }
   }
+  if constexpr (US > 2) __syncwarp();  // latency shape: reconverge before the group sums
 #pragma unroll
   for (int u = 0; u < US; ++u) {
     const int xi = base + u * RPI + grp;
@@ -117,6 +119,7 @@ __device__ __forceinline__ void child_pass(WarpBuf<S>& B, const char* Th, const 
       wide[u] = dot_tree<S>(q, x);
     }
   }
+  if constexpr (US > 2) __syncwarp();  // latency shape: reconverge before the group sums
 #pragma unroll
   for (int u = 0; u < US; ++u) {
     const int xi = base + u * RPI + grp;
@@ -144,11 +147,38 @@ __device__ __noinline__ void write_selection(const WarpBuf<S>& B, int nf, int ns
   for (int pp = nf + nsel_win + lane; pp < max_keys; pp += 32) io[pp] = -1;
 }
 
-template <typename S, int D, int MODE>
-__global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_kernel(const QueryArgs a) {
+// Any node of the forest (a key at level 0, an int16 or int32 tree row above) as this lane's 16
+// per-dimension integers; used by the latency mode's batched passes over causal-sum rows and roots.
+template <int D, bool kNarrow>
+__device__ __forceinline__ void ld_node32(const char* Th, const int8_t* Kh, int n, int narrow,
+                                          int pd, int sub, int (&x)[16]) {
+  const int lvl = desc_level(pd);
+  const int st = desc_start(pd);
+  if (lvl == 0) {
+    int xp[4];
+    ld_key<D>(Kh + (long long)st * D, sub, xp);
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[4 * v + e] = sx8(xp[v], e);
+  } else if (kNarrow && lvl <= narrow) {
+    ld_tree16_as32<D>(Th + tree_row_offset<D>(n, narrow, lvl, st >> lvl), sub, x);
+  } else {
+    ld_tree<D>(Th + tree_row_offset<D>(n, narrow, lvl, st >> lvl), sub, x);
+  }
+}
+
+// LAT selects the latency mode, for launches with too few queries to fill the GPU (decode): every
+// warp keeps many more rows in flight per pass (registers are no constraint at one CTA per SM),
+// so a descent step takes one or two round trips to memory instead of up to ten.
+template <typename S, int D, int MODE, bool LAT>
+__global__ void __launch_bounds__(kWarps * 32, LAT ? 1 : min_blocks_per_sm<S>())
+    query_kernel(const QueryArgs a) {
   constexpr int TPR = Lay<D>::TPR;
   constexpr int RPI = Lay<D>::RPI;
-  constexpr int U = tree_rows_in_flight<S, D>();  // tree rows per group per pass
+  constexpr int U = LAT ? (D == 128 ? 8 : 4) : tree_rows_in_flight<S, D>();  // tree rows per group per pass
+  constexpr int UK = LAT ? 8 : 1;  // key rows per group per pass
+  constexpr int UV = LAT ? 8 : 2;  // value-row passes in flight
   constexpr bool kUsesW = (MODE == kForwardPredict || MODE == kPredictOnly);
   constexpr bool kDescend = (MODE != kPredictOnly);
   constexpr bool kAttend = (MODE == kForwardPredict || MODE == kForwardOverride);
@@ -235,6 +265,51 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
         B.plist[rank] = make_desc(start, b) | kFlagG | ((M > 0 && b > p) ? kFlagRoot : 0);
       }
       __syncwarp();
+      if constexpr (LAT) {
+        // All causal-sum rows in one or two round trips: UG rows per group per pass, at most
+        // NP passes (i + 1 < 2^20 has at most 20 blocks). The shared roots' scores are kept in
+        // registers and stored after the cross-group sum of G_i: with the (divergent) stores
+        // inside the pass, that sum came out wrong on sm_100a.
+        constexpr int UG = 4;
+        constexpr int NP = (kMaxLevels + UG * RPI - 1) / (UG * RPI);
+        S rsc[NP][UG];
+#pragma unroll
+        for (int ps = 0; ps < NP; ++ps) {
+          const int base = ps * UG * RPI;
+          int x[UG][16];
+#pragma unroll
+          for (int u = 0; u < UG; ++u) {
+            const int k = base + u * RPI + grp;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) x[u][j] = 0;
+            if (k < nA) ld_node32<D, kNarrow>(Th, Kh, n, narrow, B.plist[k], sub, x[u]);
+          }
+#pragma unroll
+          for (int u = 0; u < UG; ++u) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) G[j] += x[u][j];
+            rsc[ps][u] = base < nA ? group_sum<S, TPR>(dot_tree<S>(q, x[u])) : S(0);
+          }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int off = TPR; off < 32; off *= 2)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) G[j] += __shfl_xor_sync(kFull, G[j], off);
+#pragma unroll
+        for (int ps = 0; ps < NP; ++ps)
+#pragma unroll
+          for (int u = 0; u < UG; ++u) {
+            const int k = ps * UG * RPI + u * RPI + grp;
+            if (k < nA && sub == 0) {
+              const int pd = B.plist[k];
+              if (pd & kFlagRoot) {
+                B.cdesc[k] = pd & ~(kFlagRoot | kFlagG);
+                B.cscore[k] = rsc[ps][u];
+              }
+            }
+          }
+      } else
       for (int base = 0; base < nA; base += RPI) {
         const int k = base + grp;
         const bool active = k < nA;
@@ -267,10 +342,12 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
           B.cscore[k] = sc;
         }
       }
+      if constexpr (!LAT) {
 #pragma unroll
-      for (int off = TPR; off < 32; off *= 2)
+        for (int off = TPR; off < 32; off *= 2)
 #pragma unroll
-        for (int j = 0; j < 16; ++j) G[j] += __shfl_xor_sync(kFull, G[j], off);
+          for (int j = 0; j < 16; ++j) G[j] += __shfl_xor_sync(kFull, G[j], off);
+      }
 
       // ---- 2. budget predictor: group grp scores classes grp, grp+RPI, ...
       long long best = ScoreLimits<long long>::lowest;
@@ -317,6 +394,29 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
         B.plist[__popc(rest >> b) - 1] = make_desc(int((Mu >> b) << b) - (1 << b), b);
       }
       __syncwarp();
+      if constexpr (LAT) {
+        constexpr int UR = 4;
+        for (int base = 0; base < nB; base += UR * RPI) {
+          int x[UR][16];
+#pragma unroll
+          for (int u = 0; u < UR; ++u) {
+            const int k = base + u * RPI + grp;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) x[u][j] = 0;
+            if (k < nB) ld_node32<D, kNarrow>(Th, Kh, n, narrow, B.plist[k], sub, x[u]);
+          }
+          __syncwarp();  // reconverge after the per-group branches, before the group sums
+#pragma unroll
+          for (int u = 0; u < UR; ++u) {
+            const int k = base + u * RPI + grp;
+            const S sc = group_sum<S, TPR>(dot_tree<S>(q, x[u]));
+            if (k < nB && sub == 0) {
+              B.cdesc[n_common + k] = B.plist[k];
+              B.cscore[n_common + k] = sc;
+            }
+          }
+        }
+      } else
       for (int base = 0; base < nB; base += RPI) {
         const int k = base + grp;
         const bool active = k < nB;
@@ -421,13 +521,23 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
           if constexpr (kNarrow) child_pass<U, S, D>(B, Th, q, base, nw, nhi, grp, sub);
           else tree_child_pass<U, S, D>(B, Th, q, base, nhi, grp, sub);
         }
-        // left children that are keys
-        for (int base = nhi; base < nx; base += RPI) {
-          const int xi = base + grp;
-          int xp[4] = {0, 0, 0, 0};
-          if (xi < nx) ld_key<D>(Kh + B.xrow[xi], sub, xp);
-          const int left = group_sum<int, TPR>(dot_key(q, xp));
-          if (xi < nx && sub == 0) B.xleft[xi] = S(left);
+        // left children that are keys: UK rows per group in flight
+        for (int base = nhi; base < nx; base += UK * RPI) {
+          int xp[UK][4];
+#pragma unroll
+          for (int u = 0; u < UK; ++u) {
+            const int xi = base + u * RPI + grp;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) xp[u][v] = 0;
+            if (xi < nx) ld_key<D>(Kh + B.xrow[xi], sub, xp[u]);
+          }
+          if constexpr (LAT) __syncwarp();
+#pragma unroll
+          for (int u = 0; u < UK; ++u) {
+            const int xi = base + u * RPI + grp;
+            const int left = group_sum<int, TPR>(dot_key(q, xp[u]));
+            if (xi < nx && sub == 0) B.xleft[xi] = S(left);
+          }
         }
         __syncwarp();
         // both children of every expanded node, one node per lane
@@ -445,12 +555,22 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
 
     // ---- window key scores (attention only needs the selected ones)
     if constexpr (kAttend) {
-      for (int base = 0; base < nsel_win; base += RPI) {
-        const int x = base + grp;
-        int xp[4] = {0, 0, 0, 0};
-        if (x < nsel_win) ld_key<D>(Kh + (long long)(i - x) * D, sub, xp);
-        const int s = group_sum<int, TPR>(dot_key(q, xp));
-        if (x < nsel_win && sub == 0) B.winsc[x] = s;
+      for (int base = 0; base < nsel_win; base += UK * RPI) {
+        int xp[UK][4];
+#pragma unroll
+        for (int u = 0; u < UK; ++u) {
+          const int x = base + u * RPI + grp;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) xp[u][v] = 0;
+          if (x < nsel_win) ld_key<D>(Kh + (long long)(i - x) * D, sub, xp[u]);
+        }
+        if constexpr (LAT) __syncwarp();
+#pragma unroll
+        for (int u = 0; u < UK; ++u) {
+          const int x = base + u * RPI + grp;
+          const int s = group_sum<int, TPR>(dot_key(q, xp[u]));
+          if (x < nsel_win && sub == 0) B.winsc[x] = s;
+        }
       }
     }
     __syncwarp();
@@ -505,7 +625,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>()) query_ker
         }
       }
       __syncwarp();
-      gather_values<D, 2>(B.selk, B.selp, nsel_win + nf, 1.f / den, a.V + bh * (long long)n * D,
+      gather_values<D, UV>(B.selk, B.selp, nsel_win + nf, 1.f / den, a.V + bh * (long long)n * D,
                           lane, a.out + qi * D);
     }
   }
@@ -591,7 +711,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(const QueryArgs a) 
 
 namespace {
 
-constexpr int kOccSlots = 20;
+constexpr int kOccSlots = 40;
 
 // Grid size of a persistent launch: the resident CTAs of every SM, capped by the work. The
 // per-device occupancy (and the opt-in to more than 48 KB of dynamic shared memory) is
@@ -623,18 +743,42 @@ int blocks_for(KernelT kernel, int slot, size_t smem, long long queries, cudaErr
   return int(need < cap ? need : cap);
 }
 
-template <typename S, int D, int MODE>
-cudaError_t launch_query(const QueryArgs& a, cudaStream_t st) {
-  constexpr int slot = (MODE * 2 + (D == 128 ? 1 : 0)) * 2 + (sizeof(S) == 8 ? 1 : 0);
-  static_assert(slot < 16, "occupancy cache slot");
+template <typename S, int D, int MODE, bool LAT>
+cudaError_t launch_query_mode(const QueryArgs& a, cudaStream_t st) {
+  constexpr int slot = ((MODE * 2 + (D == 128 ? 1 : 0)) * 2 + (sizeof(S) == 8 ? 1 : 0)) * 2 +
+                       (LAT ? 1 : 0);
+  static_assert(slot < 32, "occupancy cache slot");
   constexpr size_t smem = QuerySmem<S, D, MODE>::bytes;
-  auto kern = query_kernel<S, D, MODE>;
+  auto kern = query_kernel<S, D, MODE, LAT>;
   cudaError_t err;
   const int blocks = blocks_for(kern, slot, smem, a.num_queries, &err);
   if (err != cudaSuccess) return err;
   if (blocks <= 0) return cudaSuccess;
   kern<<<blocks, kWarps * 32, smem, st>>>(a);
   return cudaGetLastError();
+}
+
+std::atomic<int> g_launch_mode{0};
+
+// Auto: a launch whose queries fit one warp each at one CTA per SM (8 per SM) cannot fill the
+// GPU, so it takes the latency shape; measured on B200 the throughput shape wins from about 2048
+// queries up.
+template <typename S, int D, int MODE>
+cudaError_t launch_query(const QueryArgs& a, cudaStream_t st) {
+  const int mode = g_launch_mode.load(std::memory_order_relaxed);
+  bool lat = mode == 2;
+  if (mode == 0) {
+    static thread_local int cached_dev = -1, sms = 148;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev != cached_dev) {
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      cached_dev = dev;
+    }
+    lat = a.num_queries <= (long long)sms * kWarps;
+  }
+  return lat ? launch_query_mode<S, D, MODE, true>(a, st)
+             : launch_query_mode<S, D, MODE, false>(a, st);
 }
 
 template <int MODE>
@@ -663,14 +807,17 @@ cudaError_t launch_predict(const QueryArgs& a, int d, int score_bits, cudaStream
   return dispatch_query<kPredictOnly>(a, d, score_bits, st);
 }
 
+void set_query_launch_mode(int mode) { g_launch_mode.store(mode, std::memory_order_relaxed); }
+int query_launch_mode() { return g_launch_mode.load(std::memory_order_relaxed); }
+
 cudaError_t launch_attend(const QueryArgs& a, int d, cudaStream_t st) {
   cudaError_t err;
   if (d == 64) {
-    const int blocks = blocks_for(attend_kernel<64>, 16, 0, a.num_queries, &err);
+    const int blocks = blocks_for(attend_kernel<64>, 32, 0, a.num_queries, &err);
     if (err != cudaSuccess) return err;
     attend_kernel<64><<<blocks, kWarps * 32, 0, st>>>(a);
   } else {
-    const int blocks = blocks_for(attend_kernel<128>, 17, 0, a.num_queries, &err);
+    const int blocks = blocks_for(attend_kernel<128>, 33, 0, a.num_queries, &err);
     if (err != cudaSuccess) return err;
     attend_kernel<128><<<blocks, kWarps * 32, 0, st>>>(a);
   }
