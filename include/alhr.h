@@ -156,6 +156,32 @@ ALHR_API alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, voi
                                      uint32_t* dev_err, void* stream);
 
 /*
+ * alhr_update_tree -- the tree after rows [lo, hi) of K changed, e.g. the keys of new tokens
+ * appended during decoding [README §Inference stage, first paragraph: the tree is built on the
+ * key matrix; page "ALHR把注意力变成树搜索", §"ALHR是什么：让每个Query沿树寻找Key": a new
+ * token's attention during decoding; §"接下来最该验证的不是更高压缩比": per-token decode latency
+ * is one of the figures to report].
+ *
+ * Precondition: for every (b,h), `tree` equals what alhr_build_tree wrote (or this call left)
+ * for a key matrix that differs from K at most in rows [lo, hi). Postcondition: `tree` equals
+ * alhr_build_tree(K), byte for byte. Only the rows over [lo, hi) are read and written: for
+ * hi - lo <= 64 one kernel moves every ancestor by the exact change of the level-1 sums beneath
+ * it (the old pair sum is the stored level-1 row, so no old key is needed; O(log2 n) rows per
+ * (b,h) for one key); larger ranges rebuild the 128-row chunks that cover them, level group by
+ * level group. Reads dims->batch, heads, n, d and value_bound.
+ *   K       device, int8 [batch][heads][n][d], read only (rows outside [lo, hi) too: the pair
+ *           and chunk neighbours)
+ *   tree    device, as for alhr_build_tree, updated in place
+ *   lo, hi  0 <= lo <= hi <= n, the same for every (b,h); lo == hi does nothing
+ *   dev_err device uint32 or NULL; ALHR_DEVERR_VALUE_RANGE if some |K| > value_bound in the rows
+ *           read
+ * ALHR_ERR_INVALID_ARG for a bad range or pointer. Not thread-safe against kernels reading the
+ * same tree on another stream (order them with the caller's stream or events).
+ */
+ALHR_API alhr_status alhr_update_tree(const alhr_dims* dims, const int8_t* K, void* tree,
+                                      int32_t lo, int32_t hi, uint32_t* dev_err, void* stream);
+
+/*
  * alhr_tree_unpack -- the tree as plain int32 rows: nodes[b][h][r][:] for r in [0, n-1), level l
  * at rows [n - (n >> (l-1)), n - (n >> l)) (level-major, level 1 first). Reads dims->batch,
  * heads, n, d and value_bound.

@@ -150,7 +150,14 @@ def test_entry_points_reject_bad_arguments_before_launch(A):
     assert L.alhr_route(d, fake, fake, fake, fake, null, fake, null, null, null) == 1
     assert L.alhr_attend(d, fake, fake, fake, fake, fake, null, null, null) == 1
     assert L.alhr_predict_budget(d, fake, fake, fake, null, fake, null, null) == 1
+    n = _dims(A).n
+    for lo, hi in ((-1, 1), (3, 2), (0, n + 1), (n, n + 1)):
+        assert L.alhr_update_tree(d, fake, fake, lo, hi, null, null) == 1, (lo, hi)
+    assert L.alhr_update_tree(d, null, fake, 0, 1, null, null) == 1
+    assert L.alhr_update_tree(d, fake, odd, 0, 1, null, null) == 1
+    assert L.alhr_update_tree(ctypes.byref(_dims(A, d=32)), fake, fake, 0, 1, null, null) == 2
     # nothing to do: no pointer is needed
+    assert L.alhr_update_tree(d, null, null, 5, 5, null, null) == 0
     assert L.alhr_forward(ctypes.byref(_dims(A, nq=0)), null, null, null, null, null, null, null,
                           null, null, null, null, null, null) == 0
     assert L.alhr_status_string(3) == b"ALHR_ERR_OVERFLOW"

@@ -26,8 +26,9 @@ LAUNCH_MODES = {"auto": 0, "throughput": 1, "latency": 2}
 
 EXPORTS = ["alhr_tree_rows", "alhr_tree_narrow_levels", "alhr_tree_bytes",
            "alhr_tree_level_offset", "alhr_score_bits", "alhr_status_string", "alhr_build_info",
-           "alhr_build_tree", "alhr_tree_unpack", "alhr_predict_budget", "alhr_route",
-           "alhr_attend", "alhr_forward", "alhr_set_launch_mode", "alhr_get_launch_mode"]
+           "alhr_build_tree", "alhr_update_tree", "alhr_tree_unpack", "alhr_predict_budget",
+           "alhr_route", "alhr_attend", "alhr_forward", "alhr_set_launch_mode",
+           "alhr_get_launch_mode"]
 
 
 class AlhrError(RuntimeError):
@@ -65,6 +66,7 @@ def lib() -> ctypes.CDLL:
         L.alhr_status_string.argtypes, L.alhr_status_string.restype = [I32], ctypes.c_char_p
         L.alhr_build_info.argtypes, L.alhr_build_info.restype = [], ctypes.c_char_p
         L.alhr_build_tree.argtypes = [DP, P, P, P, P]
+        L.alhr_update_tree.argtypes = [DP, P, P, I32, I32, P, P]
         L.alhr_tree_unpack.argtypes = [DP, P, P, P]
         L.alhr_predict_budget.argtypes = [DP, P, P, P, P, P, P, P]
         L.alhr_route.argtypes = [DP, P, P, P, P, P, P, P, P, P]
@@ -72,8 +74,9 @@ def lib() -> ctypes.CDLL:
         L.alhr_forward.argtypes = [DP, P, P, P, P, P, P, P, P, P, P, P, P, P]
         L.alhr_set_launch_mode.argtypes = [I32]
         L.alhr_get_launch_mode.argtypes, L.alhr_get_launch_mode.restype = [], I32
-        for f in ("alhr_build_tree", "alhr_tree_unpack", "alhr_predict_budget", "alhr_route",
-                  "alhr_attend", "alhr_forward", "alhr_set_launch_mode"):
+        for f in ("alhr_build_tree", "alhr_update_tree", "alhr_tree_unpack",
+                  "alhr_predict_budget", "alhr_route", "alhr_attend", "alhr_forward",
+                  "alhr_set_launch_mode"):
             getattr(L, f).restype = I32
         _lib = L
     return _lib
@@ -152,6 +155,19 @@ def build_tree(K: torch.Tensor, tree: torch.Tensor | None = None, value_bound: i
     dims = make_dims(None, K, value_bound=value_bound)
     _check(lib().alhr_build_tree(ctypes.byref(dims), _ptr(K), _ptr(tree), _ptr(dev_err),
                                  _stream(K.device)), "alhr_build_tree")
+    return tree
+
+
+def update_tree(K: torch.Tensor, tree: torch.Tensor, lo: int, hi: int, value_bound: int = 16,
+                dev_err: torch.Tensor | None = None) -> torch.Tensor:
+    """After rows [lo, hi) of K changed (e.g. appended keys): updates `tree` in place to equal
+    build_tree(K), given that it was the tree of K before the change. Returns `tree`."""
+    B, H, n, d = K.shape
+    _want(K, torch.int8, (B, H, n, d), "K")
+    _want(tree, torch.uint8, (B, H, tree_bytes(n, d, value_bound)), "tree")
+    dims = make_dims(None, K, value_bound=value_bound)
+    _check(lib().alhr_update_tree(ctypes.byref(dims), _ptr(K), _ptr(tree), int(lo), int(hi),
+                                  _ptr(dev_err), _stream(K.device)), "alhr_update_tree")
     return tree
 
 

@@ -145,6 +145,20 @@ alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, void* tree,
                                            static_cast<cudaStream_t>(stream)));
 }
 
+alhr_status alhr_update_tree(const alhr_dims* dims, const int8_t* K, void* tree, int32_t lo,
+                             int32_t hi, uint32_t* dev_err, void* stream) {
+  const alhr_status s = check_common(dims);
+  if (s != ALHR_OK) return s;
+  if (lo < 0 || hi < lo || hi > dims->n) return ALHR_ERR_INVALID_ARG;
+  if (lo == hi) return ALHR_OK;
+  if (!K || !tree || !aligned16(K) || !aligned16(tree)) return ALHR_ERR_INVALID_ARG;
+  const long long bh = (long long)dims->batch * dims->heads;
+  const alhr::TreeLayout tl = alhr::make_tree_layout(dims->n, dims->d, dims->value_bound);
+  return from_cuda(alhr::launch_update_tree(K, static_cast<char*>(tree), tl, bh, lo, hi,
+                                            value_bound_of(dims), dev_err,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 alhr_status alhr_tree_unpack(const alhr_dims* dims, const void* tree, int32_t* nodes,
                              void* stream) {
   const alhr_status s = check_common(dims);

@@ -13,6 +13,11 @@ struct QueryArgs;
 // Tree build: levels 1..log2 n of every (b,h) block (see tree_build.cu).
 cudaError_t launch_build_tree(const int8_t* K, char* tree, const TreeLayout& tl, long long bh,
                               int value_bound, uint32_t* dev_err, cudaStream_t st);
+// After rows [lo, hi) of K changed: every tree row over them, made equal to a full build's
+// (see tree_build.cu).
+cudaError_t launch_update_tree(const int8_t* K, char* tree, const TreeLayout& tl, long long bh,
+                               int lo, int hi, int value_bound, uint32_t* dev_err,
+                               cudaStream_t st);
 // The tree as plain int32 rows, level-major (see tree_build.cu).
 cudaError_t launch_tree_unpack(const char* tree, const TreeLayout& tl, long long bh,
                                int32_t* nodes, cudaStream_t st);

@@ -28,11 +28,12 @@ enum InKind : int { kFromKeys = 0, kFromNarrow = 1, kFromWide = 2 };
 template <int D, int IN>
 __global__ void __launch_bounds__(kTreeThreads)
     tree_chunk_kernel(const int8_t* __restrict__ K, char* __restrict__ tree, const TreeLayout tl,
-                      int lin, int m, int chunks_per_head, int value_bound, uint32_t* dev_err) {
+                      int lin, int m, int chunk0, int chunks_per_head, int value_bound,
+                      uint32_t* dev_err) {
   extern __shared__ int4 smem4[];  // [2^m][D] int32
   constexpr int Q4 = D / 4;        // int4 per row
   const long long bh = blockIdx.x / chunks_per_head;
-  const int chunk = blockIdx.x - int(bh * chunks_per_head);
+  const int chunk = chunk0 + int(blockIdx.x - bh * chunks_per_head);
   const int rows = 1 << m;
   const int n = tl.n;
   char* Th = tree + bh * tl.block_bytes;
@@ -142,11 +143,126 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// ---- incremental update of a few keys (decode appends)
+//
+// Rows [lo, hi) of K changed. Every level-1 row over them moves by delta(k) = K[2k] + K[2k+1]
+// - stored row (the stored row is the old pair sum, so no old key is needed), and every
+// ancestor at level l moves by the sum of the deltas of the level-1 rows beneath it. One CTA
+// per (b,h): the deltas go to shared memory first (reading the old level-1 rows), then every
+// affected row of every level is read, moved and written once, with the (level, row, column)
+// items of all levels in one flat index space so that their loads are independent.
+constexpr int kDeltaMaxKeys = 64;  // larger ranges are rebuilt chunk by chunk
+constexpr int kDeltaThreads = 256;
+
+template <int D>
+__device__ __forceinline__ int4 ld_row4(const char* Th, const TreeLayout& tl, int l, int j, int c) {
+  const char* row = Th + tl.offset_of(l) + (long long)j * tl.row_bytes(l);
+  if (l <= tl.narrow) {
+    const uint2 p = *(reinterpret_cast<const uint2*>(row) + c);
+    return make_int4(int(p.x << 16) >> 16, int(p.x) >> 16, int(p.y << 16) >> 16, int(p.y) >> 16);
+  }
+  return *(reinterpret_cast<const int4*>(row) + c);
+}
+
+template <int D>
+__device__ __forceinline__ void st_row4(char* Th, const TreeLayout& tl, int l, int j, int c,
+                                        int4 v) {
+  char* row = Th + tl.offset_of(l) + (long long)j * tl.row_bytes(l);
+  if (l <= tl.narrow) {
+    *(reinterpret_cast<uint2*>(row) + c) =
+        make_uint2((unsigned(v.x) & 0xffffu) | (unsigned(v.y) << 16),
+                   (unsigned(v.z) & 0xffffu) | (unsigned(v.w) << 16));
+  } else {
+    *(reinterpret_cast<int4*>(row) + c) = v;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDeltaThreads)
+    tree_delta_kernel(const int8_t* __restrict__ K, char* __restrict__ tree, const TreeLayout tl,
+                      int lo, int hi, int value_bound, uint32_t* dev_err) {
+  constexpr int Q4 = D / 4;
+  __shared__ int4 delta[(kDeltaMaxKeys / 2 + 1) * Q4];
+  const long long bh = blockIdx.x;
+  const int n = tl.n;
+  char* Th = tree + bh * tl.block_bytes;
+  const int8_t* Kh = K + bh * (long long)n * D;
+  const int k0 = lo >> 1, k1 = (hi - 1) >> 1;  // level-1 rows over [lo, hi)
+  const int span = k1 - k0 + 1;
+
+  bool bad = false;
+  for (int t = threadIdx.x; t < span * Q4; t += kDeltaThreads) {
+    const int kk = t / Q4, c = t - kk * Q4;
+    const int k = k0 + kk;
+    const int a = __ldg(reinterpret_cast<const int*>(Kh + (long long)(2 * k) * D) + c);
+    const int b = __ldg(reinterpret_cast<const int*>(Kh + (long long)(2 * k + 1) * D) + c);
+    const int4 va = make_int4((a << 24) >> 24, (a << 16) >> 24, (a << 8) >> 24, a >> 24);
+    const int4 vb = make_int4((b << 24) >> 24, (b << 16) >> 24, (b << 8) >> 24, b >> 24);
+    const bool in_a = 2 * k >= lo && 2 * k < hi, in_b = 2 * k + 1 >= lo && 2 * k + 1 < hi;
+    if (in_a) bad |= va.x > value_bound | va.x < -value_bound | va.y > value_bound |
+                     va.y < -value_bound | va.z > value_bound | va.z < -value_bound |
+                     va.w > value_bound | va.w < -value_bound;
+    if (in_b) bad |= vb.x > value_bound | vb.x < -value_bound | vb.y > value_bound |
+                     vb.y < -value_bound | vb.z > value_bound | vb.z < -value_bound |
+                     vb.w > value_bound | vb.w < -value_bound;
+    const int4 old = ld_row4<D>(Th, tl, 1, k, c);
+    delta[t] = make_int4(va.x + vb.x - old.x, va.y + vb.y - old.y, va.z + vb.z - old.z,
+                         va.w + vb.w - old.w);
+  }
+  if (__syncthreads_or(bad) && threadIdx.x == 0 && dev_err)
+    atomicOr(dev_err, ALHR_DEVERR_VALUE_RANGE);
+
+  int total = 0;
+  for (int l = 1; l <= tl.L; ++l) total += (((hi - 1) >> l) - (lo >> l) + 1) * Q4;
+  // kPer items per thread per round: all their rows are loaded before any is written back
+  // (items are disjoint rows/columns), so one round costs one memory round trip
+  constexpr int kPer = 4;
+  for (int f0 = 0; f0 < total; f0 += kPer * kDeltaThreads) {
+    int lv[kPer], jv[kPer], cv[kPer];
+    int4 acc[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int f = f0 + u * kDeltaThreads + threadIdx.x;
+      lv[u] = 0;
+      if (f < total) {
+        int l = 1, g = f;
+        for (;;) {  // level of flat item f
+          const int items = (((hi - 1) >> l) - (lo >> l) + 1) * Q4;
+          if (g < items) break;
+          g -= items;
+          ++l;
+        }
+        const int jj = g / Q4;
+        lv[u] = l;
+        jv[u] = (lo >> l) + jj;
+        cv[u] = g - jj * Q4;
+        acc[u] = ld_row4<D>(Th, tl, l, jv[u], cv[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      if (lv[u] == 0) continue;
+      const int l = lv[u], j = jv[u], c = cv[u];
+      // level-1 rows beneath node (l, j), clipped to the updated span
+      const int s0 = max(j << (l - 1), k0) - k0;
+      const int s1 = min(((j + 1) << (l - 1)) - 1, k1) - k0;
+      for (int s = s0; s <= s1; ++s) {
+        const int4 dv = delta[s * Q4 + c];
+        acc[u].x += dv.x;
+        acc[u].y += dv.y;
+        acc[u].z += dv.z;
+        acc[u].w += dv.w;
+      }
+      st_row4<D>(Th, tl, l, j, c, acc[u]);
+    }
+  }
+}
+
+// Levels lin+1 .. of the chunks covering keys [lo, hi) (all of them for [0, n)).
 template <int D>
 cudaError_t build_tree_d(const int8_t* K, char* tree, const TreeLayout& tl, long long bh,
-                         int value_bound, uint32_t* dev_err, cudaStream_t st) {
+                         int lo, int hi, int value_bound, uint32_t* dev_err, cudaStream_t st) {
   const int L = tl.L;
-  const int n = tl.n;
   const size_t smem_max = size_t(1 << kChunkLog) * D * sizeof(int);
   // the opt-in above 48 KB of dynamic shared memory is a per-device function attribute
   static bool configured[128] = {};
@@ -167,19 +283,20 @@ cudaError_t build_tree_d(const int8_t* K, char* tree, const TreeLayout& tl, long
   int lin = 0;
   while (lin < L) {
     const int m = (L - lin) < kChunkLog ? (L - lin) : kChunkLog;
-    const int chunks = (n >> lin) >> m;
+    const int c0 = (lo >> lin) >> m, c1 = ((hi - 1) >> lin) >> m;
+    const int chunks = c1 - c0 + 1;
     const long long grid = bh * chunks;
     const size_t smem = size_t(1 << m) * D * sizeof(int);
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     if (lin == 0) {
       tree_chunk_kernel<D, kFromKeys><<<unsigned(grid), kTreeThreads, smem, st>>>(
-          K, tree, tl, lin, m, chunks, value_bound, dev_err);
+          K, tree, tl, lin, m, c0, chunks, value_bound, dev_err);
     } else if (lin <= tl.narrow) {
       tree_chunk_kernel<D, kFromNarrow><<<unsigned(grid), kTreeThreads, smem, st>>>(
-          K, tree, tl, lin, m, chunks, value_bound, dev_err);
+          K, tree, tl, lin, m, c0, chunks, value_bound, dev_err);
     } else {
       tree_chunk_kernel<D, kFromWide><<<unsigned(grid), kTreeThreads, smem, st>>>(
-          K, tree, tl, lin, m, chunks, value_bound, dev_err);
+          K, tree, tl, lin, m, c0, chunks, value_bound, dev_err);
     }
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -192,8 +309,25 @@ cudaError_t build_tree_d(const int8_t* K, char* tree, const TreeLayout& tl, long
 
 cudaError_t launch_build_tree(const int8_t* K, char* tree, const TreeLayout& tl, long long bh,
                               int value_bound, uint32_t* dev_err, cudaStream_t st) {
-  return tl.d == 64 ? build_tree_d<64>(K, tree, tl, bh, value_bound, dev_err, st)
-                    : build_tree_d<128>(K, tree, tl, bh, value_bound, dev_err, st);
+  return tl.d == 64 ? build_tree_d<64>(K, tree, tl, bh, 0, tl.n, value_bound, dev_err, st)
+                    : build_tree_d<128>(K, tree, tl, bh, 0, tl.n, value_bound, dev_err, st);
+}
+
+cudaError_t launch_update_tree(const int8_t* K, char* tree, const TreeLayout& tl, long long bh,
+                               int lo, int hi, int value_bound, uint32_t* dev_err,
+                               cudaStream_t st) {
+  if (hi <= lo) return cudaSuccess;
+  if (hi - lo > kDeltaMaxKeys)
+    return tl.d == 64 ? build_tree_d<64>(K, tree, tl, bh, lo, hi, value_bound, dev_err, st)
+                      : build_tree_d<128>(K, tree, tl, bh, lo, hi, value_bound, dev_err, st);
+  if (bh > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  if (tl.d == 64)
+    tree_delta_kernel<64><<<unsigned(bh), kDeltaThreads, 0, st>>>(K, tree, tl, lo, hi,
+                                                                  value_bound, dev_err);
+  else
+    tree_delta_kernel<128><<<unsigned(bh), kDeltaThreads, 0, st>>>(K, tree, tl, lo, hi,
+                                                                   value_bound, dev_err);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_tree_unpack(const char* tree, const TreeLayout& tl, long long bh,
