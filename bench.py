@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--impl", default="alhr", choices=["alhr", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stages", action="store_true",
+                    help="instead of the bench line: per-stage times of the workload through the "
+                         "unfused entry points, and fused-forward time against N (1 GPU)")
     ap.add_argument("--cpu-sample-stride", type=int, default=8,
                     help="CPU baseline: every k-th query row of every (b,h) block")
     ap.add_argument("--ref-stride", type=int, default=64,
@@ -371,6 +374,80 @@ def run_alhr(args, dist, rank, world):
     return line
 
 
+def _event_time(fn, reps: int, flush) -> float:
+    """Median seconds of fn() over reps, L2 flushed before each, CUDA events on the stream."""
+    ts = []
+    stream = torch.cuda.current_stream()
+    for r in range(reps):
+        flush.fill_(r & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) / 1e3)
+    return statistics.median(ts)
+
+
+def run_stages(args):
+    """Per-stage split of one step (tree build, predictor, route, unfused attend, and the fused
+    forward that does the last three in one kernel), then the fused forward against N at fixed
+    batch and heads (prefill of every position), with the fitted log-log exponent of its time."""
+    from tree_routed_sparse_b200 import alhr, synth
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    reps = max(args.steps, 5)
+
+    def stages(wl):
+        vb = max(-wl.qk_lo, wl.qk_hi)
+        inp = synth.make_inputs(wl, dev)
+        Q, K, V, W, bo = inp["Q"], inp["K"], inp["V"], inp["W"], inp["budget_override"]
+        kw = dict(q_start=wl.q_start, window=wl.window, max_keys=wl.max_keys,
+                  score_bits=wl.score_bits, value_bound=vb)
+        tree = alhr.build_tree(K, value_bound=vb)
+        budget = bo if W is None else alhr.predict_budget(Q, K, tree, W, **kw)
+        r = alhr.route(Q, K, tree, budget, with_expansions=False, **kw)
+        idx, count = r["idx"], r["count"]
+        out = torch.empty((wl.batch, wl.heads, wl.nq, wl.d), dtype=torch.float32, device=dev)
+        for _ in range(args.warmup):
+            alhr.forward(Q, K, V, tree, W=W, budget_override=bo, out=out, **kw)
+        t = {"tree_build": _event_time(lambda: alhr.build_tree(K, tree, value_bound=vb), reps, flush)}
+        if W is not None:
+            t["predict_budget"] = _event_time(
+                lambda: alhr.predict_budget(Q, K, tree, W, budget=budget, **kw), reps, flush)
+        t["route"] = _event_time(lambda: alhr.route(Q, K, tree, budget, idx=idx, count=count,
+                                                    with_expansions=False, **kw), reps, flush)
+        akw = {k: v for k, v in kw.items() if k != "score_bits"}
+        t["attend"] = _event_time(lambda: alhr.attend(Q, K, V, idx, count, out=out, **akw),
+                                  reps, flush)
+        t["fused_forward"] = _event_time(
+            lambda: alhr.forward(Q, K, V, tree, W=W, budget_override=bo, out=out, **kw), reps, flush)
+        keys = float(count.float().mean())
+        del inp, tree, out, idx, count, budget
+        torch.cuda.empty_cache()
+        return t, keys
+
+    base = synth.WORKLOADS[args.workload]
+    t, keys = stages(base)
+    report = {"report": "stages", "workload": describe(base), "reps": reps,
+              "stage_ms": {k: v * 1e3 for k, v in t.items()}, "mean_keys_per_query": keys,
+              "scaling": []}
+    sweep = [1024, 4096, 16384, 65536]
+    for n in sweep:
+        wl = base.replace(n=n, nq=n, q_start=0)
+        t, keys = stages(wl)
+        q = wl.bh * wl.nq
+        report["scaling"].append({"n": n, "queries": q, "fused_forward_ms": t["fused_forward"] * 1e3,
+                                  "tree_build_ms": t["tree_build"] * 1e3,
+                                  "ns_per_query": t["fused_forward"] / q * 1e9,
+                                  "mean_keys_per_query": keys})
+    xs = np.log([e["n"] for e in report["scaling"]])
+    ys = np.log([e["fused_forward_ms"] for e in report["scaling"]])
+    report["loglog_exponent_fused_forward_vs_n"] = float(np.polyfit(xs, ys, 1)[0])
+    report["gpu"] = torch.cuda.get_device_name(dev)
+    print(json.dumps(report))
+
+
 def profiled_traffic(workload: str):
     """DRAM bytes per launch of the fused kernel from the committed ncu summary, if that
     summary was taken on the kernel source as it is now; else None."""
@@ -416,6 +493,14 @@ def main():
             "e2e": {"value": r["value"], "unit": "queries/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
         }))
+        return
+
+    if args.stages:
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA device")
+        from tree_routed_sparse_b200 import build
+        build.build()
+        run_stages(args)
         return
 
     dist, rank, world = dist_setup(args.gpus)

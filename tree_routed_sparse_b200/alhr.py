@@ -198,12 +198,16 @@ def predict_budget(Q, K, tree, W, q_start=0, window=16, max_keys=96, score_bits=
 
 
 def route(Q, K, tree, budget, q_start=0, window=16, max_keys=96, score_bits=0,
-          value_bound=16, with_expansions=True, dev_err=None) -> dict:
+          value_bound=16, with_expansions=True, idx=None, count=None, dev_err=None) -> dict:
     dims = make_dims(Q, K, q_start, window, max_keys, score_bits, value_bound)
     B, H, nq, d = Q.shape
     _want(budget, torch.int32, (B, H, nq), "budget")
-    idx = torch.empty((B, H, nq, max_keys), dtype=torch.int32, device=Q.device)
-    count = torch.empty((B, H, nq), dtype=torch.int32, device=Q.device)
+    if idx is None:
+        idx = torch.empty((B, H, nq, max_keys), dtype=torch.int32, device=Q.device)
+    if count is None:
+        count = torch.empty((B, H, nq), dtype=torch.int32, device=Q.device)
+    _want(idx, torch.int32, (B, H, nq, max_keys), "idx")
+    _want(count, torch.int32, (B, H, nq), "count")
     exp = (torch.empty((B, H, nq, 3), dtype=torch.int32, device=Q.device)
            if with_expansions else None)
     _check(lib().alhr_route(ctypes.byref(dims), _ptr(Q), _ptr(K), _ptr(tree), _ptr(budget),
