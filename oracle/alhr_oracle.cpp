@@ -33,6 +33,18 @@
 //   R7  the reuse of what earlier queries found among their own neighbours (§Inference stage,
 //       third paragraph) is read as a cache that changes no selected set; ignored.
 //   R8  attention is softmax(q . k / sqrt(d)) . V over the selected keys, no temperature.
+// Two descent variants (off by default; both off is the method above):
+//   R9  mean-normalised scores: candidates are ranked by q . node_sum / 2^level, the mean of
+//       the keys beneath them (what block-sparse methods rank blocks by; page "ALHR把注意力
+//       变成树搜索", §"它和块稀疏、线性注意力有什么区别"). Compared exactly, as fractions with
+//       power-of-two denominators; equal means go to the lower start.
+//   R10 leaf buckets of 2^b keys (page "ALHR把注意力变成树搜索", §"次二次复杂度成立，需要满足三个
+//       前提": the leaf bucket size must not grow with the sequence): a node of level <= b is
+//       a bucket and is not expanded; the beam keeps r >> b nodes (the routed key budget r
+//       counted in whole buckets, so at most r keys); the descent ends when the frontier holds
+//       only buckets, and every key of every kept bucket is selected. b = 0 is the method above.
+//       The frontier is pruned after every expansion step and also when the forest's roots are
+//       all buckets already.
 
 #include <algorithm>
 #include <cmath>
@@ -57,6 +69,20 @@ struct Node {
   int64_t start;  // first key position covered; the node covers [start, start + 2^level)
   int64_t score;  // q . node_sum
 };
+
+// Candidate order: the larger score first (raw sums, or under R9 the larger mean
+// score / 2^level, compared as a.score * 2^b.level against b.score * 2^a.level), then the
+// lower start.
+bool ranks_before(const Node& a, const Node& b, bool norm) {
+  if (norm) {
+    const __int128 x = static_cast<__int128>(a.score) * (static_cast<__int128>(1) << b.level);
+    const __int128 y = static_cast<__int128>(b.score) * (static_cast<__int128>(1) << a.level);
+    if (x != y) return x > y;
+  } else if (a.score != b.score) {
+    return a.score > b.score;
+  }
+  return a.start < b.start;
+}
 
 // The stored sum row of a node: K itself at level 0, the tree above.
 int64_t node_score(int n, int d, const int8_t* K, const int32_t* nodes, const int8_t* q,
@@ -140,9 +166,10 @@ int oracle_predict(int d, const int8_t* q, const int64_t* G, const int8_t* W, in
 // {nodes of level >= 2 expanded, level-1 nodes expanded} into expansions (nullable) and the
 // number of expanded nodes of each level l into by_level[l], l < 32 (nullable).
 // Returns the selection size min(B_eff, i+1) with B_eff = min(max(B,1), i+1, max_keys).
+// score_norm selects R9, bucket_log the bucket size 2^bucket_log of R10 (0: single keys).
 int oracle_route(int n, int d, const int8_t* K, const int32_t* nodes, const int8_t* q, int i,
-                 int budget, int w, int max_keys, int32_t* sel, int32_t* expansions,
-                 int32_t* by_level) {
+                 int budget, int w, int max_keys, int score_norm, int bucket_log, int32_t* sel,
+                 int32_t* expansions, int32_t* by_level) {
   if (by_level)
     for (int l = 0; l < 32; ++l) by_level[l] = 0;
   int64_t b_eff = std::max(budget, 1);
@@ -167,14 +194,24 @@ int oracle_route(int n, int d, const int8_t* K, const int32_t* nodes, const int8
         s += int64_t(1) << b;
       }
     }
-    // R6: expand every non-leaf, then keep the r best, until only keys remain
+    // R6: expand every non-leaf, then keep the r best, until only keys remain (R10: leaves
+    // are the buckets, nodes of level <= bucket_log, and the beam keeps r >> bucket_log)
+    const int64_t keep = r >> bucket_log;
+    const bool norm = score_norm != 0;
     for (;;) {
       bool any_inner = false;
-      for (const Node& nd : frontier) any_inner |= (nd.level > 0);
-      if (!any_inner) break;
+      for (const Node& nd : frontier) any_inner |= (nd.level > bucket_log);
+      if (!any_inner) {
+        if (int64_t(frontier.size()) > keep) {  // roots that are all buckets (R10)
+          std::sort(frontier.begin(), frontier.end(),
+                    [norm](const Node& a, const Node& b) { return ranks_before(a, b, norm); });
+          frontier.resize(size_t(keep));
+        }
+        break;
+      }
       std::vector<Node> cand;
       for (const Node& nd : frontier) {
-        if (nd.level == 0) {
+        if (nd.level <= bucket_log) {
           cand.push_back(nd);
           continue;
         }
@@ -185,16 +222,15 @@ int oracle_route(int n, int d, const int8_t* K, const int32_t* nodes, const int8
         cand.push_back({cl, left, node_score(n, d, K, nodes, q, cl, left)});
         cand.push_back({cl, right, node_score(n, d, K, nodes, q, cl, right)});
       }
-      if (int64_t(cand.size()) > r) {
-        std::sort(cand.begin(), cand.end(), [](const Node& a, const Node& b) {
-          if (a.score != b.score) return a.score > b.score;
-          return a.start < b.start;
-        });
-        cand.resize(size_t(r));
+      if (int64_t(cand.size()) > keep) {
+        std::sort(cand.begin(), cand.end(),
+                  [norm](const Node& a, const Node& b) { return ranks_before(a, b, norm); });
+        cand.resize(size_t(keep));
       }
       frontier.swap(cand);
     }
-    for (const Node& nd : frontier) chosen.push_back(nd.start);
+    for (const Node& nd : frontier)
+      for (int64_t t = nd.start; t < nd.start + (int64_t(1) << nd.level); ++t) chosen.push_back(t);
   }
   std::sort(chosen.begin(), chosen.end());
   for (size_t k = 0; k < chosen.size(); ++k) sel[k] = int32_t(chosen[k]);
@@ -233,13 +269,15 @@ void oracle_attend(int d, const int8_t* q, const int8_t* K, const uint16_t* V,
 }
 
 // The whole path for a set of queries of one (b,h) block, in the README's order: causal sum
-// and budget predictor (or the given budget), neighbour search and descent, attention.
+// and budget predictor (or the given budget), neighbour search and descent (with the R9 / R10
+// variants as oracle_route), attention.
 //   Q [nq][d], K [n][d], V [n][d], nodes [n-1][d] (this oracle's own tree), W [32][2d] or NULL,
 //   budget_override [nq] or NULL, rows: the query rows to compute (NULL = all nq rows).
 // Outputs (rows not listed are left untouched): out [nq][d], idx [nq][max_keys] (-1 padded),
 // count [nq], expansions [nq][2], budget_out [nq] (the budget used, after the clamp to >= 1),
 // by_level [nq][32] or NULL (expanded nodes per level).
-void oracle_forward(int n, int d, int q_start, int nq, int w, int max_keys, const int8_t* Q,
+void oracle_forward(int n, int d, int q_start, int nq, int w, int max_keys, int score_norm,
+                    int bucket_log, const int8_t* Q,
                     const int8_t* K, const uint16_t* V, const int32_t* nodes, const int8_t* W,
                     const int32_t* budget_override, const int32_t* rows, int n_rows,
                     double* out, int32_t* idx, int32_t* count, int32_t* expansions,
@@ -258,7 +296,8 @@ void oracle_forward(int n, int d, int q_start, int nq, int w, int max_keys, cons
       oracle_causal_sum(d, K, i, G.data());
       budget = 3 * (oracle_predict(d, q, G.data(), W, nullptr) + 1);
     }
-    const int c = oracle_route(n, d, K, nodes, q, i, budget, w, max_keys, sel.data(),
+    const int c = oracle_route(n, d, K, nodes, q, i, budget, w, max_keys, score_norm,
+                               bucket_log, sel.data(),
                                expansions + int64_t(row) * 2,
                                by_level ? by_level + int64_t(row) * 32 : nullptr);
     oracle_attend(d, q, K, V, sel.data(), c, out + int64_t(row) * d);

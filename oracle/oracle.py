@@ -51,11 +51,12 @@ def _configure(L):
     L.oracle_causal_sum.restype = None
     L.oracle_predict.argtypes = [I, P, P, P, P]
     L.oracle_predict.restype = I
-    L.oracle_route.argtypes = [I, I, P, P, P, I, I, I, I, P, P, P]
+    L.oracle_route.argtypes = [I, I, P, P, P, I, I, I, I, I, I, P, P, P]
     L.oracle_route.restype = I
     L.oracle_attend.argtypes = [I, P, P, P, P, I, P]
     L.oracle_attend.restype = None
-    L.oracle_forward.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, P, P, P]
+    L.oracle_forward.argtypes = [I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, P, P,
+                                 P]
     L.oracle_forward.restype = None
     return L
 
@@ -116,8 +117,10 @@ def predict(q: np.ndarray, G: np.ndarray, W: np.ndarray):
     return c, logits
 
 
-def route(K, nodes, q, i: int, budget: int, window: int, max_keys: int, by_level=False):
-    """-> (selected positions ascending, (exp_hi, exp_l1)[, expanded nodes per level [32]])."""
+def route(K, nodes, q, i: int, budget: int, window: int, max_keys: int, by_level=False,
+          score_norm: bool = False, bucket_log: int = 0):
+    """-> (selected positions ascending, (exp_hi, exp_l1)[, expanded nodes per level [32]]).
+    score_norm / bucket_log: the mean-normalised and leaf-bucket descent variants."""
     K = _c(K, np.int8)
     nodes = _c(nodes, np.int32)
     q = _c(q, np.int8)
@@ -126,7 +129,7 @@ def route(K, nodes, q, i: int, budget: int, window: int, max_keys: int, by_level
     exp = np.zeros(2, dtype=np.int32)
     lv = np.zeros(32, dtype=np.int32) if by_level else None
     c = lib().oracle_route(n, d, _p(K), _p(nodes), _p(q), i, budget, window, max_keys,
-                           _p(sel), _p(exp), _p(lv))
+                           int(bool(score_norm)), int(bucket_log), _p(sel), _p(exp), _p(lv))
     if by_level:
         return sel[:c].copy(), (int(exp[0]), int(exp[1])), lv
     return sel[:c].copy(), (int(exp[0]), int(exp[1]))
@@ -144,7 +147,7 @@ def attend(q, K, V_bits, sel) -> np.ndarray:
 
 
 def forward(Q, K, V_bits, nodes, W, budget_override, q_start: int, window: int,
-            max_keys: int, rows=None) -> dict:
+            max_keys: int, rows=None, score_norm: bool = False, bucket_log: int = 0) -> dict:
     """The whole path for one (b,h) block. Q int8 [nq, d]; K int8 [n, d]; V_bits uint16
     [n, d]; nodes int32 [n-1, d] (from build_tree); W int8 [32, 2d] or None; budget_override
     int32 [nq] or None; rows: query rows to compute (None = all).
@@ -165,7 +168,8 @@ def forward(Q, K, V_bits, nodes, W, budget_override, q_start: int, window: int,
     exp = np.zeros((nq, 2), dtype=np.int32)
     bud = np.zeros(nq, dtype=np.int32)
     lv = np.zeros((nq, 32), dtype=np.int32)
-    lib().oracle_forward(n, d, q_start, nq, window, max_keys, _p(Q), _p(K), _p(V_bits),
+    lib().oracle_forward(n, d, q_start, nq, window, max_keys, int(bool(score_norm)),
+                         int(bucket_log), _p(Q), _p(K), _p(V_bits),
                          _p(nodes), _p(W), _p(bo), _p(rws), 0 if rws is None else len(rws),
                          _p(out), _p(idx), _p(count), _p(exp), _p(bud), _p(lv))
     return dict(out=out, idx=idx, count=count, expansions=exp, budget=bud, by_level=lv)

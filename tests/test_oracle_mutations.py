@@ -16,8 +16,7 @@ _SRC = os.path.join(os.path.dirname(orc.__file__), "alhr_oracle.cpp")
 
 MUTATIONS = {
     "tie_to_higher_start": ("return a.start < b.start;", "return a.start > b.start;"),
-    "keep_lowest_scores": ("if (a.score != b.score) return a.score > b.score;",
-                           "if (a.score != b.score) return a.score < b.score;"),
+    "keep_lowest_scores": ("    return a.score > b.score;", "    return a.score < b.score;"),
     "window_one_too_wide": ("t > int64_t(i) - w &&", "t >= int64_t(i) - w &&"),
     "forest_covers_window_key": ("const int64_t m = int64_t(i) - w + 1;",
                                  "const int64_t m = int64_t(i) - w + 2;"),
@@ -39,7 +38,15 @@ MUTATIONS = {
                                        "std::exp(mx - s[size_t(k)])"),
     "budget_not_clamped": ("budget = std::max(budget_override[row], 1);",
                            "budget = budget_override[row];"),
-    "prune_keeps_one_less": ("cand.resize(size_t(r));", "cand.resize(size_t(r - 1));"),
+    "prune_keeps_one_less": ("cand.resize(size_t(keep));", "cand.resize(size_t(keep - 1));"),
+    "mean_scaled_by_own_level": ("static_cast<__int128>(a.score) * (static_cast<__int128>(1) << b.level)",
+                                 "static_cast<__int128>(a.score) * (static_cast<__int128>(1) << a.level)"),
+    "mean_ignored": ("if (norm) {", "if (false) {"),
+    "bucket_beam_in_keys": ("const int64_t keep = r >> bucket_log;", "const int64_t keep = r;"),
+    "bucket_level_expanded": ("if (nd.level <= bucket_log) {", "if (nd.level < bucket_log) {"),
+    "bucket_last_key_dropped": ("t < nd.start + (int64_t(1) << nd.level); ++t)",
+                                "t + 1 < nd.start + (int64_t(1) << nd.level); ++t)"),
+    "bucket_roots_not_pruned": ("if (int64_t(frontier.size()) > keep) {", "if (false) {"),
 }
 
 PIN_TESTS = [
@@ -57,6 +64,11 @@ PIN_TESTS = [
     ("dense", lambda g: pins.test_full_budget_is_dense_causal_attention(64, 8, 4)),
     ("attention_closed_forms", lambda g: pins.test_attention_closed_forms()),
     ("clamp", lambda g: pins.test_forward_budget_override_clamp_and_predictor()),
+    ("mean_hand", lambda g: pins.test_mean_normalised_hand_example()),
+    ("mean_single_root", lambda g: pins.test_mean_normalised_single_root_equals_raw(64, 16)),
+    ("bucket_wide", lambda g: pins.test_buckets_wide_beam_route_the_whole_past(2)),
+    ("bucket_hand", lambda g: pins.test_bucket_hand_example()),
+    ("bucket_roots", lambda g: pins.test_buckets_prune_roots_that_are_all_buckets()),
 ]
 
 

@@ -243,9 +243,13 @@ def test_route_structure_random():
         assert (routed <= i - w).all() and (routed >= 0).all()
 
 
-def _alt_route(K, q, i, B, w, max_keys):
+def _alt_route(K, q, i, B, w, max_keys, norm=False, bucket_log=0):
     """Independent formulation: intervals [lo, hi) halved recursively, sums straight from K,
-    roots as the largest aligned blocks taken greedily from the left."""
+    roots as the largest aligned blocks taken greedily from the left. norm ranks intervals by
+    their exact mean score (a Fraction); bucket_log makes intervals of at most 2^bucket_log keys
+    leaves, the beam r >> bucket_log wide, and selects every key of the kept intervals."""
+    from fractions import Fraction
+    bsz = 1 << bucket_log
     b_eff = min(max(B, 1), i + 1, max_keys)
     win = [t for t in range(i, max(-1, i - w), -1)][:b_eff]
     r = b_eff - len(win)
@@ -263,21 +267,27 @@ def _alt_route(K, q, i, B, w, max_keys):
         qq = q.astype(np.int64)
 
         def score(iv):
-            return int(K[iv[0]: iv[1]].astype(np.int64).sum(0) @ qq)
+            s = int(K[iv[0]: iv[1]].astype(np.int64).sum(0) @ qq)
+            return Fraction(s, iv[1] - iv[0]) if norm else s
 
-        while any(hi - lo > 1 for lo, hi in F):
+        keep = r // bsz
+        while True:
+            if not any(hi - lo > bsz for lo, hi in F):
+                if len(F) > keep:
+                    F = sorted(F, key=lambda iv: (-score(iv), iv[0]))[:keep]
+                break
             C = []
             for lo, hi in F:
-                if hi - lo == 1:
+                if hi - lo <= bsz:
                     C.append((lo, hi))
                     continue
                 exp[0 if hi - lo >= 4 else 1] += 1
                 mid = (lo + hi) // 2
                 C += [(lo, mid), (mid, hi)]
-            if len(C) > r:
-                C = sorted(C, key=lambda iv: (-score(iv), iv[0]))[:r]
+            if len(C) > keep:
+                C = sorted(C, key=lambda iv: (-score(iv), iv[0]))[:keep]
             F = C
-        routed = [lo for lo, _ in F]
+        routed = [t for lo, hi in F for t in range(lo, hi)]
     return sorted(win + routed), tuple(exp)
 
 
@@ -297,6 +307,126 @@ def test_route_matches_independent_formulation(n, d):
         ref_sel, ref_exp = _alt_route(K, q, i, B, w, 96)
         assert sel.tolist() == ref_sel
         assert exp == ref_exp
+
+
+@pytest.mark.parametrize("n,d", [(8, 2), (16, 4), (64, 8), (256, 8)])
+@pytest.mark.parametrize("norm,bucket_log", [(True, 0), (False, 1), (False, 2), (True, 2),
+                                             (True, 3)])
+def test_descent_variants_match_independent_formulation(n, d, norm, bucket_log):
+    rng = _rng(n * 13 + d + 101 * bucket_log + 7 * norm)
+    for trial in range(40):
+        lo, hi = (-16, 16) if trial % 2 else (-1, 1)
+        K = _rand_qk(rng, (n, d), lo, hi)
+        nodes = orc.build_tree(K)
+        q = _rand_qk(rng, (d,), lo, hi)
+        i = int(rng.integers(0, n))
+        w = int(rng.integers(1, 6))
+        B = int(rng.integers(1, n + 2))
+        sel, exp = orc.route(K, nodes, q, i, B, w, 96, score_norm=norm, bucket_log=bucket_log)
+        ref_sel, ref_exp = _alt_route(K, q, i, B, w, 96, norm=norm, bucket_log=bucket_log)
+        assert sel.tolist() == ref_sel, (trial, i, w, B)
+        assert exp == ref_exp
+
+
+def test_variants_off_are_the_method():
+    rng = _rng(5)
+    n, d = 256, 8
+    K = _rand_qk(rng, (n, d))
+    nodes = orc.build_tree(K)
+    for _ in range(50):
+        q = _rand_qk(rng, (d,))
+        i, B = int(rng.integers(0, n)), int(rng.integers(1, 97))
+        a = orc.route(K, nodes, q, i, B, 16, 96)
+        b = orc.route(K, nodes, q, i, B, 16, 96, score_norm=False, bucket_log=0)
+        assert a[0].tolist() == b[0].tolist() and a[1] == b[1]
+
+
+def test_mean_normalised_hand_example():
+    """Worked by hand: keys 0..7 each score 1 against q, key 8 scores 3, window w = 1 at
+    i = 9 (so the forest is [0, 8) and the key 8), one routed place (B = 2). Raw sums: [0, 8)
+    (8) is expanded, its halves (4, 4) beat key 8 (3), and the descent ends on key 0 (ties go
+    to the lower start). Means: the halves average 1, key 8 averages 3, so key 8 is kept."""
+    d = 2
+    K = np.zeros((16, d), dtype=np.int8)
+    K[0:8] = [1, 0]
+    K[8] = [3, 0]
+    q = np.array([1, 0], dtype=np.int8)
+    nodes = orc.build_tree(K)
+    raw, _ = orc.route(K, nodes, q, 9, 2, 1, 96)
+    mean, _ = orc.route(K, nodes, q, 9, 2, 1, 96, score_norm=True)
+    assert raw.tolist() == [0, 9]
+    assert mean.tolist() == [8, 9]
+
+
+@pytest.mark.parametrize("n,w", [(64, 16), (256, 4)])
+def test_mean_normalised_single_root_equals_raw(n, w):
+    """When the past [0, i-w] is one aligned block, every frontier holds nodes of one level, so
+    ranking by means and by sums is the same order: the two descents agree."""
+    rng = _rng(n + w + 3)
+    d = 8
+    K = _rand_qk(rng, (n, d))
+    nodes = orc.build_tree(K)
+    for m in (1, 2, 4, 8, 16, 32):
+        i = m + w - 1
+        if i >= n:
+            continue
+        for _ in range(6):
+            q = _rand_qk(rng, (d,))
+            B = int(rng.integers(w + 1, w + 60))
+            a = orc.route(K, nodes, q, i, B, w, 96)
+            b = orc.route(K, nodes, q, i, B, w, 96, score_norm=True)
+            assert a[0].tolist() == b[0].tolist() and a[1] == b[1]
+
+
+@pytest.mark.parametrize("bucket_log", [1, 2, 4])
+def test_buckets_wide_beam_route_the_whole_past(bucket_log):
+    """When the past [0, m) is a whole number of buckets, a budget of every past key is a beam
+    of exactly m >> bucket_log buckets: every key before the window is selected, and no node at
+    or below the bucket level is expanded."""
+    rng = _rng(bucket_log)
+    n, d, w = 256, 4, 8
+    K = _rand_qk(rng, (n, d))
+    nodes = orc.build_tree(K)
+    for t in (1, 3, 5, 10, 31):
+        i = (t << bucket_log) + w - 1
+        if i >= n:
+            continue
+        q = _rand_qk(rng, (d,))
+        B = (n + 8) << bucket_log
+        sel, _, lv = orc.route(K, nodes, q, i, B, w, B, by_level=True, bucket_log=bucket_log)
+        assert sel.tolist() == list(range(i + 1))
+        assert lv[: bucket_log + 1].sum() == 0
+
+
+def test_bucket_hand_example():
+    """Worked by hand: 16 past keys, buckets of 4, routed budget 8 -> 2 buckets. Key 9 alone
+    scores 10, every other key 0, and the window is w = 1 at i = 16. Step 1 expands [0, 16)
+    into [0, 8) (0) and [8, 16) (10); both stay. Step 2 expands them into four buckets scoring
+    0, 0, 10, 0: [8, 12) first, then [0, 4) by the lower start. Selected: keys 0-3, 8-11, 16."""
+    d = 2
+    K = np.zeros((32, d), dtype=np.int8)
+    K[9] = [5, 0]
+    q = np.array([2, 1], dtype=np.int8)
+    nodes = orc.build_tree(K)
+    sel, exp = orc.route(K, nodes, q, 16, 9, 1, 96, bucket_log=2)
+    assert sel.tolist() == [0, 1, 2, 3, 8, 9, 10, 11, 16]
+    assert exp == (3, 0)
+    # a routed budget of 7 keys holds only one whole bucket
+    sel, _ = orc.route(K, nodes, q, 16, 8, 1, 96, bucket_log=2)
+    assert sel.tolist() == [8, 9, 10, 11, 16]
+
+
+def test_buckets_prune_roots_that_are_all_buckets():
+    """i = 6, w = 1: the past [0, 6) is the forest [0, 4), [4, 6), both buckets of size <= 4.
+    With one bucket allowed (budget 1 + 4), only the better root is kept, without expansion."""
+    d = 1
+    K = np.zeros((8, d), dtype=np.int8)
+    K[5] = [3]
+    q = np.array([1], dtype=np.int8)
+    nodes = orc.build_tree(K)
+    sel, exp = orc.route(K, nodes, q, 6, 5, 1, 96, bucket_log=2)
+    assert sel.tolist() == [4, 5, 6]
+    assert exp == (0, 0)
 
 
 # ---------------------------------------------------------------- attention
