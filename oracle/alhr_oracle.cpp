@@ -42,7 +42,8 @@
 //       前提": the leaf bucket size must not grow with the sequence): a node of level <= b is
 //       a bucket and is not expanded; the beam keeps r >> b nodes (the routed key budget r
 //       counted in whole buckets, so at most r keys); the descent ends when the frontier holds
-//       only buckets, and every key of every kept bucket is selected. b = 0 is the method above.
+//       only buckets, and every key of every kept bucket is selected; when r >> b is 0 there is
+//       no beam and no descent. b = 0 is the method above.
 //       The frontier is pruned after every expansion step and also when the forest's roots are
 //       all buckets already.
 
@@ -184,7 +185,8 @@ int oracle_route(int n, int d, const int8_t* K, const int32_t* nodes, const int8
   int64_t exp_hi = 0, exp_l1 = 0;
   const int64_t r = b_eff - int64_t(chosen.size());
   const int64_t m = int64_t(i) - w + 1;  // keys strictly before the window: [0, m)
-  if (r > 0 && m > 0) {
+  const int64_t keep = r >> bucket_log;  // the beam: r keys, or r >> b whole buckets (R10)
+  if (keep > 0 && m > 0) {
     // R5: the maximal aligned power-of-two blocks of [0, m), largest first
     std::vector<Node> frontier;
     int64_t s = 0;
@@ -196,7 +198,6 @@ int oracle_route(int n, int d, const int8_t* K, const int32_t* nodes, const int8
     }
     // R6: expand every non-leaf, then keep the r best, until only keys remain (R10: leaves
     // are the buckets, nodes of level <= bucket_log, and the beam keeps r >> bucket_log)
-    const int64_t keep = r >> bucket_log;
     const bool norm = score_norm != 0;
     for (;;) {
       bool any_inner = false;

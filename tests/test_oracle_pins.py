@@ -256,7 +256,7 @@ def _alt_route(K, q, i, B, w, max_keys, norm=False, bucket_log=0):
     m = i - w + 1
     exp = [0, 0]
     routed = []
-    if r > 0 and m > 0:
+    if r // bsz > 0 and m > 0:
         F, lo = [], 0
         while lo < m:
             size = 1
@@ -414,6 +414,9 @@ def test_bucket_hand_example():
     # a routed budget of 7 keys holds only one whole bucket
     sel, _ = orc.route(K, nodes, q, 16, 8, 1, 96, bucket_log=2)
     assert sel.tolist() == [8, 9, 10, 11, 16]
+    # 3 routed keys hold no bucket: no beam, nothing expanded
+    sel, exp = orc.route(K, nodes, q, 16, 4, 1, 96, bucket_log=2)
+    assert sel.tolist() == [16] and exp == (0, 0)
 
 
 def test_buckets_prune_roots_that_are_all_buckets():
