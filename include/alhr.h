@@ -94,7 +94,25 @@ typedef struct {
   int32_t max_keys;    /* cap on keys per query, 1 <= max_keys <= 96                      */
   int32_t score_bits;  /* 0 = choose, 32 = int32 scores (checked), 64 = int64 scores      */
   int32_t value_bound; /* bound on |Q|, |K|; 0 means 16; at most 127                      */
+  int32_t score_norm;  /* descent variant: 0 rank by q . node_sum (the method), 1 by mean    */
+  int32_t bucket_log;  /* descent variant: 0 descend to keys (the method), b in 1..15: stop  */
+                       /* at buckets of 2^b keys                                          */
 } alhr_dims;
+
+/*
+ * Descent variants (alhr_route and alhr_forward; both 0 is the method as described):
+ *   score_norm = 1: candidates are ranked by their mean score q . node_sum / 2^level instead of
+ *     the sum, compared exactly (the kernel ranks by q . node_sum * 2^(log2 n - level)); equal
+ *     means go to the lower start. Block-sparse methods rank blocks by such means [page
+ *     "ALHR把注意力变成树搜索", §"它和块稀疏、线性注意力有什么区别"].
+ *   bucket_log = b > 0: leaf buckets of 2^b keys [same page, §"次二次复杂度成立，需要满足三个前提":
+ *     the leaf bucket must not grow with the sequence]. A node of level <= b is not expanded;
+ *     the beam keeps r >> b nodes, r being the routed key budget (so at most r keys); the
+ *     descent ends when the frontier holds only buckets (the roots are pruned too when they all
+ *     are buckets) and every key of every kept bucket is selected and scored.
+ * With score_norm = 1 the int32 score width needs d * value_bound^2 * n < 2^31 (the ranking
+ * value of a key is q . k * n).
+ */
 
 /* Number of tree rows per (b,h): n - 1. Returns 0 when n is not a power of two in [2, 2^20]. */
 ALHR_API size_t alhr_tree_rows(int32_t n);

@@ -32,8 +32,10 @@ def v_bits(V: torch.Tensor) -> np.ndarray:
     return V.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def oracle_slice(inp_cpu: dict, wl, b: int, h: int, rows=None, nodes=None) -> dict:
-    """Oracle results for the (b, h) block of a workload's inputs (host tensors)."""
+def oracle_slice(inp_cpu: dict, wl, b: int, h: int, rows=None, nodes=None, score_norm=False,
+                 bucket_log=0) -> dict:
+    """Oracle results for the (b, h) block of a workload's inputs (host tensors); score_norm /
+    bucket_log select the descent variants."""
     K = inp_cpu["K"][b, h].numpy()
     Q = inp_cpu["Q"][b, h].numpy()
     V = v_bits(inp_cpu["V"][b, h])
@@ -42,7 +44,8 @@ def oracle_slice(inp_cpu: dict, wl, b: int, h: int, rows=None, nodes=None) -> di
     W = None if inp_cpu["W"] is None else inp_cpu["W"].numpy()
     bo = None if inp_cpu["budget_override"] is None else inp_cpu["budget_override"][b, h].numpy()
     res = orc.forward(Q, K, V, nodes, W, bo, q_start=wl.q_start, window=wl.window,
-                      max_keys=wl.max_keys, rows=rows)
+                      max_keys=wl.max_keys, rows=rows, score_norm=score_norm,
+                      bucket_log=bucket_log)
     res["nodes"] = nodes
     res["narrow"] = metrics.narrow_levels(wl.n, wl.d, max(-wl.qk_lo, wl.qk_hi))
     return res

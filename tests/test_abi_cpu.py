@@ -108,7 +108,7 @@ def test_tree_layout_matches_documented_layout(A, n, d, vb):
 
 def _dims(A, **kw):
     base = dict(batch=2, heads=8, n=16384, d=64, q_start=0, nq=16384, window=16, max_keys=96,
-                score_bits=0, value_bound=16)
+                score_bits=0, value_bound=16, score_norm=0, bucket_log=0)
     base.update(kw)
     return A.Dims(*[base[f] for f, _ in A.Dims._fields_])
 
@@ -124,6 +124,12 @@ def test_score_width_choice(A):
     assert sb(score_bits=64) == 64
     assert sb(d=96) == -2 and sb(n=1000) == -1 and sb(window=33) == -2 and sb(max_keys=97) == -2
     assert sb(max_keys=0) == -1 and sb(q_start=1) == -1 and sb(score_bits=16) == -1
+    # ranked by means, a key's ranking value is q . k * n: the bound doubles
+    assert sb(n=65536, d=128) == 32                    # 128 * 256 * 2^15 = 2^30
+    assert sb(n=65536, d=128, score_norm=1) == 64      # 128 * 256 * 2^16 = 2^31
+    assert sb(n=65536, d=128, score_norm=1, score_bits=32) == -3
+    assert sb(score_norm=1) == 32 and sb(bucket_log=4) == 32
+    assert sb(score_norm=2) == -1 and sb(bucket_log=-1) == -1 and sb(bucket_log=16) == -1
 
 
 def test_entry_points_reject_bad_arguments_before_launch(A):

@@ -192,6 +192,53 @@ def test_decode_style_queries(alhr, synth, shape):
             compare_rows(res, oracle_slice(cpu, wl, b, h), b, h, np.arange(7), TOL, "decode")
 
 
+# ------------------------------------------------------------------ descent variants
+
+
+VARIANTS = [(True, 0), (False, 1), (False, 2), (True, 2), (False, 4), (True, 5)]
+
+
+@pytest.mark.parametrize("norm,bucket", VARIANTS)
+@pytest.mark.parametrize("n,d,bits", [(512, 64, 0), (1024, 128, 64)])
+def test_descent_variants_all_queries(alhr, synth, norm, bucket, n, d, bits, shape):
+    """Mean-normalised ranking and leaf buckets, with the predicted budget, every query."""
+    wl = synth.WORKLOADS["prefill_b4h8_n4096"].replace(
+        batch=2, heads=2, n=n, d=d, nq=n, score_bits=bits, seed=n + d + 10 * bucket + norm)
+    inp = synth.make_inputs(wl, "cuda")
+    res = _run_forward(alhr, wl, inp, score_norm=norm, bucket_log=bucket)
+    cpu = _to(inp, "cpu")
+    for b in range(wl.batch):
+        for h in range(wl.heads):
+            ref = oracle_slice(cpu, wl, b, h, score_norm=norm, bucket_log=bucket)
+            compare_rows(res, ref, b, h, np.arange(n), TOL, f"norm={norm} b={bucket} b{b}h{h}")
+    assert res["dev_err"] == 0
+
+
+@pytest.mark.parametrize("norm,bucket", [(False, 2), (True, 3), (True, 0)])
+def test_descent_variants_route_and_ties(alhr, synth, norm, bucket, shape):
+    """The route entry point with a budget override (values in {-1, 0, 1}: ties everywhere),
+    against the oracle and against the fused forward."""
+    wl = synth.WORKLOADS["tiny_prefill_n1024"].replace(n=512, nq=512, qk_lo=-1, qk_hi=1,
+                                                       seed=77 + bucket)
+    inp = synth.make_inputs(wl, "cuda")
+    vb = 1
+    tree = alhr.build_tree(inp["K"], value_bound=vb)
+    kw = dict(q_start=0, window=wl.window, max_keys=wl.max_keys, value_bound=vb,
+              score_norm=norm, bucket_log=bucket)
+    budget = inp["budget_override"]
+    r = alhr.route(inp["Q"], inp["K"], tree, budget, **kw)
+    f = alhr.forward(inp["Q"], inp["K"], inp["V"], tree, budget_override=budget, want_idx=True,
+                     want_count=True, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(r["idx"], f["idx"]) and torch.equal(r["count"], f["count"])
+    cpu = _to(inp, "cpu")
+    for b in range(wl.batch):
+        for h in range(wl.heads):
+            ref = oracle_slice(cpu, wl, b, h, score_norm=norm, bucket_log=bucket)
+            compare_rows({"idx": r["idx"], "count": r["count"], "out": f["out"]}, ref, b, h,
+                         np.arange(wl.nq), TOL, f"route norm={norm} b={bucket}")
+
+
 # ------------------------------------------------------------------ unfused entry points
 
 

@@ -1,5 +1,6 @@
 """The algorithmic byte model on hand-counted cases (N=8, d=2, w=2: the golden example), and
 the tree layout sizes."""
+import numpy as np
 import pytest
 
 from tree_routed_sparse_b200 import metrics
@@ -58,3 +59,18 @@ def test_tree_block_bytes(n, d, vb):
     assert narrow == ({(16384, 128): 10, (262144, 128): 10}.get((n, d), narrow))
     if d == 64:
         assert narrow == 0
+
+
+def test_bucket_keys_are_read_once_more():
+    """Same counters, buckets of 4: the routed keys' rows (count - window keys) are read once
+    more; a query whose routed budget holds no whole bucket reads no roots."""
+    d, n, w = 64, 1024, 16
+    pos = np.array([500])
+    exp = np.array([[20, 0, 20]])
+    base = metrics.forward_bytes(pos, n, d, w, [40], exp, [40], False)
+    with_b = metrics.forward_bytes(pos, n, d, w, [40], exp, [40], False, bucket_log=2)
+    assert with_b - base == (40 - 16) * d
+    none = np.array([[0, 0, 0]])
+    a = metrics.forward_bytes(pos, n, d, w, [16], none, [19], False, bucket_log=2)  # r = 3 < 4
+    b = metrics.forward_bytes(pos, n, d, w, [16], none, [19], False)                # r = 3
+    assert b - a == metrics._rows_bytes(np.array([500 - w + 1]), d, 0)[0]

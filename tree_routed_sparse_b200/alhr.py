@@ -40,7 +40,7 @@ class AlhrError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [(f, ctypes.c_int32) for f in
                 ("batch", "heads", "n", "d", "q_start", "nq", "window", "max_keys",
-                 "score_bits", "value_bound")]
+                 "score_bits", "value_bound", "score_norm", "bucket_log")]
 
 
 _lib = None
@@ -107,10 +107,12 @@ def _stream(device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
-def make_dims(Q, K, q_start=0, window=16, max_keys=96, score_bits=0, value_bound=16) -> Dims:
+def make_dims(Q, K, q_start=0, window=16, max_keys=96, score_bits=0, value_bound=16,
+              score_norm=False, bucket_log=0) -> Dims:
     B, H, n, d = K.shape
     nq = 0 if Q is None else Q.shape[2]
-    return Dims(B, H, n, d, q_start, nq, window, max_keys, score_bits, value_bound)
+    return Dims(B, H, n, d, q_start, nq, window, max_keys, score_bits, value_bound,
+                int(bool(score_norm)), int(bucket_log))
 
 
 def _want(t, dtype, shape, name):
@@ -198,8 +200,11 @@ def predict_budget(Q, K, tree, W, q_start=0, window=16, max_keys=96, score_bits=
 
 
 def route(Q, K, tree, budget, q_start=0, window=16, max_keys=96, score_bits=0,
-          value_bound=16, with_expansions=True, idx=None, count=None, dev_err=None) -> dict:
-    dims = make_dims(Q, K, q_start, window, max_keys, score_bits, value_bound)
+          value_bound=16, with_expansions=True, idx=None, count=None, dev_err=None,
+          score_norm=False, bucket_log=0) -> dict:
+    """The descent alone (score_norm / bucket_log select the descent variants)."""
+    dims = make_dims(Q, K, q_start, window, max_keys, score_bits, value_bound, score_norm,
+                     bucket_log)
     B, H, nq, d = Q.shape
     _want(budget, torch.int32, (B, H, nq), "budget")
     if idx is None:
@@ -232,9 +237,12 @@ def attend(Q, K, V, idx, count, q_start=0, window=16, max_keys=96, value_bound=1
 
 def forward(Q, K, V, tree, W=None, budget_override=None, q_start=0, window=16, max_keys=96,
             score_bits=0, value_bound=16, out=None, want_idx=False, want_count=False,
-            want_expansions=False, want_budget=False, dev_err=None) -> dict:
-    """The fused path. Returns a dict with `out` and the optional outputs asked for."""
-    dims = make_dims(Q, K, q_start, window, max_keys, score_bits, value_bound)
+            want_expansions=False, want_budget=False, dev_err=None, score_norm=False,
+            bucket_log=0) -> dict:
+    """The fused path. Returns a dict with `out` and the optional outputs asked for.
+    score_norm / bucket_log select the descent variants (include/alhr.h)."""
+    dims = make_dims(Q, K, q_start, window, max_keys, score_bits, value_bound, score_norm,
+                     bucket_log)
     B, H, nq, d = Q.shape
     dev = Q.device
     _want(Q, torch.int8, (B, H, nq, d), "Q")

@@ -43,14 +43,18 @@ alhr_status check_queries(const alhr_dims* d) {
   if (d->max_keys < 1) return ALHR_ERR_INVALID_ARG;
   if (d->max_keys > alhr::kMaxKeys) return ALHR_ERR_UNSUPPORTED;
   if (d->score_bits != 0 && d->score_bits != 32 && d->score_bits != 64) return ALHR_ERR_INVALID_ARG;
+  if (d->score_norm != 0 && d->score_norm != 1) return ALHR_ERR_INVALID_ARG;
+  if (d->bucket_log < 0 || d->bucket_log > 15) return ALHR_ERR_INVALID_ARG;
   return ALHR_OK;
 }
 
-// Largest |q . node| over every node a query can score: the biggest root of [0, i - w] has
-// level <= log2 n - 1, so |score| <= d * vb^2 * n/2 (and d * vb^2 for a key).
+// Largest |ranking value| over every node a query can score: the biggest root of [0, i - w]
+// has level <= log2 n - 1, so |q . node| <= d * vb^2 * n/2 (and d * vb^2 for a key); ranked by
+// means, a node's value is q . node << (log2 n - level), at most d * vb^2 * n.
 int64_t score_bound(const alhr_dims* d) {
   const int64_t vb = value_bound_of(d);
-  return int64_t(d->d) * vb * vb * (int64_t(d->n) / 2);
+  const int64_t per = int64_t(d->d) * vb * vb;
+  return d->score_norm ? per * int64_t(d->n) : per * (int64_t(d->n) / 2);
 }
 
 int resolve_bits(const alhr_dims* d, alhr_status* st) {
@@ -76,6 +80,8 @@ alhr::QueryArgs base_args(const alhr_dims* d) {
   a.num_queries = int64_t(d->batch) * d->heads * d->nq;
   a.scale = float(1.0 / std::sqrt(double(d->d)));
   a.tl = alhr::make_tree_layout(d->n, d->d, d->value_bound);
+  a.norm_l = d->score_norm ? a.L : 0;
+  a.bucket = d->bucket_log;
   return a;
 }
 

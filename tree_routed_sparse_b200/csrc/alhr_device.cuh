@@ -46,6 +46,8 @@ __device__ __forceinline__ long long level_row(int n, int level) {
 
 struct QueryArgs {
   int n, L, q_start, nq, window, max_keys, value_bound;
+  int norm_l;  // 0: rank candidates by q . node_sum; L: by q . node_sum << (L - level) (means)
+  int bucket;  // leaf bucket level: nodes of level <= bucket are not expanded (0: keys)
   long long num_queries;  // batch * heads * nq
   float scale;            // fl32(1/sqrt(d))
   const int8_t* Q;
@@ -369,8 +371,9 @@ __device__ __noinline__ int tie_cut(TieStarts<NS> ts, int need) {
 // lower start, and packs them into the front of the buffer. Exact: the r-th largest score T is
 // found by bisection on the integer score; candidates tied at T are then cut by bisection on
 // their start position (starts are distinct).
-template <typename S, int NS>
-__device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int lane) {
+template <typename S, int NS, bool NORM>
+__device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int lane,
+                                                int norm_l) {
   constexpr S kLow = ScoreLimits<S>::lowest;
   S sc[NS];
   int ds[NS];
@@ -380,6 +383,8 @@ __device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int
     const bool ok = e < C;
     sc[s] = ok ? B.cscore[e] : kLow;
     ds[s] = ok ? B.cdesc[e] : 0;
+    // ranking by means: q . sum / 2^level, scaled by 2^L to stay an exact integer
+    if (NORM && norm_l && ok) sc[s] = sc[s] * (S(1) << (norm_l - desc_level(ds[s])));
   }
   S mn = ScoreLimits<S>::highest, mx = kLow;
 #pragma unroll
@@ -438,20 +443,22 @@ __device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int
     if (keep) {
       const int pos = base + __popc(bal & lanemask_lt(lane));
       B.cdesc[pos] = ds[s];
-      B.cscore[pos] = sc[s];
+      B.cscore[pos] = (NORM && norm_l) ? S(sc[s] >> (norm_l - desc_level(ds[s]))) : sc[s];
     }
     base += __popc(bal);
   }
   __syncwarp();
 }
 
-template <typename S>
-__device__ __forceinline__ void select_top_r(WarpBuf<S>& B, int C, int r, int lane) {
+// NORM compiles in the ranking by means (norm_l != 0: scores scaled by 2^(norm_l - level)).
+template <typename S, bool NORM>
+__device__ __forceinline__ void select_top_r(WarpBuf<S>& B, int C, int r, int lane,
+                                             int norm_l) {
   __syncwarp();
   // two instantiations only: the fused kernel is large enough that instruction-cache misses
   // cost more than the spare slot comparisons (measured)
-  if (C <= 96) select_top_r_ns<S, 3>(B, C, r, lane);
-  else select_top_r_ns<S, 6>(B, C, r, lane);
+  if (C <= 96) select_top_r_ns<S, 3, NORM>(B, C, r, lane, norm_l);
+  else select_top_r_ns<S, 6, NORM>(B, C, r, lane, norm_l);
 }
 
 }  // namespace alhr

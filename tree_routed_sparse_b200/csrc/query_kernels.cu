@@ -17,6 +17,9 @@
 //      best r by an exact integer bisection (select_top_r);
 //   4. attention: the selected window keys are scored, routed keys keep the scores of the
 //      descent (their key rows are not read again), and the value rows are gathered.
+// Descent variants (runtime, both off by default): ranking by means (the selection scales each
+// candidate's sum by 2^(L - level)), and leaf buckets (nodes of level <= b are not expanded, the
+// beam keeps r >> b of them, and their keys are listed and scored after the descent).
 #include <atomic>
 #include <cuda_runtime.h>
 
@@ -128,6 +131,50 @@ __device__ __forceinline__ void child_pass(WarpBuf<S>& B, const char* Th, const 
   }
 }
 
+// Leaf buckets (descent variant): the kept nodes, all of level <= bucket, become the list of
+// their keys, each scored q . k, in place of the frontier; returns the number of keys. At most
+// r >> bucket nodes (< 64) and r keys (< 96). Out of line: only the bucket variant reaches it.
+template <typename S, int D>
+__device__ __noinline__ int expand_buckets(WarpBuf<S>& B, int nf, const int8_t* Kh, const RowQ q,
+                                           int lane) {
+  constexpr int TPR = Lay<D>::TPR;
+  constexpr int RPI = Lay<D>::RPI;
+  const int grp = lane / TPR, sub = lane % TPR;
+  int total = 0;
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    const int e = lane + 32 * s;
+    int sz = 0, st = 0;
+    if (e < nf) {
+      const int ds = B.cdesc[e];
+      sz = 1 << desc_level(ds);
+      st = desc_start(ds);
+    }
+    int incl = sz;  // inclusive scan of the bucket sizes over the lanes
+#pragma unroll
+    for (int off = 1; off < 32; off *= 2) {
+      const int y = __shfl_up_sync(kFull, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const int pos = total + incl - sz;
+    for (int t = 0; t < sz; ++t) B.xrow[pos + t] = st + t;
+    total += __shfl_sync(kFull, incl, 31);
+  }
+  __syncwarp();
+  for (int base = 0; base < total; base += RPI) {
+    const int k = base + grp;
+    int xp[4] = {0, 0, 0, 0};
+    if (k < total) ld_key<D>(Kh + (long long)B.xrow[k] * D, sub, xp);
+    const int sc = group_sum<int, TPR>(dot_key(q, xp));
+    if (k < total && sub == 0) {
+      B.cdesc[k] = make_desc(B.xrow[k], 0);
+      B.cscore[k] = S(sc);
+    }
+  }
+  __syncwarp();
+  return total;
+}
+
 // The selection in ascending order, -1 padded: the routed keys (all below the window) sorted by
 // rank counting, then the window keys. Out of line: only the route outputs ask for it.
 template <typename S>
@@ -171,7 +218,9 @@ __device__ __forceinline__ void ld_node32(const char* Th, const int8_t* Kh, int 
 // LAT selects the latency mode, for launches with too few queries to fill the GPU (decode): every
 // warp keeps many more rows in flight per pass (registers are no constraint at one CTA per SM),
 // so a descent step takes one or two round trips to memory instead of up to ten.
-template <typename S, int D, int MODE, bool LAT>
+// VAR compiles in the descent variants (ranking by means, leaf buckets; chosen at run time from
+// the arguments); without it the method's descent carries none of their code.
+template <typename S, int D, int MODE, bool LAT, bool VAR>
 __global__ void __launch_bounds__(kWarps * 32, LAT ? 1 : min_blocks_per_sm<S>())
     query_kernel(const QueryArgs a) {
   constexpr int TPR = Lay<D>::TPR;
@@ -211,6 +260,8 @@ __global__ void __launch_bounds__(kWarps * 32, LAT ? 1 : min_blocks_per_sm<S>())
   const int w = a.window;
   const long long tree_block = a.tl.block_bytes;
   const int narrow = kNarrow ? a.tl.narrow : 0;  // int16 levels 1 .. narrow (d = 128 only)
+  const int bucket = VAR ? a.bucket : 0;          // descent variants: leaf bucket level,
+  const int norm_l = VAR ? a.norm_l : 0;          // ranking by means (0: by sums)
   const long long stride = (long long)gridDim.x * kWarps;
 
   for (long long qi = (long long)blockIdx.x * kWarps + warp; qi < a.num_queries; qi += stride) {
@@ -384,7 +435,8 @@ __global__ void __launch_bounds__(kWarps * 32, LAT ? 1 : min_blocks_per_sm<S>())
 
     // ---- 3. descent of the past-only forest
     int nf = 0, exp_hi = 0, exp_l1 = 0, exp_wide = 0;
-    if (kDescend && r > 0) {  // r > 0 implies i >= w, i.e. M > 0
+    const int keep = r >> bucket;  // beam width in buckets (keys when bucket = 0)
+    if (kDescend && keep > 0) {    // r > 0 implies i >= w, i.e. M > 0
       // roots not yet scored: the blocks of [0, M) below the shared ones
       const unsigned rest = Mu & low_mask;
       const int nB = __popc(rest);
@@ -468,7 +520,7 @@ __global__ void __launch_bounds__(kWarps * 32, LAT ? 1 : min_blocks_per_sm<S>())
               fd[s] = B.cdesc[e];
               fs[s] = B.cscore[e];
               const int lv = desc_level(fd[s]);
-              cat[s] = lv == 0 ? 1 : (lv == 1 ? 4 : ((!kNarrow || lv - 1 > narrow) ? 2 : 3));
+              cat[s] = lv <= bucket ? 1 : (lv == 1 ? 4 : ((!kNarrow || lv - 1 > narrow) ? 2 : 3));
             }
             bl_[s] = __ballot_sync(kFull, cat[s] == 1);
             bw_[s] = __ballot_sync(kFull, cat[s] == 2);
@@ -482,7 +534,16 @@ __global__ void __launch_bounds__(kWarps * 32, LAT ? 1 : min_blocks_per_sm<S>())
         }
         const int nhi = nw + nn;  // tree-row children
         const int nx = nhi + nk;
-        if (nx == 0) break;
+        if (nx == 0) {
+          // nothing to expand; more nodes than the beam only when the roots are all buckets
+          if constexpr (VAR) {
+            if (nf > keep) {
+              select_top_r<S, true>(B, nf, keep, lane, norm_l);
+              nf = keep;
+            }
+          }
+          break;
+        }
         exp_hi += nhi;
         exp_l1 += nk;
         exp_wide += nw;
@@ -544,13 +605,15 @@ __global__ void __launch_bounds__(kWarps * 32, LAT ? 1 : min_blocks_per_sm<S>())
         for (int x0 = lane; x0 < nx; x0 += 32)
           put_children<S>(B, nl, x0, B.xdesc[x0], B.xscore[x0], B.xleft[x0]);
         const int C = nl + 2 * nx;
-        if (C > r) {
-          select_top_r<S>(B, C, r, lane);
-          nf = r;
+        if (C > keep) {
+          select_top_r<S, VAR>(B, C, keep, lane, norm_l);
+          nf = keep;
         } else {
           nf = C;
         }
       }
+      if constexpr (VAR)
+        if (bucket > 0) nf = expand_buckets<S, D>(B, nf, Kh, q, lane);
     }
 
     // ---- window key scores (attention only needs the selected ones)
@@ -711,7 +774,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(const QueryArgs a) 
 
 namespace {
 
-constexpr int kOccSlots = 40;
+constexpr int kOccSlots = 66;
 
 // Grid size of a persistent launch: the resident CTAs of every SM, capped by the work. The
 // per-device occupancy (and the opt-in to more than 48 KB of dynamic shared memory) is
@@ -743,13 +806,13 @@ int blocks_for(KernelT kernel, int slot, size_t smem, long long queries, cudaErr
   return int(need < cap ? need : cap);
 }
 
-template <typename S, int D, int MODE, bool LAT>
+template <typename S, int D, int MODE, bool LAT, bool VAR>
 cudaError_t launch_query_mode(const QueryArgs& a, cudaStream_t st) {
-  constexpr int slot = ((MODE * 2 + (D == 128 ? 1 : 0)) * 2 + (sizeof(S) == 8 ? 1 : 0)) * 2 +
-                       (LAT ? 1 : 0);
-  static_assert(slot < 32, "occupancy cache slot");
+  constexpr int slot = (((MODE * 2 + (D == 128 ? 1 : 0)) * 2 + (sizeof(S) == 8 ? 1 : 0)) * 2 +
+                        (LAT ? 1 : 0)) * 2 + (VAR ? 1 : 0);
+  static_assert(slot < 64, "occupancy cache slot");
   constexpr size_t smem = QuerySmem<S, D, MODE>::bytes;
-  auto kern = query_kernel<S, D, MODE, LAT>;
+  auto kern = query_kernel<S, D, MODE, LAT, VAR>;
   cudaError_t err;
   const int blocks = blocks_for(kern, slot, smem, a.num_queries, &err);
   if (err != cudaSuccess) return err;
@@ -777,8 +840,12 @@ cudaError_t launch_query(const QueryArgs& a, cudaStream_t st) {
     }
     lat = a.num_queries <= (long long)sms * kWarps;
   }
-  return lat ? launch_query_mode<S, D, MODE, true>(a, st)
-             : launch_query_mode<S, D, MODE, false>(a, st);
+  // the predictor alone never descends: it needs no variant instantiation
+  if (MODE != kPredictOnly && (a.norm_l != 0 || a.bucket != 0))
+    return lat ? launch_query_mode<S, D, MODE, true, MODE != kPredictOnly>(a, st)
+               : launch_query_mode<S, D, MODE, false, MODE != kPredictOnly>(a, st);
+  return lat ? launch_query_mode<S, D, MODE, true, false>(a, st)
+             : launch_query_mode<S, D, MODE, false, false>(a, st);
 }
 
 template <int MODE>
@@ -813,11 +880,11 @@ int query_launch_mode() { return g_launch_mode.load(std::memory_order_relaxed); 
 cudaError_t launch_attend(const QueryArgs& a, int d, cudaStream_t st) {
   cudaError_t err;
   if (d == 64) {
-    const int blocks = blocks_for(attend_kernel<64>, 32, 0, a.num_queries, &err);
+    const int blocks = blocks_for(attend_kernel<64>, 64, 0, a.num_queries, &err);
     if (err != cudaSuccess) return err;
     attend_kernel<64><<<blocks, kWarps * 32, 0, st>>>(a);
   } else {
-    const int blocks = blocks_for(attend_kernel<128>, 33, 0, a.num_queries, &err);
+    const int blocks = blocks_for(attend_kernel<128>, 65, 0, a.num_queries, &err);
     if (err != cudaSuccess) return err;
     attend_kernel<128><<<blocks, kWarps * 32, 0, st>>>(a);
   }

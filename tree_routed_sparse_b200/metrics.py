@@ -13,7 +13,8 @@ Row sizes: a key row d bytes, a tree row of a narrow level (at d = 128, value_bo
                                 exp_l1 * d
   value rows                    count * 2d (bf16)
   output row                    4d (fp32)
-plus the predictor weights (64 d) once per launch. Routed keys' rows are not re-read.
+plus the predictor weights (64 d) once per launch. Routed keys' rows are not re-read, except
+under the leaf-bucket variant, where the kept buckets' keys are read once to be scored.
 The tree build reads K once and writes every tree row once. The counters (count, the three
 expansion counters, budgets) come from the run's own outputs, which match the oracle's, so the
 byte total is exact for the run.
@@ -60,11 +61,14 @@ def _highest_bit(x: np.ndarray) -> np.ndarray:
 
 
 def forward_bytes(positions, n: int, d: int, window: int, count, expansions, budget,
-                  predictor: bool, max_keys: int = 96, value_bound: int = 16) -> int:
+                  predictor: bool, max_keys: int = 96, value_bound: int = 16,
+                  bucket_log: int = 0) -> int:
     """Algorithmic bytes of one alhr_forward launch over the given queries.
 
     positions: query positions i (any shape); count, budget: same shape; expansions: [..., 3]
-    (level >= 2 expanded, level 1 expanded, expanded with an int32 child row)."""
+    (level >= 2 expanded, level 1 expanded, expanded with an int32 child row). With leaf
+    buckets (bucket_log > 0) the descent runs only when r >> bucket_log > 0, and the keys of the
+    kept buckets are read once more to be scored."""
     narrow = narrow_levels(n, d, value_bound)
     i = np.asarray(positions, dtype=np.int64).ravel()
     count = np.asarray(count, dtype=np.int64).ravel()
@@ -84,8 +88,10 @@ def forward_bytes(positions, n: int, d: int, window: int, count, expansions, bud
     else:
         g_rows = np.zeros_like(i)
         rest = M
-    root_rows = np.where(r > 0, _rows_bytes(rest, d, narrow), 0)
+    root_rows = np.where((r >> bucket_log) > 0, _rows_bytes(rest, d, narrow), 0)
     descent = exp[:, 2] * 4 * d + (exp[:, 0] - exp[:, 2]) * 2 * d + exp[:, 1] * d
+    if bucket_log > 0:
+        descent = descent + (count - nsel_win) * d
     per_q = d + g_rows + root_rows + nsel_win * d + descent + count * 2 * d + 4 * d
     return int(per_q.sum()) + (64 * d if predictor else 0)
 
