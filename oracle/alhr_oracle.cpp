@@ -33,6 +33,8 @@
 //   R7  the reuse of what earlier queries found among their own neighbours (§Inference stage,
 //       third paragraph) is read as a cache that changes no selected set; ignored.
 //   R8  attention is softmax(q . k / sqrt(d)) . V over the selected keys, no temperature.
+//   R11 phase-2 labels: the top-k keys of a query's causal attention row are its k largest
+//       q . k, equal scores to the lower position (softmax keeps the order of the scores).
 // Two descent variants (off by default; both off is the method above):
 //   R9  mean-normalised scores: candidates are ranked by q . node_sum / 2^level, the mean of
 //       the keys beneath them (what block-sparse methods rank blocks by; page "ALHR把注意力
@@ -51,6 +53,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <utility>
 #include <vector>
 
 namespace {
@@ -305,6 +308,38 @@ void oracle_forward(int n, int d, int q_start, int nq, int w, int max_keys, int 
     for (int s = 0; s < max_keys; ++s) idx[int64_t(row) * max_keys + s] = s < c ? sel[size_t(s)] : -1;
     count[row] = c;
     budget_out[row] = budget;
+  }
+}
+
+// Phase-2 labels [README §Training stage, Phase 2: the dense model's attention matrix gives the
+// top-k keys of every query; §Results and Variables: k = 16]. Softmax is monotonic in the score,
+// so the top-k of an attention row are the k largest q . K[t] over the causal keys t <= i, taken
+// here as exact integers; equal scores go to the lower key position (R11). Writes, per query
+// row, labels[row][0..k) (positions, best first, -1 when fewer than k keys exist) and
+// scores[row][0..k) (the dot products, 0 in padded slots; scores may be NULL).
+void oracle_topk_labels(int n, int d, const int8_t* Q, const int8_t* K, int q_start, int nq,
+                        int k, int32_t* labels, int32_t* scores) {
+  (void)n;
+  std::vector<std::pair<int64_t, int64_t>> row;  // (score, position)
+  for (int r = 0; r < nq; ++r) {
+    const int i = q_start + r;
+    const int8_t* q = Q + int64_t(r) * d;
+    row.clear();
+    for (int64_t t = 0; t <= i; ++t) {
+      int64_t s = 0;
+      for (int u = 0; u < d; ++u) s += int64_t(q[u]) * int64_t(K[t * d + u]);
+      row.push_back({s, t});
+    }
+    std::sort(row.begin(), row.end(), [](const std::pair<int64_t, int64_t>& a,
+                                         const std::pair<int64_t, int64_t>& b) {
+      if (a.first != b.first) return a.first > b.first;
+      return a.second < b.second;
+    });
+    for (int j = 0; j < k; ++j) {
+      const bool ok = size_t(j) < row.size();
+      labels[int64_t(r) * k + j] = ok ? int32_t(row[size_t(j)].second) : -1;
+      if (scores) scores[int64_t(r) * k + j] = ok ? int32_t(row[size_t(j)].first) : 0;
+    }
   }
 }
 

@@ -58,6 +58,8 @@ def _configure(L):
     L.oracle_forward.argtypes = [I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, P, P,
                                  P]
     L.oracle_forward.restype = None
+    L.oracle_topk_labels.argtypes = [I, I, P, P, I, I, I, P, P]
+    L.oracle_topk_labels.restype = None
     return L
 
 
@@ -173,3 +175,16 @@ def forward(Q, K, V_bits, nodes, W, budget_override, q_start: int, window: int,
                          _p(nodes), _p(W), _p(bo), _p(rws), 0 if rws is None else len(rws),
                          _p(out), _p(idx), _p(count), _p(exp), _p(bud), _p(lv))
     return dict(out=out, idx=idx, count=count, expansions=exp, budget=bud, by_level=lv)
+
+
+def topk_labels(Q, K, q_start: int, k: int = 16):
+    """Phase-2 labels of one (b,h) block: Q int8 [nq, d], K int8 [n, d] -> (labels int32
+    [nq, k] best first, -1 padded; scores int32 [nq, k], 0 padded)."""
+    Q = _c(Q, np.int8)
+    K = _c(K, np.int8)
+    nq, d = Q.shape
+    labels = np.full((nq, k), -1, dtype=np.int32)
+    scores = np.zeros((nq, k), dtype=np.int32)
+    lib().oracle_topk_labels(K.shape[0], d, _p(Q), _p(K), q_start, nq, k, _p(labels),
+                             _p(scores))
+    return labels, scores

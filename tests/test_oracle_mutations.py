@@ -47,6 +47,10 @@ MUTATIONS = {
     "bucket_last_key_dropped": ("t < nd.start + (int64_t(1) << nd.level); ++t)",
                                 "t + 1 < nd.start + (int64_t(1) << nd.level); ++t)"),
     "bucket_roots_not_pruned": ("if (int64_t(frontier.size()) > keep) {", "if (false) {"),
+    "labels_exclude_own_key": ("for (int64_t t = 0; t <= i; ++t) {", "for (int64_t t = 0; t < i; ++t) {"),
+    "labels_ties_to_higher_position": ("      return a.second < b.second;", "      return a.second > b.second;"),
+    "labels_lowest_scores": ("      if (a.first != b.first) return a.first > b.first;",
+                             "      if (a.first != b.first) return a.first < b.first;"),
 }
 
 PIN_TESTS = [
@@ -69,6 +73,9 @@ PIN_TESTS = [
     ("bucket_wide", lambda g: pins.test_buckets_wide_beam_route_the_whole_past(2)),
     ("bucket_hand", lambda g: pins.test_bucket_hand_example()),
     ("bucket_roots", lambda g: pins.test_buckets_prune_roots_that_are_all_buckets()),
+    ("labels_numpy", lambda g: pins.test_labels_match_numpy(64, 8, 0, 16)),
+    ("labels_planted", lambda g: pins.test_labels_planted_keys_and_short_rows()),
+    ("labels_argmax", lambda g: pins.test_labels_top1_is_causal_argmax()),
 ]
 
 

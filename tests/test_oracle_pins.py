@@ -533,3 +533,65 @@ def test_expansions_by_level_add_up(golden_n8):
                 for l in range(1, b + 1):
                     expect[l] += 1 << (b - l)
         assert lv.tolist() == expect.tolist()
+
+
+# ---------------------------------------------------------------- phase-2 labels (top-k)
+
+
+def _labels_numpy(Q, K, q_start, k):
+    """Independent formulation: the full causal score matrix with numpy, then per row a stable
+    argsort of the negated scores (stable = equal scores keep ascending positions)."""
+    S = Q.astype(np.int64) @ K.astype(np.int64).T
+    nq = Q.shape[0]
+    lab = np.full((nq, k), -1, dtype=np.int32)
+    sc = np.zeros((nq, k), dtype=np.int32)
+    for r in range(nq):
+        i = q_start + r
+        row = S[r, : i + 1]
+        order = np.argsort(-row, kind="stable")[:k]
+        lab[r, : len(order)] = order
+        sc[r, : len(order)] = row[order]
+    return lab, sc
+
+
+@pytest.mark.parametrize("n,d,q_start,k", [(64, 8, 0, 16), (256, 64, 0, 16), (512, 16, 300, 16),
+                                           (128, 128, 5, 4), (32, 4, 0, 32)])
+def test_labels_match_numpy(n, d, q_start, k):
+    rng = _rng(n + d + q_start + k)
+    for lo, hi in ((-16, 16), (-1, 1)):  # the narrow range makes ties everywhere
+        K = _rand_qk(rng, (n, d), lo, hi)
+        Q = _rand_qk(rng, (n - q_start, d), lo, hi)
+        lab, sc = orc.topk_labels(Q, K, q_start, k)
+        ref_lab, ref_sc = _labels_numpy(Q, K, q_start, k)
+        assert np.array_equal(lab, ref_lab) and np.array_equal(sc, ref_sc)
+
+
+def test_labels_planted_keys_and_short_rows():
+    """K is zero except 16 planted keys that score 1..16 against q: every row at or after the
+    last planted key lists them from the best down; a row before it lists the planted keys
+    already seen, then zero-score keys by position; rows with fewer than k keys are padded."""
+    n, d = 256, 4
+    q = np.array([1, 0, 0, 0], dtype=np.int8)
+    K = np.zeros((n, d), dtype=np.int8)
+    pos = np.array([3, 9, 17, 30, 31, 44, 60, 61, 77, 90, 101, 120, 140, 141, 150, 199])
+    for v, p in enumerate(pos, start=1):
+        K[p, 0] = v
+    Q = np.tile(q, (n, 1))
+    lab, sc = orc.topk_labels(Q, K, 0, 16)
+    assert lab[255].tolist() == pos[::-1].tolist()
+    assert sc[255].tolist() == list(range(16, 0, -1))
+    seen = pos[pos <= 50][::-1].tolist()                       # 3, 9, 17, 30, 31, 44
+    zeros = [t for t in range(51) if t not in pos][: 16 - len(seen)]
+    assert lab[50].tolist() == seen + zeros
+    assert lab[2].tolist() == [0, 1, 2] + [-1] * 13 and sc[2].tolist() == [0] * 16
+
+
+def test_labels_top1_is_causal_argmax():
+    rng = _rng(17)
+    n, d = 300, 16
+    K = _rand_qk(rng, (n, d))
+    Q = _rand_qk(rng, (n, d))
+    lab, sc = orc.topk_labels(Q, K, 0, 1)
+    for i in range(n):
+        s = K[: i + 1].astype(np.int64) @ Q[i].astype(np.int64)
+        assert lab[i, 0] == int(np.argmax(s)) and sc[i, 0] == s.max()
