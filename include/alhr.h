@@ -81,6 +81,8 @@ typedef enum {
 #define ALHR_DEVERR_BUDGET_LOW  0x1u /* a budget < 1 was read; it was treated as 1          */
 #define ALHR_DEVERR_VALUE_RANGE 0x2u /* a Q or K value had |value| > value_bound            */
 #define ALHR_DEVERR_INDEX       0x4u /* alhr_attend: an idx entry outside [0, i] was skipped */
+#define ALHR_DEVERR_TIMEOUT     0x8u /* alhr_topk_labels: a bounded wait on the tensor core ran
+                                        out; that CTA's rows were not written                */
 
 /* Problem sizes, shared by every entry point. */
 typedef struct {
@@ -172,6 +174,26 @@ ALHR_API int32_t alhr_get_launch_mode(void);
  */
 ALHR_API alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, void* tree,
                                      uint32_t* dev_err, void* stream);
+
+/*
+ * alhr_topk_labels -- phase-2 labels [README §Training stage, Phase 2: the top-k keys of every
+ * query are read off the dense model's attention matrix; §Results and Variables: k = 16].
+ *
+ * For every (b,h) and query row r (position i = q_start + r) writes the k keys t <= i with the
+ * largest exact q . K[t] (the order softmax keeps), best first, equal scores to the lower t;
+ * rows with fewer than k causal keys are padded with -1 (and score 0). Scores are computed on
+ * the tensor cores (int8 x int8 -> int32, exact) tile by tile; nothing of size n x n is stored.
+ * Reads dims->batch, heads, n, d, q_start, nq.
+ *   Q       device, int8 [batch][heads][nq][d]; K device, int8 [batch][heads][n][d]
+ *   k       1 <= k <= 16
+ *   labels  device int32 [batch][heads][nq][k], written
+ *   scores  device int32 [batch][heads][nq][k] or NULL, written
+ *   dev_err device uint32 or NULL; ALHR_DEVERR_TIMEOUT if a bounded wait ran out (not expected)
+ * ALHR_ERR_INVALID_ARG for bad sizes or pointers (Q, K 16-byte aligned).
+ */
+ALHR_API alhr_status alhr_topk_labels(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
+                                      int32_t k, int32_t* labels, int32_t* scores,
+                                      uint32_t* dev_err, void* stream);
 
 /*
  * alhr_update_tree -- the tree after rows [lo, hi) of K changed, e.g. the keys of new tokens

@@ -22,13 +22,14 @@ STATUS = {0: "ALHR_OK", 1: "ALHR_ERR_INVALID_ARG", 2: "ALHR_ERR_UNSUPPORTED",
 DEVERR_BUDGET_LOW = 0x1
 DEVERR_VALUE_RANGE = 0x2
 DEVERR_INDEX = 0x4
+DEVERR_TIMEOUT = 0x8
 LAUNCH_MODES = {"auto": 0, "throughput": 1, "latency": 2}
 
 EXPORTS = ["alhr_tree_rows", "alhr_tree_narrow_levels", "alhr_tree_bytes",
            "alhr_tree_level_offset", "alhr_score_bits", "alhr_status_string", "alhr_build_info",
            "alhr_build_tree", "alhr_update_tree", "alhr_tree_unpack", "alhr_predict_budget",
            "alhr_route", "alhr_attend", "alhr_forward", "alhr_set_launch_mode",
-           "alhr_get_launch_mode"]
+           "alhr_get_launch_mode", "alhr_topk_labels"]
 
 
 class AlhrError(RuntimeError):
@@ -72,11 +73,12 @@ def lib() -> ctypes.CDLL:
         L.alhr_route.argtypes = [DP, P, P, P, P, P, P, P, P, P]
         L.alhr_attend.argtypes = [DP, P, P, P, P, P, P, P, P]
         L.alhr_forward.argtypes = [DP, P, P, P, P, P, P, P, P, P, P, P, P, P]
+        L.alhr_topk_labels.argtypes = [DP, P, P, I32, P, P, P, P]
         L.alhr_set_launch_mode.argtypes = [I32]
         L.alhr_get_launch_mode.argtypes, L.alhr_get_launch_mode.restype = [], I32
         for f in ("alhr_build_tree", "alhr_update_tree", "alhr_tree_unpack",
                   "alhr_predict_budget", "alhr_route", "alhr_attend", "alhr_forward",
-                  "alhr_set_launch_mode"):
+                  "alhr_set_launch_mode", "alhr_topk_labels"):
             getattr(L, f).restype = I32
         _lib = L
     return _lib
@@ -271,3 +273,24 @@ def forward(Q, K, V, tree, W=None, budget_override=None, q_start=0, window=16, m
                               _ptr(res.get("budget")), _ptr(dev_err), _stream(dev)),
            "alhr_forward")
     return res
+
+
+def topk_labels(Q, K, k: int = 16, q_start: int = 0, with_scores: bool = True,
+                labels=None, scores=None, dev_err=None) -> dict:
+    """Phase-2 labels: for every query, its k best causal keys by exact q . k (best first,
+    -1 padded), computed on the tensor cores. Q int8 [B,H,nq,d], K int8 [B,H,n,d]."""
+    dims = make_dims(Q, K, q_start)
+    B, H, nq, d = Q.shape
+    _want(Q, torch.int8, (B, H, nq, d), "Q")
+    _want(K, torch.int8, (B, H, K.shape[2], d), "K")
+    if labels is None:
+        labels = torch.empty((B, H, nq, k), dtype=torch.int32, device=Q.device)
+    if scores is None and with_scores:
+        scores = torch.empty((B, H, nq, k), dtype=torch.int32, device=Q.device)
+    _want(labels, torch.int32, (B, H, nq, k), "labels")
+    if scores is not None:
+        _want(scores, torch.int32, (B, H, nq, k), "scores")
+    _check(lib().alhr_topk_labels(ctypes.byref(dims), _ptr(Q), _ptr(K), int(k), _ptr(labels),
+                                  _ptr(scores), _ptr(dev_err), _stream(Q.device)),
+           "alhr_topk_labels")
+    return dict(labels=labels, scores=scores)

@@ -151,6 +151,21 @@ alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, void* tree,
                                            static_cast<cudaStream_t>(stream)));
 }
 
+alhr_status alhr_topk_labels(const alhr_dims* dims, const int8_t* Q, const int8_t* K, int32_t k,
+                             int32_t* labels, int32_t* scores, uint32_t* dev_err, void* stream) {
+  const alhr_status s = check_common(dims);
+  if (s != ALHR_OK) return s;
+  if (dims->q_start < 0 || dims->nq < 0 || int64_t(dims->q_start) + dims->nq > dims->n)
+    return ALHR_ERR_INVALID_ARG;
+  if (k < 1 || k > 16) return ALHR_ERR_INVALID_ARG;
+  if (dims->nq == 0) return ALHR_OK;
+  if (!Q || !K || !labels || !aligned16(Q) || !aligned16(K)) return ALHR_ERR_INVALID_ARG;
+  const long long bh = (long long)dims->batch * dims->heads;
+  return from_cuda(alhr::launch_topk_labels(Q, K, labels, scores, dims->n, dims->d,
+                                            dims->q_start, dims->nq, k, bh, dev_err,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 alhr_status alhr_update_tree(const alhr_dims* dims, const int8_t* K, void* tree, int32_t lo,
                              int32_t hi, uint32_t* dev_err, void* stream) {
   const alhr_status s = check_common(dims);

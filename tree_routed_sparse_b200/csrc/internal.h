@@ -29,6 +29,11 @@ cudaError_t launch_route(const QueryArgs& a, int d, int score_bits, cudaStream_t
 cudaError_t launch_predict(const QueryArgs& a, int d, int score_bits, cudaStream_t st);
 cudaError_t launch_attend(const QueryArgs& a, int d, cudaStream_t st);
 
+// Phase-2 labels: top-k keys of every query's causal q . K row (see label_kernels.cu).
+cudaError_t launch_topk_labels(const int8_t* Q, const int8_t* K, int32_t* labels,
+                               int32_t* scores, int n, int d, int q_start, int nq, int k,
+                               long long bh, uint32_t* dev_err, cudaStream_t st);
+
 // Process-wide launch shape of the per-query kernels: 0 auto, 1 throughput, 2 latency.
 void set_query_launch_mode(int mode);
 int query_launch_mode();

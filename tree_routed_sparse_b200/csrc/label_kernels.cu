@@ -1,0 +1,305 @@
+// label_kernels.cu -- phase-2 labels of ALHR on sm_100a: the top-k keys of every query's dense
+// causal attention row.
+//
+// README of ALHR, section "Training stage", Phase 2: the dense teacher's attention matrix is
+// read and the top-k keys of every query are labelled; section "Results and Variables": k = 16.
+// Softmax keeps the order of the scores, so the labels are the k largest exact q . k over the
+// causal keys t <= i, equal scores to the lower position.
+//
+// One CTA of 4 warps takes 128 queries of one (b,h). For every 128-key tile up to the tile's
+// last query position, the scores Q_tile . K_tile^T (int8 x int8 -> int32, exact) are computed by
+// the 5th-generation tensor core (tcgen05.mma kind::i8, M = N = 128, K = 32 per instruction) into
+// a 128 x 128 int32 accumulator in tensor memory; thread t then reads row t of it (tcgen05.ld,
+// one TMEM lane per thread) 32 columns at a time, queues the columns that beat its current 16th
+// best in shared memory, and inserts the queued ones into a sorted 16-entry list held in
+// registers. Operand tiles are staged with cp.async in the no-swizzle K-major core-matrix layout
+// (8 rows x 16 bytes per 128-byte core matrix). Every wait on the MMA's mbarrier is bounded; on
+// timeout the CTA stops, sets ALHR_DEVERR_TIMEOUT and still frees its tensor memory.
+#include <climits>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "alhr_device.cuh"
+#include "internal.h"
+
+namespace alhr {
+
+namespace {
+
+constexpr int kLT = 128;          // queries per CTA tile (M) and keys per key tile (N)
+constexpr int kLThreads = 128;    // warp w reads TMEM lanes 32w .. 32w+31: one query row each
+constexpr int kListK = 16;        // labels kept per query (k <= 16 is returned)
+constexpr int kTmemCols = 128;    // one 128 x 128 int32 accumulator
+constexpr uint32_t kWaitLimit = 1u << 24;  // bounded mbarrier polling
+
+template <int D>
+struct LabelSmem {
+  static constexpr int tile_bytes = kLT * D;                  // one int8 operand tile
+  static constexpr int q_off = 0;
+  static constexpr int k_off = tile_bytes;
+  static constexpr int queue_off = 2 * tile_bytes;            // [32][128] int32
+  static constexpr int misc_off = queue_off + 32 * kLThreads * 4;
+  static constexpr int used = misc_off + 64;
+  // Requested size: at most 4 CTAs per SM, so that their accumulators (4 x 128 columns) fit
+  // the 512 columns of tensor memory and no allocation ever waits on another CTA.
+  static constexpr int bytes = 56 * 1024;
+  static_assert(used <= bytes, "label kernel shared memory");
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Shared-memory matrix descriptor of tcgen05 (no swizzle): start address, leading byte offset
+// (between the 16-byte column blocks of a K-major tile), stride byte offset (between 8-row
+// groups), descriptor version 1 at bits 46-47, base offset 0, no swizzle.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// Instruction descriptor of tcgen05.mma kind::i8: int32 accumulator, signed int8 A and B, both
+// K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+constexpr uint32_t kIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) |
+                              (static_cast<uint32_t>(kLT >> 3) << 17) |
+                              (static_cast<uint32_t>(kLT >> 4) << 24);
+
+// Byte offset of (row, byte column kb) of an R x D int8 tile in the core-matrix layout.
+template <int D>
+__device__ __forceinline__ int core_offset(int row, int kb) {
+  return ((row >> 3) * (D / 16) + (kb >> 4)) * 128 + (row & 7) * 16 + (kb & 15);
+}
+
+// cp.async of a 16-byte row piece; src_bytes = 0 fills zeros (rows outside the matrix).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
+template <int D>
+__device__ __forceinline__ void load_tile(unsigned char* tile, const int8_t* base, int first_row,
+                                          int valid_rows, int tid) {
+  constexpr int CPR = D / 16;  // 16-byte chunks per row
+  for (int c = tid; c < kLT * CPR; c += kLThreads) {
+    const int r = c / CPR, kc = c - r * CPR;
+    const bool ok = r < valid_rows;
+    const int8_t* src = ok ? base + (static_cast<long long>(first_row) + r) * D + kc * 16 : base;
+    cp_async16(smem_u32(tile + core_offset<D>(r, kc * 16)), src, ok ? 16 : 0);
+  }
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t mbar, uint32_t phase) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(mbar), "r"(phase)
+      : "memory");
+  return done != 0;
+}
+
+// Insert (v, key) into the list sorted by score (descending); v beats the 16th entry, and key
+// is larger than every key in the list, so an equal score stays below the older entry.
+__device__ __forceinline__ void list_insert(int (&s)[kListK], int (&ix)[kListK], int v, int key) {
+#pragma unroll
+  for (int j = kListK - 1; j >= 1; --j) {
+    const bool up = v > s[j - 1];
+    const bool here = !up && v > s[j];
+    s[j] = up ? s[j - 1] : (here ? v : s[j]);
+    ix[j] = up ? ix[j - 1] : (here ? key : ix[j]);
+  }
+  const bool top = v > s[0];
+  s[0] = top ? v : s[0];
+  ix[0] = top ? key : ix[0];
+}
+
+template <int D>
+__global__ void __launch_bounds__(kLThreads, 4)
+    topk_label_kernel(const int8_t* __restrict__ Q, const int8_t* __restrict__ K,
+                      int32_t* __restrict__ labels, int32_t* __restrict__ scores, int n,
+                      int q_start, int nq, int k, long long bh_count, int tiles_per_head,
+                      uint32_t* dev_err) {
+  using L = LabelSmem<D>;
+  extern __shared__ __align__(1024) unsigned char lsm[];
+  unsigned char* sQ = lsm + L::q_off;
+  unsigned char* sK = lsm + L::k_off;
+  int* queue = reinterpret_cast<int*>(lsm + L::queue_off);
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(lsm + L::misc_off);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lsm + L::misc_off + 16);
+  int* abort_flag = reinterpret_cast<int*>(lsm + L::misc_off + 32);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  // the longest tiles (the last queries of every head) first
+  const long long bid = blockIdx.x;
+  const int qt = tiles_per_head - 1 - static_cast<int>(bid / bh_count);
+  const long long bh = bid - (bid / bh_count) * bh_count;
+  const int q0 = qt * kLT;
+  const int rows = min(kLT, nq - q0);
+  const int8_t* Qh = Q + bh * static_cast<long long>(nq) * D;
+  const int8_t* Kh = K + bh * static_cast<long long>(n) * D;
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(mbar)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    *abort_flag = 0;
+  }
+  load_tile<D>(sQ, Qh, q0, rows, tid);
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+
+  const int r = tid;  // this thread's query row in the tile (= its TMEM lane)
+  const bool row_ok = r < rows;
+  const int i = q_start + q0 + r;  // its position
+  const int i_last = q_start + q0 + rows - 1;
+  int s[kListK], ix[kListK];
+#pragma unroll
+  for (int j = 0; j < kListK; ++j) {
+    s[j] = INT_MIN;
+    ix[j] = -1;
+  }
+
+  const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK);
+  constexpr uint32_t kLbo = 128, kSbo = 8 * D;
+  uint32_t phase = 0;
+  for (int k0 = 0; k0 <= i_last; k0 += kLT) {
+    load_tile<D>(sK, Kh, k0, min(kLT, n - k0), tid);
+    asm volatile("cp.async.wait_all;\n" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    __syncthreads();
+    if (tid == 0) {
+      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+#pragma unroll
+      for (int ks = 0; ks < D / 32; ++ks) {
+        const uint64_t adesc = smem_desc(qa + ks * 256, kLbo, kSbo);
+        const uint64_t bdesc = smem_desc(ka + ks * 256, kLbo, kSbo);
+        asm volatile(
+            "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+            " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+            "l"(adesc), "l"(bdesc), "r"(kIdescI8), "r"(ks)
+            : "memory");
+      }
+      asm volatile(
+          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+              smem_u32(mbar))
+          : "memory");
+    }
+    bool ok = false;
+    for (uint32_t t = 0; t < kWaitLimit && !ok; ++t) ok = mbar_try_wait(smem_u32(mbar), phase);
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) {
+        *abort_flag = 1;
+        if (dev_err) atomicOr(dev_err, ALHR_DEVERR_TIMEOUT);
+      }
+      break;
+    }
+    phase ^= 1u;
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+
+#pragma unroll 1
+    for (int c = 0; c < kLT / 32; ++c) {
+      uint32_t v[32];
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + c * 32;
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+          "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+            "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+            "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+            "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+            "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+            "=r"(v[31])
+          : "r"(taddr)
+          : "memory");
+      asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+      // queue the columns that beat the current 16th best (score << 7 | column)
+      const int T = s[kListK - 1];
+      const int kbase = k0 + c * 32;
+      int cnt = 0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int sc = static_cast<int>(v[j]);
+        if (row_ok && kbase + j <= i && sc > T) {
+          queue[cnt * kLThreads + tid] = (sc << 7) | (c * 32 + j);
+          ++cnt;
+        }
+      }
+      const int rounds = __reduce_max_sync(0xffffffffu, cnt);
+      for (int e = 0; e < rounds; ++e) {
+        if (e < cnt) {
+          const int p = queue[e * kLThreads + tid];
+          const int sc = p >> 7;
+          if (sc > s[kListK - 1]) list_insert(s, ix, sc, k0 + (p & 127));
+        }
+      }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+    __syncthreads();
+  }
+
+  if (row_ok && !*abort_flag) {
+    const long long o = (bh * nq + q0 + r) * static_cast<long long>(k);
+#pragma unroll
+    for (int j = 0; j < kListK; ++j) {
+      if (j < k) {
+        labels[o + j] = ix[j];
+        if (scores) scores[o + j] = ix[j] >= 0 ? s[j] : 0;
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+}
+
+template <int D>
+cudaError_t launch_labels_d(const int8_t* Q, const int8_t* K, int32_t* labels, int32_t* scores,
+                            int n, int q_start, int nq, int k, long long bh, uint32_t* dev_err,
+                            cudaStream_t st) {
+  static bool configured[128] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 128 || !configured[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        topk_label_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, LabelSmem<D>::bytes);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 128) configured[dev] = true;
+  }
+  const int tiles = (nq + kLT - 1) / kLT;
+  const long long grid = bh * tiles;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  topk_label_kernel<D><<<static_cast<unsigned>(grid), kLThreads, LabelSmem<D>::bytes, st>>>(
+      Q, K, labels, scores, n, q_start, nq, k, bh, tiles, dev_err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_topk_labels(const int8_t* Q, const int8_t* K, int32_t* labels,
+                               int32_t* scores, int n, int d, int q_start, int nq, int k,
+                               long long bh, uint32_t* dev_err, cudaStream_t st) {
+  if (nq == 0 || bh == 0) return cudaSuccess;
+  return d == 64 ? launch_labels_d<64>(Q, K, labels, scores, n, q_start, nq, k, bh, dev_err, st)
+                 : launch_labels_d<128>(Q, K, labels, scores, n, q_start, nq, k, bh, dev_err, st);
+}
+
+}  // namespace alhr
