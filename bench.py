@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--impl", default="alhr", choices=["alhr", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--labels", action="store_true",
+                    help="instead of the bench line: time the phase-2 label kernel "
+                         "(alhr_topk_labels, top-16 keys of every query) on the workload (1 GPU)")
     ap.add_argument("--stages", action="store_true",
                     help="instead of the bench line: per-stage times of the workload through the "
                          "unfused entry points, and fused-forward time against N (1 GPU)")
@@ -448,6 +451,35 @@ def run_stages(args):
     print(json.dumps(report))
 
 
+def run_labels(args):
+    """The phase-2 label kernel on the workload's Q and K: one JSON line with its time, the
+    causal scores it ranks per second and the int8 tensor operations it issues."""
+    from tree_routed_sparse_b200 import alhr, synth
+    dev = torch.device("cuda", 0)
+    wl = synth.WORKLOADS[args.workload]
+    inp = synth.make_inputs(wl, dev)
+    Q, K = inp["Q"], inp["K"]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    shape = (wl.batch, wl.heads, wl.nq, 16)
+    lab = torch.empty(shape, dtype=torch.int32, device=dev)
+    sc = torch.empty(shape, dtype=torch.int32, device=dev)
+    run = lambda: alhr.topk_labels(Q, K, k=16, q_start=wl.q_start, labels=lab, scores=sc)
+    for _ in range(args.warmup):
+        run()
+    t = _event_time(run, max(args.steps, 3), flush)
+    i = np.arange(wl.q_start, wl.q_start + wl.nq, dtype=np.float64)
+    scores = float(wl.bh * (i + 1).sum())
+    tiles = 0  # 128-query x 64-key tensor-core tiles issued (each up to the tile's last query)
+    for q0 in range(0, wl.nq, 128):
+        last = wl.q_start + min(q0 + 128, wl.nq) - 1
+        tiles += last // 64 + 1
+    mma_ops = 2.0 * wl.bh * tiles * 128 * 64 * wl.d
+    print(json.dumps({"report": "labels", "workload": describe(wl), "k": 16,
+                      "ms": t * 1e3, "queries_per_s": wl.bh * wl.nq / t,
+                      "causal_scores_per_s": scores / t, "int8_tensor_tops": mma_ops / t / 1e12,
+                      "gpu": torch.cuda.get_device_name(dev)}))
+
+
 def profiled_traffic(workload: str):
     """DRAM bytes per launch of the fused kernel from the committed ncu summary, if that
     summary was taken on the kernel source as it is now; else None."""
@@ -495,6 +527,13 @@ def main():
         }))
         return
 
+    if args.labels:
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA device")
+        from tree_routed_sparse_b200 import build
+        build.build()
+        run_labels(args)
+        return
     if args.stages:
         if not torch.cuda.is_available():
             raise SystemExit("bench.py needs a CUDA device")

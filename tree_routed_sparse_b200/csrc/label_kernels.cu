@@ -6,14 +6,15 @@
 // Softmax keeps the order of the scores, so the labels are the k largest exact q . k over the
 // causal keys t <= i, equal scores to the lower position.
 //
-// One CTA of 4 warps takes 128 queries of one (b,h). For every 128-key tile up to the tile's
+// One CTA of 4 warps takes 128 queries of one (b,h). For every 64-key tile up to the tile's
 // last query position, the scores Q_tile . K_tile^T (int8 x int8 -> int32, exact) are computed by
-// the 5th-generation tensor core (tcgen05.mma kind::i8, M = N = 128, K = 32 per instruction) into
-// a 128 x 128 int32 accumulator in tensor memory; thread t then reads row t of it (tcgen05.ld,
-// one TMEM lane per thread) 32 columns at a time, queues the columns that beat its current 16th
-// best in shared memory, and inserts the queued ones into a sorted 16-entry list held in
-// registers. Operand tiles are staged with cp.async in the no-swizzle K-major core-matrix layout
-// (8 rows x 16 bytes per 128-byte core matrix). Every wait on the MMA's mbarrier is bounded; on
+// the 5th-generation tensor core (tcgen05.mma kind::i8, M = 128, N = 64, K = 32 per instruction)
+// into one of two 128 x 64 int32 accumulators in tensor memory, so that the next tile's cp.async
+// load and MMA run while this one is scanned; thread t reads row t of the accumulator
+// (tcgen05.ld, one TMEM lane per thread) 32 columns at a time, queues the columns that beat its
+// current 16th best in shared memory, and inserts the queued ones into a sorted 16-entry list
+// held in registers. Operand tiles are staged with cp.async in the no-swizzle K-major
+// core-matrix layout (8 rows x 16 bytes per 128-byte core matrix). Every wait on the MMA's mbarrier is bounded; on
 // timeout the CTA stops, sets ALHR_DEVERR_TIMEOUT and still frees its tensor memory.
 #include <climits>
 #include <cstdint>
@@ -26,18 +27,20 @@ namespace alhr {
 
 namespace {
 
-constexpr int kLT = 128;          // queries per CTA tile (M) and keys per key tile (N)
+constexpr int kLT = 128;          // queries per CTA tile (M)
+constexpr int kNT = 64;           // keys per key tile (N): two accumulators in flight
 constexpr int kLThreads = 128;    // warp w reads TMEM lanes 32w .. 32w+31: one query row each
 constexpr int kListK = 16;        // labels kept per query (k <= 16 is returned)
-constexpr int kTmemCols = 128;    // one 128 x 128 int32 accumulator
+constexpr int kTmemCols = 128;    // two 128 x 64 int32 accumulators
 constexpr uint32_t kWaitLimit = 1u << 24;  // bounded mbarrier polling
 
 template <int D>
 struct LabelSmem {
-  static constexpr int tile_bytes = kLT * D;                  // one int8 operand tile
+  static constexpr int q_bytes = kLT * D;                     // int8 query tile
+  static constexpr int k_bytes = kNT * D;                     // one int8 key tile
   static constexpr int q_off = 0;
-  static constexpr int k_off = tile_bytes;
-  static constexpr int queue_off = 2 * tile_bytes;            // [32][128] int32
+  static constexpr int k_off = q_bytes;                       // two key tiles
+  static constexpr int queue_off = q_bytes + 2 * k_bytes;     // [32][128] int32, one chunk
   static constexpr int misc_off = queue_off + 32 * kLThreads * 4;
   static constexpr int used = misc_off + 64;
   // Requested size: at most 4 CTAs per SM, so that their accumulators (4 x 128 columns) fit
@@ -65,7 +68,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 // Instruction descriptor of tcgen05.mma kind::i8: int32 accumulator, signed int8 A and B, both
 // K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
 constexpr uint32_t kIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) |
-                              (static_cast<uint32_t>(kLT >> 3) << 17) |
+                              (static_cast<uint32_t>(kNT >> 3) << 17) |
                               (static_cast<uint32_t>(kLT >> 4) << 24);
 
 // Byte offset of (row, byte column kb) of an R x D int8 tile in the core-matrix layout.
@@ -81,11 +84,11 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int sr
                : "memory");
 }
 
-template <int D>
+template <int D, int ROWS>
 __device__ __forceinline__ void load_tile(unsigned char* tile, const int8_t* base, int first_row,
                                           int valid_rows, int tid) {
   constexpr int CPR = D / 16;  // 16-byte chunks per row
-  for (int c = tid; c < kLT * CPR; c += kLThreads) {
+  for (int c = tid; c < ROWS * CPR; c += kLThreads) {
     const int r = c / CPR, kc = c - r * CPR;
     const bool ok = r < valid_rows;
     const int8_t* src = ok ? base + (static_cast<long long>(first_row) + r) * D + kc * 16 : base;
@@ -120,6 +123,43 @@ __device__ __forceinline__ void list_insert(int (&s)[kListK], int (&ix)[kListK],
   ix[0] = top ? key : ix[0];
 }
 
+// Queue the columns of 32 scores that beat the row's current 16th best, then insert them.
+// lim: columns j <= lim are causal keys of this row (lim >= 31: all of them).
+__device__ __forceinline__ void scan_chunk(const uint32_t (&v)[32], int lim, int col0, int k0,
+                                           int* queue, int tid, int (&s)[kListK],
+                                           int (&ix)[kListK]) {
+  const int T = s[kListK - 1];
+  int* qp = queue + tid;
+  if (lim >= 31) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int sc = static_cast<int>(v[j]);
+      if (sc > T) {
+        *qp = (sc << 7) | (col0 + j);
+        qp += kLThreads;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int sc = static_cast<int>(v[j]);
+      if (j <= lim && sc > T) {
+        *qp = (sc << 7) | (col0 + j);
+        qp += kLThreads;
+      }
+    }
+  }
+  const int cnt = static_cast<int>(qp - (queue + tid)) / kLThreads;
+  const int rounds = __reduce_max_sync(0xffffffffu, cnt);
+  for (int e = 0; e < rounds; ++e) {
+    if (e < cnt) {
+      const int p = queue[e * kLThreads + tid];
+      const int sc = p >> 7;
+      if (sc > s[kListK - 1]) list_insert(s, ix, sc, k0 + (p & 127));
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kLThreads, 4)
     topk_label_kernel(const int8_t* __restrict__ Q, const int8_t* __restrict__ K,
@@ -129,9 +169,9 @@ __global__ void __launch_bounds__(kLThreads, 4)
   using L = LabelSmem<D>;
   extern __shared__ __align__(1024) unsigned char lsm[];
   unsigned char* sQ = lsm + L::q_off;
-  unsigned char* sK = lsm + L::k_off;
+  unsigned char* sK = lsm + L::k_off;  // key tile b at sK + b * k_bytes
   int* queue = reinterpret_cast<int*>(lsm + L::queue_off);
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(lsm + L::misc_off);
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(lsm + L::misc_off);  // two barriers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lsm + L::misc_off + 16);
   int* abort_flag = reinterpret_cast<int*>(lsm + L::misc_off + 32);
 
@@ -145,6 +185,8 @@ __global__ void __launch_bounds__(kLThreads, 4)
   const int rows = min(kLT, nq - q0);
   const int8_t* Qh = Q + bh * static_cast<long long>(nq) * D;
   const int8_t* Kh = K + bh * static_cast<long long>(n) * D;
+  const int i_last = q_start + q0 + rows - 1;
+  const int ntiles = i_last / kNT + 1;  // key tiles [0, 64), [64, 128), ... up to i_last
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
@@ -155,10 +197,14 @@ __global__ void __launch_bounds__(kLThreads, 4)
   }
   if (tid == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(mbar)) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(mbar + 1)) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     *abort_flag = 0;
   }
-  load_tile<D>(sQ, Qh, q0, rows, tid);
+  // group 0: the query tile and key tile 0; group 1: key tile 1
+  load_tile<D, kLT>(sQ, Qh, q0, rows, tid);
+  load_tile<D, kNT>(sK, Kh, 0, min(kNT, n), tid);
+  if (ntiles > 1) load_tile<D, kNT>(sK + L::k_bytes, Kh, kNT, min(kNT, n - kNT), tid);
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
@@ -167,7 +213,6 @@ __global__ void __launch_bounds__(kLThreads, 4)
   const int r = tid;  // this thread's query row in the tile (= its TMEM lane)
   const bool row_ok = r < rows;
   const int i = q_start + q0 + r;  // its position
-  const int i_last = q_start + q0 + rows - 1;
   int s[kListK], ix[kListK];
 #pragma unroll
   for (int j = 0; j < kListK; ++j) {
@@ -177,31 +222,41 @@ __global__ void __launch_bounds__(kLThreads, 4)
 
   const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK);
   constexpr uint32_t kLbo = 128, kSbo = 8 * D;
-  uint32_t phase = 0;
-  for (int k0 = 0; k0 <= i_last; k0 += kLT) {
-    load_tile<D>(sK, Kh, k0, min(kLT, n - k0), tid);
-    asm volatile("cp.async.wait_all;\n" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-    __syncthreads();
-    if (tid == 0) {
-      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  // MMA of key tile t into accumulator t & 1, arriving on barrier t & 1 (thread 0)
+  auto issue_mma = [&](int t) {
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    const uint32_t kb = ka + (t & 1) * L::k_bytes;
 #pragma unroll
-      for (int ks = 0; ks < D / 32; ++ks) {
-        const uint64_t adesc = smem_desc(qa + ks * 256, kLbo, kSbo);
-        const uint64_t bdesc = smem_desc(ka + ks * 256, kLbo, kSbo);
-        asm volatile(
-            "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-            " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
-            "l"(adesc), "l"(bdesc), "r"(kIdescI8), "r"(ks)
-            : "memory");
-      }
+    for (int ks = 0; ks < D / 32; ++ks) {
+      const uint64_t adesc = smem_desc(qa + ks * 256, kLbo, kSbo);
+      const uint64_t bdesc = smem_desc(kb + ks * 256, kLbo, kSbo);
       asm volatile(
-          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
-              smem_u32(mbar))
+          "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+          " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+              tmem + (t & 1) * kNT),
+          "l"(adesc), "l"(bdesc), "r"(kIdescI8), "r"(ks)
           : "memory");
     }
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+            smem_u32(mbar + (t & 1)))
+        : "memory");
+  };
+
+  // prologue: wait for the query tile and key tile 0, start their MMA
+  if (ntiles > 1) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+  else asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+  __syncthreads();
+  if (tid == 0) issue_mma(0);
+
+  uint32_t phases = 0u;  // bit b: the parity to wait for on barrier b
+  for (int t = 0; t < ntiles; ++t) {
+    const int b = t & 1;
+    // 1. MMA t done: its accumulator is ready and its key buffer is free
     bool ok = false;
-    for (uint32_t t = 0; t < kWaitLimit && !ok; ++t) ok = mbar_try_wait(smem_u32(mbar), phase);
+    for (uint32_t w = 0; w < kWaitLimit && !ok; ++w)
+      ok = mbar_try_wait(smem_u32(mbar + b), (phases >> b) & 1u);
     if (__syncthreads_or(!ok)) {
       if (tid == 0) {
         *abort_flag = 1;
@@ -209,46 +264,53 @@ __global__ void __launch_bounds__(kLThreads, 4)
       }
       break;
     }
-    phase ^= 1u;
+    phases ^= 1u << b;
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-
-#pragma unroll 1
-    for (int c = 0; c < kLT / 32; ++c) {
-      uint32_t v[32];
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + c * 32;
-      asm volatile(
-          "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-          "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-            "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
-            "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
-            "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
-            "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
-            "=r"(v[31])
-          : "r"(taddr)
-          : "memory");
-      asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-      // queue the columns that beat the current 16th best (score << 7 | column)
-      const int T = s[kListK - 1];
-      const int kbase = k0 + c * 32;
-      int cnt = 0;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int sc = static_cast<int>(v[j]);
-        if (row_ok && kbase + j <= i && sc > T) {
-          queue[cnt * kLThreads + tid] = (sc << 7) | (c * 32 + j);
-          ++cnt;
-        }
-      }
-      const int rounds = __reduce_max_sync(0xffffffffu, cnt);
-      for (int e = 0; e < rounds; ++e) {
-        if (e < cnt) {
-          const int p = queue[e * kLThreads + tid];
-          const int sc = p >> 7;
-          if (sc > s[kListK - 1]) list_insert(s, ix, sc, k0 + (p & 127));
-        }
-      }
+    // 2. key tile t + 2 into the freed buffer (its own cp.async group)
+    if (t + 2 < ntiles) {
+      const int k2 = (t + 2) * kNT;
+      load_tile<D, kNT>(sK + b * L::k_bytes, Kh, k2, min(kNT, n - k2), tid);
     }
+    // 3. key tile t + 1 has landed: start its MMA into the other accumulator (read back in the
+    //    previous iteration, before that iteration's closing barrier)
+    if (t + 1 < ntiles) {
+      if (t + 2 < ntiles) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+      else asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      __syncthreads();
+      if (tid == 0) issue_mma(t + 1);
+    }
+    // 4. this thread's row of scores for tile t, 64 columns as two loads of 32
+    uint32_t v0[32], v1[32];
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + b * kNT;
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+        : "=r"(v0[0]), "=r"(v0[1]), "=r"(v0[2]), "=r"(v0[3]), "=r"(v0[4]), "=r"(v0[5]),
+          "=r"(v0[6]), "=r"(v0[7]), "=r"(v0[8]), "=r"(v0[9]), "=r"(v0[10]), "=r"(v0[11]),
+          "=r"(v0[12]), "=r"(v0[13]), "=r"(v0[14]), "=r"(v0[15]), "=r"(v0[16]), "=r"(v0[17]),
+          "=r"(v0[18]), "=r"(v0[19]), "=r"(v0[20]), "=r"(v0[21]), "=r"(v0[22]), "=r"(v0[23]),
+          "=r"(v0[24]), "=r"(v0[25]), "=r"(v0[26]), "=r"(v0[27]), "=r"(v0[28]), "=r"(v0[29]),
+          "=r"(v0[30]), "=r"(v0[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+        : "=r"(v1[0]), "=r"(v1[1]), "=r"(v1[2]), "=r"(v1[3]), "=r"(v1[4]), "=r"(v1[5]),
+          "=r"(v1[6]), "=r"(v1[7]), "=r"(v1[8]), "=r"(v1[9]), "=r"(v1[10]), "=r"(v1[11]),
+          "=r"(v1[12]), "=r"(v1[13]), "=r"(v1[14]), "=r"(v1[15]), "=r"(v1[16]), "=r"(v1[17]),
+          "=r"(v1[18]), "=r"(v1[19]), "=r"(v1[20]), "=r"(v1[21]), "=r"(v1[22]), "=r"(v1[23]),
+          "=r"(v1[24]), "=r"(v1[25]), "=r"(v1[26]), "=r"(v1[27]), "=r"(v1[28]), "=r"(v1[29]),
+          "=r"(v1[30]), "=r"(v1[31])
+        : "r"(taddr + 32)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+    const int k0 = t * kNT;
+    const int lim = row_ok ? i - k0 : -1;  // columns j <= lim are causal keys of this row
+    scan_chunk(v0, lim, 0, k0, queue, tid, s, ix);
+    scan_chunk(v1, lim - 32, 32, k0, queue, tid, s, ix);
+    // 5. accumulator t & 1 is read: the MMA of tile t + 2 may overwrite it
     asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
     __syncthreads();
   }
@@ -263,6 +325,7 @@ __global__ void __launch_bounds__(kLThreads, 4)
       }
     }
   }
+  asm volatile("cp.async.wait_all;\n" ::: "memory");  // nothing in flight after an abort
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
   if (warp == 0)
