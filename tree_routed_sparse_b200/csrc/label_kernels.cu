@@ -12,8 +12,8 @@
 // into one of two 128 x 64 int32 accumulators in tensor memory, so that the next tile's cp.async
 // load and MMA run while this one is scanned; thread t reads row t of the accumulator
 // (tcgen05.ld, one TMEM lane per thread) 32 columns at a time, queues the columns that beat its
-// current 16th best in shared memory, and inserts the queued ones into a sorted 16-entry list
-// held in registers. Operand tiles are staged with cp.async in the no-swizzle K-major
+// 16th best in shared memory, and inserts the queued ones in deferred rounds into a sorted
+// 16-entry list held in registers. Operand tiles are staged with cp.async in the no-swizzle K-major
 // core-matrix layout (8 rows x 16 bytes per 128-byte core matrix). Every wait on the MMA's mbarrier is bounded; on
 // timeout the CTA stops, sets ALHR_DEVERR_TIMEOUT and still frees its tensor memory.
 #include <climits>
@@ -40,12 +40,16 @@ struct LabelSmem {
   static constexpr int k_bytes = kNT * D;                     // one int8 key tile
   static constexpr int q_off = 0;
   static constexpr int k_off = q_bytes;                       // two key tiles
-  static constexpr int queue_off = q_bytes + 2 * k_bytes;     // [32][128] int32, one chunk
-  static constexpr int misc_off = queue_off + 32 * kLThreads * 4;
-  static constexpr int used = misc_off + 64;
   // Requested size: at most 4 CTAs per SM, so that their accumulators (4 x 128 columns) fit
   // the 512 columns of tensor memory and no allocation ever waits on another CTA.
-  static constexpr int bytes = 56 * 1024;
+  static constexpr int bytes = 56 * 1024 - 64;
+  static constexpr int misc_bytes = 64;
+  static constexpr int queue_off = q_bytes + 2 * k_bytes;     // [kQueue][128] int32
+  // candidates queued per thread before they are inserted (at least two chunks' worth)
+  static constexpr int kQueue = (bytes - misc_bytes - queue_off) / (kLThreads * 4);
+  static constexpr int misc_off = queue_off + kQueue * kLThreads * 4;
+  static constexpr int used = misc_off + misc_bytes;
+  static_assert(kQueue >= 40, "label queue");
   static_assert(used <= bytes, "label kernel shared memory");
 };
 
@@ -123,19 +127,23 @@ __device__ __forceinline__ void list_insert(int (&s)[kListK], int (&ix)[kListK],
   ix[0] = top ? key : ix[0];
 }
 
-// Queue the columns of 32 scores that beat the row's current 16th best, then insert them.
+// Candidates are queued in shared memory as (score << 9 | key - epoch), epoch a multiple of
+// 512 keys: |score| <= 128 * 128 * 128 = 2^21, so the word never overflows. They are inserted
+// in rounds (one per queued entry of the fullest lane of the warp), and only when the queue could
+// overflow or the 512-key epoch ends: rows add candidates rarely once their list is full, and a
+// round serves every lane at once, so deferring rounds saves most of them.
+constexpr int kEpochKeys = 512;
+
+// Queue the columns of 32 scores that beat the row's 16th best as of the last insertion round.
 // lim: columns j <= lim are causal keys of this row (lim >= 31: all of them).
-__device__ __forceinline__ void scan_chunk(const uint32_t (&v)[32], int lim, int col0, int k0,
-                                           int* queue, int tid, int (&s)[kListK],
-                                           int (&ix)[kListK]) {
-  const int T = s[kListK - 1];
-  int* qp = queue + tid;
+__device__ __forceinline__ int* queue_chunk(const uint32_t (&v)[32], int lim, int T, int key0,
+                                            int* qp) {
   if (lim >= 31) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const int sc = static_cast<int>(v[j]);
       if (sc > T) {
-        *qp = (sc << 7) | (col0 + j);
+        *qp = (sc << 9) | (key0 + j);
         qp += kLThreads;
       }
     }
@@ -144,20 +152,27 @@ __device__ __forceinline__ void scan_chunk(const uint32_t (&v)[32], int lim, int
     for (int j = 0; j < 32; ++j) {
       const int sc = static_cast<int>(v[j]);
       if (j <= lim && sc > T) {
-        *qp = (sc << 7) | (col0 + j);
+        *qp = (sc << 9) | (key0 + j);
         qp += kLThreads;
       }
     }
   }
-  const int cnt = static_cast<int>(qp - (queue + tid)) / kLThreads;
+  return qp;
+}
+
+// Insert this warp's queued candidates into the lists and empty the queues.
+__device__ __forceinline__ int* flush_queue(int* qbase, int* qp, int epoch, int (&s)[kListK],
+                                            int (&ix)[kListK]) {
+  const int cnt = static_cast<int>(qp - qbase) / kLThreads;
   const int rounds = __reduce_max_sync(0xffffffffu, cnt);
   for (int e = 0; e < rounds; ++e) {
     if (e < cnt) {
-      const int p = queue[e * kLThreads + tid];
-      const int sc = p >> 7;
-      if (sc > s[kListK - 1]) list_insert(s, ix, sc, k0 + (p & 127));
+      const int p = qbase[e * kLThreads];
+      const int sc = p >> 9;
+      if (sc > s[kListK - 1]) list_insert(s, ix, sc, epoch + (p & (kEpochKeys - 1)));
     }
   }
+  return qbase;
 }
 
 template <int D>
@@ -251,6 +266,9 @@ __global__ void __launch_bounds__(kLThreads, 4)
   if (tid == 0) issue_mma(0);
 
   uint32_t phases = 0u;  // bit b: the parity to wait for on barrier b
+  int* const qbase = queue + tid;  // this thread's queue column
+  int* qp = qbase;                 // next free entry
+  int epoch = 0;                   // key base of the queued entries
   for (int t = 0; t < ntiles; ++t) {
     const int b = t & 1;
     // 1. MMA t done: its accumulator is ready and its key buffer is free
@@ -308,13 +326,22 @@ __global__ void __launch_bounds__(kLThreads, 4)
     asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
     const int k0 = t * kNT;
     const int lim = row_ok ? i - k0 : -1;  // columns j <= lim are causal keys of this row
-    scan_chunk(v0, lim, 0, k0, queue, tid, s, ix);
-    scan_chunk(v1, lim - 32, 32, k0, queue, tid, s, ix);
+    if (k0 - epoch >= kEpochKeys) {        // the queued key offsets are relative to the epoch
+      qp = flush_queue(qbase, qp, epoch, s, ix);
+      epoch = k0;
+    }
+    if (__any_sync(0xffffffffu, qp - qbase > (L::kQueue - 32) * kLThreads))
+      qp = flush_queue(qbase, qp, epoch, s, ix);
+    qp = queue_chunk(v0, lim, s[kListK - 1], k0 - epoch, qp);
+    if (__any_sync(0xffffffffu, qp - qbase > (L::kQueue - 32) * kLThreads))
+      qp = flush_queue(qbase, qp, epoch, s, ix);
+    qp = queue_chunk(v1, lim - 32, s[kListK - 1], k0 + 32 - epoch, qp);
     // 5. accumulator t & 1 is read: the MMA of tile t + 2 may overwrite it
     asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
     __syncthreads();
   }
 
+  qp = flush_queue(qbase, qp, epoch, s, ix);
   if (row_ok && !*abort_flag) {
     const long long o = (bh * nq + q0 + r) * static_cast<long long>(k);
 #pragma unroll
