@@ -127,7 +127,7 @@ __device__ __forceinline__ void list_insert(int (&s)[kListK], int (&ix)[kListK],
   ix[0] = top ? key : ix[0];
 }
 
-// Candidates are queued in shared memory as (score << 9 | key - epoch), epoch a multiple of
+// Candidates are queued in shared memory as score * 512 + (key - epoch), epoch a multiple of
 // 512 keys: |score| <= 128 * 128 * 128 = 2^21, so the word never overflows. They are inserted
 // in rounds (one per queued entry of the fullest lane of the warp), and only when the queue could
 // overflow or the 512-key epoch ends: rows add candidates rarely once their list is full, and a
@@ -142,19 +142,17 @@ __device__ __forceinline__ int* queue_chunk(const uint32_t (&v)[32], int lim, in
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const int sc = static_cast<int>(v[j]);
-      if (sc > T) {
-        *qp = (sc << 9) | (key0 + j);
-        qp += kLThreads;
-      }
+      // written unconditionally to the next free entry (in bounds: a chunk starts with at
+      // least 32 free entries), kept only when the pointer moves on: no branch per score
+      *qp = sc * 512 + key0 + j;
+      qp += sc > T ? kLThreads : 0;
     }
   } else {
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const int sc = static_cast<int>(v[j]);
-      if (j <= lim && sc > T) {
-        *qp = (sc << 9) | (key0 + j);
-        qp += kLThreads;
-      }
+      *qp = sc * 512 + key0 + j;
+      qp += (j <= lim && sc > T) ? kLThreads : 0;
     }
   }
   return qp;
@@ -168,7 +166,7 @@ __device__ __forceinline__ int* flush_queue(int* qbase, int* qp, int epoch, int 
   for (int e = 0; e < rounds; ++e) {
     if (e < cnt) {
       const int p = qbase[e * kLThreads];
-      const int sc = p >> 9;
+      const int sc = p >> 9;  // floor division by 512: the key offset is the low 9 bits
       if (sc > s[kListK - 1]) list_insert(s, ix, sc, epoch + (p & (kEpochKeys - 1)));
     }
   }
