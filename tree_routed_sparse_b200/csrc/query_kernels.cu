@@ -54,8 +54,14 @@ struct QuerySmem {
   static constexpr bool kUsesW = (MODE == kForwardPredict || MODE == kPredictOnly);
   static constexpr size_t w_bytes =
       kUsesW ? size_t(32 * WLayout<D>::g_stride + 32 * WLayout<D>::q_stride) * 4 : 0;
-  static constexpr size_t bytes = w_bytes + kWarps * sizeof(WarpBuf<S>);
+  static constexpr size_t bytes_for(int warps) { return w_bytes + warps * sizeof(WarpBuf<S>); }
 };
+
+// Warps (queries in flight) per CTA: the latency shape runs 4, one per SM sub-partition, so that
+// a small launch spreads over twice as many SMs and no two of its queries share an issue slot.
+constexpr int kLatWarps = 4;
+template <bool LAT>
+constexpr int warps_per_cta() { return LAT ? kLatWarps : kWarps; }
 
 // Register budget: int32 scores keep three CTAs (24 warps) per SM with two tree rows in flight
 // per row group; int64 scores need more registers, so two CTAs and one row in flight.
@@ -221,8 +227,9 @@ __device__ __forceinline__ void ld_node32(const char* Th, const int8_t* Kh, int 
 // VAR compiles in the descent variants (ranking by means, leaf buckets; chosen at run time from
 // the arguments); without it the method's descent carries none of their code.
 template <typename S, int D, int MODE, bool LAT, bool VAR>
-__global__ void __launch_bounds__(kWarps * 32, LAT ? 1 : min_blocks_per_sm<S>())
+__global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_blocks_per_sm<S>())
     query_kernel(const QueryArgs a) {
+  constexpr int NW = warps_per_cta<LAT>();
   constexpr int TPR = Lay<D>::TPR;
   constexpr int RPI = Lay<D>::RPI;
   constexpr int U = LAT ? (D == 128 ? 8 : 4) : tree_rows_in_flight<S, D>();  // tree rows per group per pass
@@ -262,9 +269,9 @@ __global__ void __launch_bounds__(kWarps * 32, LAT ? 1 : min_blocks_per_sm<S>())
   const int narrow = kNarrow ? a.tl.narrow : 0;  // int16 levels 1 .. narrow (d = 128 only)
   const int bucket = VAR ? a.bucket : 0;          // descent variants: leaf bucket level,
   const int norm_l = VAR ? a.norm_l : 0;          // ranking by means (0: by sums)
-  const long long stride = (long long)gridDim.x * kWarps;
+  const long long stride = (long long)gridDim.x * NW;
 
-  for (long long qi = (long long)blockIdx.x * kWarps + warp; qi < a.num_queries; qi += stride) {
+  for (long long qi = (long long)blockIdx.x * NW + warp; qi < a.num_queries; qi += stride) {
     const long long bh = qi / a.nq;
     const int i = a.q_start + int(qi - bh * a.nq);
     const int8_t* Kh = a.K + bh * (long long)n * D;
@@ -780,7 +787,8 @@ constexpr int kOccSlots = 66;
 // per-device occupancy (and the opt-in to more than 48 KB of dynamic shared memory) is
 // computed once per device and kernel.
 template <typename KernelT>
-int blocks_for(KernelT kernel, int slot, size_t smem, long long queries, cudaError_t* err) {
+int blocks_for(KernelT kernel, int slot, size_t smem, long long queries, cudaError_t* err,
+               int warps = kWarps) {
   static thread_local int cached_dev = -1;
   static thread_local int sms = 0;
   static thread_local int per_sm[kOccSlots] = {0};
@@ -798,10 +806,10 @@ int blocks_for(KernelT kernel, int slot, size_t smem, long long queries, cudaErr
       if (*err != cudaSuccess) return 0;
     }
     int b = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, kWarps * 32, smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, warps * 32, smem);
     per_sm[slot] = b > 0 ? b : 1;
   }
-  const long long need = (queries + kWarps - 1) / kWarps;
+  const long long need = (queries + warps - 1) / warps;
   const long long cap = (long long)sms * per_sm[slot];
   return int(need < cap ? need : cap);
 }
@@ -811,13 +819,14 @@ cudaError_t launch_query_mode(const QueryArgs& a, cudaStream_t st) {
   constexpr int slot = (((MODE * 2 + (D == 128 ? 1 : 0)) * 2 + (sizeof(S) == 8 ? 1 : 0)) * 2 +
                         (LAT ? 1 : 0)) * 2 + (VAR ? 1 : 0);
   static_assert(slot < 64, "occupancy cache slot");
-  constexpr size_t smem = QuerySmem<S, D, MODE>::bytes;
+  constexpr int nw = warps_per_cta<LAT>();
+  constexpr size_t smem = QuerySmem<S, D, MODE>::bytes_for(nw);
   auto kern = query_kernel<S, D, MODE, LAT, VAR>;
   cudaError_t err;
-  const int blocks = blocks_for(kern, slot, smem, a.num_queries, &err);
+  const int blocks = blocks_for(kern, slot, smem, a.num_queries, &err, nw);
   if (err != cudaSuccess) return err;
   if (blocks <= 0) return cudaSuccess;
-  kern<<<blocks, kWarps * 32, smem, st>>>(a);
+  kern<<<blocks, nw * 32, smem, st>>>(a);
   return cudaGetLastError();
 }
 
