@@ -181,6 +181,33 @@ __device__ __noinline__ int expand_buckets(WarpBuf<S>& B, int nf, const int8_t* 
   return total;
 }
 
+// One pass over expanded nodes whose left child is an int16 tree row (positions [base, end) of
+// the x lists, all narrow): US rows per group, every load issued before any is scored.
+template <int US, typename S, int D>
+__device__ __forceinline__ void narrow_child_pass(WarpBuf<S>& B, const char* Th, const RowQ& q,
+                                                  int base, int end, int grp, int sub) {
+  constexpr int RPI = Lay<D>::RPI;
+  constexpr int TPR = Lay<D>::TPR;
+  int w[US][8];
+#pragma unroll
+  for (int u = 0; u < US; ++u) {
+    const int xi = base + u * RPI + grp;
+    if (xi < end) {
+      ld_tree16<D>(Th + B.xrow[xi], sub, w[u]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) w[u][j] = 0;
+    }
+  }
+  __syncwarp();  // reconverge before the group sums
+#pragma unroll
+  for (int u = 0; u < US; ++u) {
+    const int xi = base + u * RPI + grp;
+    const S left = group_sum<S, TPR>(S(dot_tree16(q, w[u])));
+    if (xi < end && sub == 0) B.xleft[xi] = left;
+  }
+}
+
 // The selection in ascending order, -1 padded: the routed keys (all below the window) sorted by
 // rank counting, then the window keys. Out of line: only the route outputs ask for it.
 template <typename S>
@@ -234,6 +261,7 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
   constexpr int RPI = Lay<D>::RPI;
   constexpr int U = LAT ? (D == 128 ? 8 : 4) : tree_rows_in_flight<S, D>();  // tree rows per group per pass
   constexpr int UK = LAT ? 8 : 1;  // key rows per group per pass
+  constexpr int UW = 4;            // latency shape, d = 128: int32 tree rows per group per pass
   constexpr int UV = LAT ? 8 : 2;  // value-row passes in flight
   constexpr bool kUsesW = (MODE == kForwardPredict || MODE == kPredictOnly);
   constexpr bool kDescend = (MODE != kPredictOnly);
@@ -585,9 +613,18 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
         __syncwarp();
         // left children that are tree rows: U rows per group in flight (a single pass body:
         // a separate short tail pass measured slower through instruction-cache misses)
-        for (int base = 0; base < nhi; base += U * RPI) {
-          if constexpr (kNarrow) child_pass<U, S, D>(B, Th, q, base, nw, nhi, grp, sub);
-          else tree_child_pass<U, S, D>(B, Th, q, base, nhi, grp, sub);
+        if constexpr (LAT && kNarrow) {
+          // latency shape: int32 and int16 rows in passes of their own, so that every pass
+          // issues all of its loads before it scores any (one memory round trip per pass)
+          for (int base = 0; base < nw; base += UW * RPI)
+            tree_child_pass<UW, S, D>(B, Th, q, base, nw, grp, sub);
+          for (int base = nw; base < nhi; base += U * RPI)
+            narrow_child_pass<U, S, D>(B, Th, q, base, nhi, grp, sub);
+        } else {
+          for (int base = 0; base < nhi; base += U * RPI) {
+            if constexpr (kNarrow) child_pass<U, S, D>(B, Th, q, base, nw, nhi, grp, sub);
+            else tree_child_pass<U, S, D>(B, Th, q, base, nhi, grp, sub);
+          }
         }
         // left children that are keys: UK rows per group in flight
         for (int base = nhi; base < nx; base += UK * RPI) {
