@@ -64,11 +64,13 @@ template <bool LAT>
 constexpr int warps_per_cta() { return LAT ? kLatWarps : kWarps; }
 
 // Register budget: int32 scores keep three CTAs (24 warps) per SM with two tree rows in flight
-// per row group; int64 scores need more registers, so two CTAs and one row in flight.
+// per row group; int64 scores need more registers, so two CTAs (and one int32 row in flight).
 template <typename S>
 constexpr int min_blocks_per_sm() { return sizeof(S) == 4 ? 3 : 2; }
+// At d = 128 this is the number of int16 rows (two 16-byte loads each) in flight; int32 rows at
+// d = 128 go one per pass.
 template <typename S, int D>
-constexpr int tree_rows_in_flight() { return (sizeof(S) == 4 && D == 64) ? 2 : 1; }
+constexpr int tree_rows_in_flight() { return D == 128 ? (sizeof(S) == 4 ? 3 : 2) : (sizeof(S) == 4 ? 2 : 1); }
 
 // One pass over expanded nodes whose left child is an int32 tree row: each row group loads US
 // rows (US in flight per lane) and leaves their scores in xleft.
@@ -93,46 +95,6 @@ __device__ __forceinline__ void tree_child_pass(WarpBuf<S>& B, const char* Th, c
   for (int u = 0; u < US; ++u) {
     const int xi = base + u * RPI + grp;
     const S left = group_sum<S, TPR>(dot_tree<S>(q, x[u]));
-    if (xi < end && sub == 0) B.xleft[xi] = left;
-  }
-}
-
-// One pass over expanded nodes whose left child is a tree row, the list ordered [int32 rows |
-// int16 rows] with `nw` int32 rows. Each row group takes US rows: the int16 rows' loads are
-// issued first, then the (few, upper-level) int32 rows are loaded and scored while those are in
-// flight, then the int16 rows are scored with two-way dp2a. Scores go to xleft.
-template <int US, typename S, int D>
-__device__ __forceinline__ void child_pass(WarpBuf<S>& B, const char* Th, const RowQ& q, int base,
-                                           int nw, int end, int grp, int sub) {
-  constexpr int RPI = Lay<D>::RPI;
-  constexpr int TPR = Lay<D>::TPR;
-  int w[US][8];
-#pragma unroll
-  for (int u = 0; u < US; ++u) {
-    const int xi = base + u * RPI + grp;
-    if (xi >= nw && xi < end) {
-      ld_tree16<D>(Th + B.xrow[xi], sub, w[u]);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) w[u][j] = 0;
-    }
-  }
-  S wide[US];
-#pragma unroll
-  for (int u = 0; u < US; ++u) {
-    const int xi = base + u * RPI + grp;
-    wide[u] = 0;
-    if (xi < nw) {
-      int x[16];
-      ld_tree<D>(Th + B.xrow[xi], sub, x);
-      wide[u] = dot_tree<S>(q, x);
-    }
-  }
-  if constexpr (US > 2) __syncwarp();  // latency shape: reconverge before the group sums
-#pragma unroll
-  for (int u = 0; u < US; ++u) {
-    const int xi = base + u * RPI + grp;
-    const S left = group_sum<S, TPR>(xi < nw ? wide[u] : S(dot_tree16(q, w[u])));
     if (xi < end && sub == 0) B.xleft[xi] = left;
   }
 }
@@ -261,7 +223,7 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
   constexpr int RPI = Lay<D>::RPI;
   constexpr int U = LAT ? (D == 128 ? 8 : 4) : tree_rows_in_flight<S, D>();  // tree rows per group per pass
   constexpr int UK = LAT ? 8 : 1;  // key rows per group per pass
-  constexpr int UW = 4;            // latency shape, d = 128: int32 tree rows per group per pass
+  constexpr int UW = LAT ? 4 : 1;  // d = 128: int32 tree rows per group per pass
   constexpr int UV = LAT ? 8 : 2;  // value-row passes in flight
   constexpr bool kUsesW = (MODE == kForwardPredict || MODE == kPredictOnly);
   constexpr bool kDescend = (MODE != kPredictOnly);
@@ -613,18 +575,16 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
         __syncwarp();
         // left children that are tree rows: U rows per group in flight (a single pass body:
         // a separate short tail pass measured slower through instruction-cache misses)
-        if constexpr (LAT && kNarrow) {
-          // latency shape: int32 and int16 rows in passes of their own, so that every pass
-          // issues all of its loads before it scores any (one memory round trip per pass)
+        if constexpr (kNarrow) {
+          // int32 and int16 rows in passes of their own, so that every pass issues all of its
+          // loads before it scores any (one memory round trip per pass)
           for (int base = 0; base < nw; base += UW * RPI)
             tree_child_pass<UW, S, D>(B, Th, q, base, nw, grp, sub);
           for (int base = nw; base < nhi; base += U * RPI)
             narrow_child_pass<U, S, D>(B, Th, q, base, nhi, grp, sub);
         } else {
-          for (int base = 0; base < nhi; base += U * RPI) {
-            if constexpr (kNarrow) child_pass<U, S, D>(B, Th, q, base, nw, nhi, grp, sub);
-            else tree_child_pass<U, S, D>(B, Th, q, base, nhi, grp, sub);
-          }
+          for (int base = 0; base < nhi; base += U * RPI)
+            tree_child_pass<U, S, D>(B, Th, q, base, nhi, grp, sub);
         }
         // left children that are keys: UK rows per group in flight
         for (int base = nhi; base < nx; base += UK * RPI) {
