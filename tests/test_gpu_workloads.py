@@ -94,3 +94,37 @@ def test_workload_parity(alhr, name, blocks):
         print(f"recall@selection {hits / (wl.batch * wl.heads * wl.plant_pairs):.3f}")
     del inp, tree, full, bench_out
     torch.cuda.empty_cache()
+
+
+def test_largest_sequence_decode_and_update(alhr):
+    """n = 2^20 keys (the largest the layout supports, 20 tree levels), d = 128, int64 scores:
+    the tree against the oracle, decode-style queries at the end of the sequence against the
+    oracle in both launch shapes, and a one-key update against a full build."""
+    from tree_routed_sparse_b200 import synth
+    n = 1 << 20
+    wl = synth.WORKLOADS["decode_s64h8_n262144_d128"].replace(batch=1, heads=2, n=n,
+                                                              q_start=n - 4, nq=4, seed=20)
+    inp = synth.make_inputs(wl, "cuda")
+    tree = alhr.build_tree(inp["K"])
+    kw = dict(q_start=wl.q_start, window=wl.window, max_keys=wl.max_keys,
+              score_bits=wl.score_bits)
+    cpu = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
+    tc = tree.cpu().numpy()
+    for h in range(wl.heads):
+        nodes = orc.build_tree(cpu["K"][0, h].numpy())
+        assert np.array_equal(decode_tree(tc[0, h], n, wl.d), nodes), h
+        ref = oracle_slice(cpu, wl, 0, h, nodes=nodes)
+        for shape in ("latency", "throughput"):
+            alhr.set_launch_mode(shape)
+            try:
+                res = alhr.forward(inp["Q"], inp["K"], inp["V"], tree, W=inp["W"], want_idx=True,
+                                   want_count=True, want_expansions=True, want_budget=True,
+                                   **kw)
+                torch.cuda.synchronize()
+            finally:
+                alhr.set_launch_mode("auto")
+            compare_rows(res, ref, 0, h, np.arange(wl.nq), TOL, f"n=2^20 {shape} h{h}")
+    K2 = inp["K"].clone()
+    K2[:, :, n - 1] = -K2[:, :, n - 1]
+    alhr.update_tree(K2, tree, n - 1, n)
+    assert torch.equal(tree, alhr.build_tree(K2))
