@@ -70,7 +70,9 @@ constexpr int min_blocks_per_sm() { return sizeof(S) == 4 ? 3 : 2; }
 // At d = 128 this is the number of int16 rows (two 16-byte loads each) in flight; int32 rows at
 // d = 128 go one per pass.
 template <typename S, int D>
-constexpr int tree_rows_in_flight() { return D == 128 ? (sizeof(S) == 4 ? 3 : 2) : (sizeof(S) == 4 ? 2 : 1); }
+constexpr int tree_rows_in_flight() {
+  return D == 128 ? (sizeof(S) == 4 ? 3 : 2) : (sizeof(S) == 4 ? 2 : 1);
+}
 
 // One pass over expanded nodes whose left child is an int32 tree row: each row group loads US
 // rows (US in flight per lane) and leaves their scores in xleft.
@@ -221,7 +223,8 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
   constexpr int NW = warps_per_cta<LAT>();
   constexpr int TPR = Lay<D>::TPR;
   constexpr int RPI = Lay<D>::RPI;
-  constexpr int U = LAT ? (D == 128 ? 8 : 4) : tree_rows_in_flight<S, D>();  // tree rows per group per pass
+  // tree rows per group per pass (at d = 128: int16 rows; int32 rows take UW)
+  constexpr int U = LAT ? (D == 128 ? 8 : 4) : tree_rows_in_flight<S, D>();
   constexpr int UK = LAT ? 8 : 1;  // key rows per group per pass
   constexpr int UW = LAT ? 4 : 1;  // d = 128: int32 tree rows per group per pass
   constexpr int UV = LAT ? 8 : 2;  // value-row passes in flight
@@ -829,9 +832,8 @@ cudaError_t launch_query_mode(const QueryArgs& a, cudaStream_t st) {
 
 std::atomic<int> g_launch_mode{0};
 
-// Auto: a launch whose queries fit one warp each at one CTA per SM (8 per SM) cannot fill the
-// GPU, so it takes the latency shape; measured on B200 the throughput shape wins from about 2048
-// queries up.
+// Auto: a launch of at most 8 queries per SM (one warp each) cannot fill the GPU, so it takes
+// the latency shape; measured on B200 the throughput shape wins from about 2048 queries up.
 template <typename S, int D, int MODE>
 cudaError_t launch_query(const QueryArgs& a, cudaStream_t st) {
   const int mode = g_launch_mode.load(std::memory_order_relaxed);
