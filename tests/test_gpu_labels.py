@@ -55,6 +55,12 @@ def test_labels_prefill_all_rows(alhr, synth, n, d):
     _check(alhr, synth, 2, 3, n, d, 0, n, 16, -16, 16, seed=n + d)
 
 
+@pytest.mark.parametrize("n,d", [(2, 64), (8, 128), (32, 64)])
+def test_labels_smallest_sequences(alhr, synth, n, d):
+    """Fewer keys than a tile and than the 16 labels: short rows padded with -1."""
+    _check(alhr, synth, 2, 2, n, d, 0, n, 16, -16, 16, seed=n)
+
+
 @pytest.mark.parametrize("q_start,nq", [(5, 200), (1000, 24), (2047, 1), (0, 129)])
 def test_labels_query_ranges(alhr, synth, q_start, nq):
     _check(alhr, synth, 2, 2, 2048, 64, q_start, nq, 16, -16, 16, seed=q_start + nq)

@@ -192,6 +192,20 @@ def test_decode_style_queries(alhr, synth, shape):
             compare_rows(res, oracle_slice(cpu, wl, b, h), b, h, np.arange(7), TOL, "decode")
 
 
+@pytest.mark.parametrize("n,d", [(2, 64), (4, 128), (8, 64), (16, 128)])
+def test_forward_smallest_sequences(alhr, synth, n, d, shape):
+    """The smallest trees (one to four levels), every query, predicted budgets."""
+    wl = synth.WORKLOADS["prefill_b4h8_n4096"].replace(batch=2, heads=3, n=n, d=d, nq=n,
+                                                      window=2, seed=n + d)
+    inp = synth.make_inputs(wl, "cuda")
+    res = _run_forward(alhr, wl, inp)
+    cpu = _to(inp, "cpu")
+    for b in range(wl.batch):
+        for h in range(wl.heads):
+            compare_rows(res, oracle_slice(cpu, wl, b, h), b, h, np.arange(n), TOL, f"n={n}")
+    assert res["dev_err"] == 0
+
+
 # ------------------------------------------------------------------ descent variants
 
 
