@@ -40,11 +40,13 @@ struct LabelSmem {
   static constexpr int k_bytes = kNT * D;                     // one int8 key tile
   static constexpr int q_off = 0;
   static constexpr int k_off = q_bytes;                       // two key tiles
-  // Requested size: at most 4 CTAs per SM, so that their accumulators (4 x 128 columns) fit
-  // the 512 columns of tensor memory and no allocation ever waits on another CTA.
-  static constexpr int bytes = 56 * 1024 - 64;
+  // Requested size: at most 4 CTAs per SM (3 at d = 128), so that their accumulators (128
+  // columns each) fit the 512 columns of tensor memory and no allocation ever waits on another
+  // CTA.
+  static constexpr int bytes = (D == 64 ? 56 : 74) * 1024 - 64;
   static constexpr int misc_bytes = 64;
-  static constexpr int queue_off = q_bytes + 2 * k_bytes;     // [kQueue][128] int32
+  static constexpr int row_off = q_bytes + 2 * k_bytes;       // [128][36] int32: a chunk per row
+  static constexpr int queue_off = row_off + kLThreads * 36 * 4;  // [kQueue][128] int32
   // candidates queued per thread before they are inserted (at least two chunks' worth)
   static constexpr int kQueue = (bytes - misc_bytes - queue_off) / (kLThreads * 4);
   static constexpr int misc_off = queue_off + kQueue * kLThreads * 4;
@@ -136,24 +138,25 @@ constexpr int kEpochKeys = 512;
 
 // Queue the columns of 32 scores that beat the row's 16th best as of the last insertion round.
 // lim: columns j <= lim are causal keys of this row (lim >= 31: all of them).
+// The candidates are found as a bit mask (two instructions per score); the chunk is parked in the
+// thread's row of shared memory so that only the candidates are read back and queued.
 __device__ __forceinline__ int* queue_chunk(const uint32_t (&v)[32], int lim, int T, int key0,
-                                            int* qp) {
-  if (lim >= 31) {
+                                            int* qp, int* rowp) {
+  unsigned mask = 0u;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int sc = static_cast<int>(v[j]);
-      // written unconditionally to the next free entry (in bounds: a chunk starts with at
-      // least 32 free entries), kept only when the pointer moves on: no branch per score
-      *qp = sc * 512 + key0 + j;
-      qp += sc > T ? kLThreads : 0;
-    }
-  } else {
+  for (int j = 0; j < 32; ++j)
+    if (static_cast<int>(v[j]) > T) mask |= 1u << j;
+  if (lim < 31) mask &= lim < 0 ? 0u : ((2u << lim) - 1u);
+  int4* r4 = reinterpret_cast<int4*>(rowp);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int sc = static_cast<int>(v[j]);
-      *qp = sc * 512 + key0 + j;
-      qp += (j <= lim && sc > T) ? kLThreads : 0;
-    }
+  for (int j = 0; j < 8; ++j)
+    r4[j] = make_int4(static_cast<int>(v[4 * j]), static_cast<int>(v[4 * j + 1]),
+                      static_cast<int>(v[4 * j + 2]), static_cast<int>(v[4 * j + 3]));
+  while (mask) {
+    const int j = __ffs(mask) - 1;
+    mask &= mask - 1u;
+    *qp = rowp[j] * 512 + key0 + j;
+    qp += kLThreads;
   }
   return qp;
 }
@@ -174,7 +177,7 @@ __device__ __forceinline__ int* flush_queue(int* qbase, int* qp, int epoch, int 
 }
 
 template <int D>
-__global__ void __launch_bounds__(kLThreads, 4)
+__global__ void __launch_bounds__(kLThreads, D == 64 ? 4 : 3)
     topk_label_kernel(const int8_t* __restrict__ Q, const int8_t* __restrict__ K,
                       int32_t* __restrict__ labels, int32_t* __restrict__ scores, int n,
                       int q_start, int nq, int k, long long bh_count, int tiles_per_head,
@@ -184,6 +187,7 @@ __global__ void __launch_bounds__(kLThreads, 4)
   unsigned char* sQ = lsm + L::q_off;
   unsigned char* sK = lsm + L::k_off;  // key tile b at sK + b * k_bytes
   int* queue = reinterpret_cast<int*>(lsm + L::queue_off);
+  int* rowp = reinterpret_cast<int*>(lsm + L::row_off) + threadIdx.x * 36;
   uint64_t* mbar = reinterpret_cast<uint64_t*>(lsm + L::misc_off);  // two barriers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lsm + L::misc_off + 16);
   int* abort_flag = reinterpret_cast<int*>(lsm + L::misc_off + 32);
@@ -330,10 +334,10 @@ __global__ void __launch_bounds__(kLThreads, 4)
     }
     if (__any_sync(0xffffffffu, qp - qbase > (L::kQueue - 32) * kLThreads))
       qp = flush_queue(qbase, qp, epoch, s, ix);
-    qp = queue_chunk(v0, lim, s[kListK - 1], k0 - epoch, qp);
+    qp = queue_chunk(v0, lim, s[kListK - 1], k0 - epoch, qp, rowp);
     if (__any_sync(0xffffffffu, qp - qbase > (L::kQueue - 32) * kLThreads))
       qp = flush_queue(qbase, qp, epoch, s, ix);
-    qp = queue_chunk(v1, lim - 32, s[kListK - 1], k0 + 32 - epoch, qp);
+    qp = queue_chunk(v1, lim - 32, s[kListK - 1], k0 + 32 - epoch, qp, rowp);
     // 5. accumulator t & 1 is read: the MMA of tile t + 2 may overwrite it
     asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
     __syncthreads();
