@@ -474,7 +474,8 @@ def run_labels(args):
 
 def profiled_traffic(workload: str):
     """DRAM bytes per launch of the fused kernel from the committed ncu summary, if that
-    summary was taken on the kernel source as it is now; else None."""
+    summary was taken on the fused kernel's source (query_kernels.cu and the headers) as it is
+    now; else None."""
     path = os.path.join(HERE, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -484,7 +485,7 @@ def profiled_traffic(workload: str):
     if not rec:
         return None
     from tree_routed_sparse_b200 import build
-    if rec.get("source_hash") != build._hash():
+    if rec.get("source_hash") != build.kernel_hash("query_kernels.cu"):
         return None
     return rec.get("dram_bytes_per_launch")
 

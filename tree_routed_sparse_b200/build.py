@@ -44,6 +44,24 @@ def _hash() -> str:
     return h.hexdigest()
 
 
+HEADERS = ["alhr_device.cuh", "internal.h", "tree_layout.h"]
+
+
+def kernel_hash(source: str) -> str:
+    """Hash of one csrc/*.cu file, the headers every source includes and the flags: it
+    identifies the build of the kernels defined in that file, so a stored profiler record of
+    one kernel stays valid while only other files change."""
+    h = hashlib.sha1()
+    files = [os.path.join(PKG, "csrc", source)] + [
+        os.path.join(PKG, "csrc", x) for x in HEADERS] + [os.path.join(ROOT, "include", "alhr.h")]
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    h.update(" ".join(FLAGS).encode())
+    return h.hexdigest()
+
+
 def is_current() -> bool:
     if not os.path.exists(LIB) or not os.path.exists(STAMP):
         return False
