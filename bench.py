@@ -52,7 +52,12 @@ def parse():
     ap.add_argument("--stages", action="store_true",
                     help="instead of the bench line: per-stage times of the workload through the "
                          "unfused entry points, and fused-forward time against N (1 GPU)")
-    ap.add_argument("--cpu-sample-stride", type=int, default=8,
+    ap.add_argument("--tree", action="store_true",
+                    help="instead of the bench line: time the tree build (alhr_build_tree) on "
+                         "the workload's keys (1 GPU)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="with --tree: replace the workload's batch (sequences)")
+    ap.add_argument("--cpu-sample-stride", type=int, default=4,
                     help="CPU baseline: every k-th query row of every (b,h) block")
     ap.add_argument("--ref-stride", type=int, default=64,
                     help="--impl reference: every k-th query row of each step's block")
@@ -313,7 +318,7 @@ def run_alhr(args, dist, rank, world):
     fwd_launch_s = t_fwd / args.steps
     achieved = fwd_bytes / fwd_launch_s / 1e9
     traffic = profiled_traffic(args.workload)
-    tree_launches = math.ceil(int(math.log2(wl.n)) / 7)
+    tree_launches = tree_build_launches(wl.bh, wl.n)
     line = {
         "metric": METRIC,
         "value": value,
@@ -367,6 +372,17 @@ def run_alhr(args, dist, rank, world):
         "wall_s_timed_region": wall,
     }
     return line
+
+
+def tree_build_launches(bh: int, n: int) -> int:
+    """Kernel launches of one alhr_build_tree: the streaming launch takes levels 1..m1 from
+    the keys (m1 = 5 below 2^24 keys in all, else 7; none below 16 keys), and every further
+    launch up to 7 levels."""
+    L = int(math.log2(n))
+    if L < 4:
+        return 1
+    m1 = min(L, 5 if bh * n < (1 << 24) else 7)
+    return 1 + math.ceil((L - m1) / 7)
 
 
 def _event_time(fn, reps: int, flush) -> float:
@@ -441,6 +457,38 @@ def run_stages(args):
     report["loglog_exponent_fused_forward_vs_n"] = float(np.polyfit(xs, ys, 1)[0])
     report["gpu"] = torch.cuda.get_device_name(dev)
     print(json.dumps(report))
+
+
+def run_tree(args):
+    """The tree build on the workload's keys: one JSON line with its time, its algorithmic bytes
+    (keys read + tree block written) and their rate against the measured copy bandwidth."""
+    from tree_routed_sparse_b200 import alhr, metrics, synth
+    dev = torch.device("cuda", 0)
+    wl = synth.WORKLOADS[args.workload]
+    if args.batch:
+        wl = wl.replace(batch=args.batch)
+    vb = max(-wl.qk_lo, wl.qk_hi)
+    K = synth.uniform_int8(wl.seed, synth.TID_K, (wl.batch, wl.heads, wl.n, wl.d), wl.qk_lo,
+                           wl.qk_hi, dev)
+    tree = torch.empty((wl.batch, wl.heads, alhr.tree_bytes(wl.n, wl.d, vb)), dtype=torch.uint8,
+                       device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    run = lambda: alhr.build_tree(K, tree, value_bound=vb)
+    for _ in range(args.warmup):
+        run()
+    t = _event_time(run, max(args.steps, 3), flush)
+    nbytes = metrics.tree_bytes(wl.bh, wl.n, wl.d, vb)  # keys read + tree rows written
+    peak = 6650.0
+    try:
+        with open(os.path.join(HERE, "MEASURED_PEAKS.json")) as f:
+            peak = float(json.load(f)["hbm_gbs"])
+    except (OSError, KeyError, ValueError):
+        pass
+    print(json.dumps({"report": "tree_build", "workload": describe(wl), "ms": t * 1e3,
+                      "algorithmic_bytes": nbytes, "GBps": nbytes / t / 1e9,
+                      "frac_of_copy_peak": nbytes / t / 1e9 / peak, "peak_GBps": peak,
+                      "launches": tree_build_launches(wl.bh, wl.n),
+                      "gpu": torch.cuda.get_device_name(dev)}))
 
 
 def run_labels(args):
@@ -526,6 +574,13 @@ def main():
         from tree_routed_sparse_b200 import build
         build.build()
         run_labels(args)
+        return
+    if args.tree:
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA device")
+        from tree_routed_sparse_b200 import build
+        build.build()
+        run_tree(args)
         return
     if args.stages:
         if not torch.cuda.is_available():

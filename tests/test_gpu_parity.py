@@ -65,7 +65,9 @@ def _run_forward(A, wl, inp, **kw):
 
 
 @pytest.mark.parametrize("B,H,n,d", [(1, 1, 2, 64), (1, 1, 8, 128), (2, 3, 128, 64),
-                                     (1, 2, 1024, 128), (2, 1, 4096, 64), (1, 1, 1 << 16, 64)])
+                                     (1, 2, 1024, 128), (2, 1, 4096, 64), (1, 1, 1 << 16, 64),
+                                     (1, 3, 16, 64), (3, 1, 32, 128), (1, 1, 256, 64),
+                                     (1, 5, 512, 128), (1, 3, 2048, 64)])
 def test_tree_bit_exact(alhr, synth, B, H, n, d):
     """Both the library's unpack and an independent host reading of the documented layout
     give the oracle's sums."""

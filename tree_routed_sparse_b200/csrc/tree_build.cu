@@ -21,7 +21,14 @@ namespace alhr {
 namespace {
 
 constexpr int kTreeThreads = 256;
-constexpr int kChunkLog = 7;  // 128 input rows per CTA
+constexpr int kChunkLog = 7;   // 128 input rows per CTA
+constexpr int kStreamP = 4;    // keys per batch of the streaming kernel: 2^kStreamP
+// Levels from the keys per row group of the streaming kernel: 7 for large builds; 5 when the
+// build is small (under 2^24 keys in all), where a shorter chain of batches per row group and
+// more row groups in flight matter more than the one extra launch for the levels above.
+constexpr int kStreamLog = 7;
+constexpr int kStreamLogSmall = 5;
+constexpr long long kStreamSmallKeys = 1LL << 24;
 
 enum InKind : int { kFromKeys = 0, kFromNarrow = 1, kFromWide = 2 };
 
@@ -112,6 +119,95 @@ __global__ void __launch_bounds__(kTreeThreads)
     }
     __syncthreads();
   }
+}
+
+// Levels 1 .. m straight from the keys, streamed: a row group of D/4 lanes owns one chunk of
+// 2^m consecutive keys of one (b,h), lane c holding columns [4c, 4c+4) of every key (one 4-byte
+// load per key). The chunk is read in batches of 2^P keys, all loads of a batch issued before
+// any sum; levels 1 .. P above a batch are summed in registers, and levels P+1 .. m are carried
+// from batch to batch in a per-lane stack that works like a binary counter on the batch index.
+// Every node is written once, as soon as the last key beneath it has been read, and no shared
+// memory or barrier is involved, so many batches of many warps are in flight at once.
+template <int D, int P>
+__global__ void __launch_bounds__(kTreeThreads)
+    tree_stream_kernel(const int8_t* __restrict__ K, char* __restrict__ tree, const TreeLayout tl,
+                       int m, int chunk0, int chunks_per_head, long long units, int value_bound,
+                       uint32_t* dev_err) {
+  constexpr int G = D / 4;          // lanes per row group
+  constexpr int R = 1 << P;         // keys per batch
+  constexpr int kMaxUp = kStreamLog - P;  // levels carried across batches (m <= kStreamLog)
+  const long long gt = blockIdx.x * (long long)kTreeThreads + threadIdx.x;
+  const long long unit = gt / G;
+  if (unit >= units) return;        // no warp-wide operation below: a partial warp may leave
+  const int c = int(gt - unit * G);
+  const long long bh = unit / chunks_per_head;
+  const int chunk = chunk0 + int(unit - bh * chunks_per_head);
+  const int n = tl.n;
+  char* Th = tree + bh * tl.block_bytes;
+  const int* src = reinterpret_cast<const int*>(K + (bh * n + ((long long)chunk << m)) * D) + c;
+  const int narrow = tl.narrow;
+
+  auto emit = [&](int l, long long j, const int4& v) {
+    char* row = Th + tl.level_off[l] + j * (long long)(l <= narrow ? 2 * D : 4 * D);
+    if (l <= narrow) {
+      // exact: |sum| <= value_bound * 2^l <= 32767 on a narrow level
+      *(reinterpret_cast<uint2*>(row) + c) =
+          make_uint2(__byte_perm(v.x, v.y, 0x5410), __byte_perm(v.z, v.w, 0x5410));
+    } else {
+      *(reinterpret_cast<int4*>(row) + c) = v;
+    }
+  };
+  auto sum4 = [](const int4& a, const int4& b) {
+    return make_int4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+  };
+
+  int4 stack[kMaxUp > 0 ? kMaxUp : 1];
+  bool bad = false;
+  const int batches = 1 << (m - P);
+  const long long key0 = (long long)chunk << m;  // first key of the chunk
+  for (int bi = 0; bi < batches; ++bi) {
+    int w[R];
+#pragma unroll
+    for (int t = 0; t < R; ++t) w[t] = __ldg(src + (bi * R + t) * (D / 4));
+    int4 lv[R / 2];
+#pragma unroll
+    for (int t = 0; t < R / 2; ++t) {
+      const int a = w[2 * t], b = w[2 * t + 1];
+      const int4 x = make_int4((a << 24) >> 24, (a << 16) >> 24, (a << 8) >> 24, a >> 24);
+      const int4 y = make_int4((b << 24) >> 24, (b << 16) >> 24, (b << 8) >> 24, b >> 24);
+      bad |= x.x > value_bound | x.x < -value_bound | x.y > value_bound | x.y < -value_bound |
+             x.z > value_bound | x.z < -value_bound | x.w > value_bound | x.w < -value_bound |
+             y.x > value_bound | y.x < -value_bound | y.y > value_bound | y.y < -value_bound |
+             y.z > value_bound | y.z < -value_bound | y.w > value_bound | y.w < -value_bound;
+      lv[t] = sum4(x, y);
+    }
+    const long long b0 = key0 + (long long)bi * R;  // first key of the batch
+#pragma unroll
+    for (int l = 1; l <= P; ++l) {
+      const int cnt = R >> l;
+#pragma unroll
+      for (int t = 0; t < cnt; ++t) {
+        if (l > 1) lv[t] = sum4(lv[2 * t], lv[2 * t + 1]);
+        emit(l, (b0 >> l) + t, lv[t]);
+      }
+    }
+    // levels above the batch: carry like a binary counter on bi
+    int4 v = lv[0];
+    bool carry = true;
+#pragma unroll
+    for (int s = 1; s <= kMaxUp; ++s) {
+      if (s <= m - P && carry) {
+        if (((bi >> (s - 1)) & 1) == 0) {
+          stack[s - 1] = v;
+          carry = false;
+        } else {
+          v = sum4(stack[s - 1], v);
+          emit(P + s, b0 >> (P + s), v);
+        }
+      }
+    }
+  }
+  if (bad && dev_err) atomicOr(dev_err, ALHR_DEVERR_VALUE_RANGE);
 }
 
 // The tree as plain int32 rows: one thread per 4 values of an output row.
@@ -280,15 +376,25 @@ cudaError_t build_tree_d(const int8_t* K, char* tree, const TreeLayout& tl, long
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 128) configured[dev] = true;
   }
+  const int stream_log =
+      bh * (long long)(hi - lo) < kStreamSmallKeys ? kStreamLogSmall : kStreamLog;
   int lin = 0;
   while (lin < L) {
-    const int m = (L - lin) < kChunkLog ? (L - lin) : kChunkLog;
+    const bool stream = lin == 0 && L >= kStreamP;
+    const int mmax = stream ? stream_log : kChunkLog;
+    const int m = (L - lin) < mmax ? (L - lin) : mmax;
     const int c0 = (lo >> lin) >> m, c1 = ((hi - 1) >> lin) >> m;
     const int chunks = c1 - c0 + 1;
     const long long grid = bh * chunks;
     const size_t smem = size_t(1 << m) * D * sizeof(int);
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    if (lin == 0) {
+    if (stream) {
+      const long long threads = grid * (D / 4);
+      const long long blocks = (threads + kTreeThreads - 1) / kTreeThreads;
+      if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+      tree_stream_kernel<D, kStreamP><<<unsigned(blocks), kTreeThreads, 0, st>>>(
+          K, tree, tl, m, c0, chunks, grid, value_bound, dev_err);
+    } else if (lin == 0) {
       tree_chunk_kernel<D, kFromKeys><<<unsigned(grid), kTreeThreads, smem, st>>>(
           K, tree, tl, lin, m, c0, chunks, value_bound, dev_err);
     } else if (lin <= tl.narrow) {
