@@ -124,8 +124,9 @@ __global__ void __launch_bounds__(kTreeThreads)
 // Levels 1 .. m straight from the keys, streamed: a row group of D/4 lanes owns one chunk of
 // 2^m consecutive keys of one (b,h), lane c holding columns [4c, 4c+4) of every key (one 4-byte
 // load per key). The chunk is read in batches of 2^P keys, all loads of a batch issued before
-// any sum; levels 1 .. P above a batch are summed in registers, and levels P+1 .. m are carried
-// from batch to batch in a per-lane stack that works like a binary counter on the batch index.
+// any sum and one batch ahead; levels 1 .. P above a batch are summed in registers, and levels
+// P+1 .. m are carried from batch to batch in a per-lane stack that works like a binary counter
+// on the batch index.
 // Every node is written once, as soon as the last key beneath it has been read, and no shared
 // memory or barrier is involved, so many batches of many warps are in flight at once.
 template <int D, int P>
@@ -165,10 +166,19 @@ __global__ void __launch_bounds__(kTreeThreads)
   bool bad = false;
   const int batches = 1 << (m - P);
   const long long key0 = (long long)chunk << m;  // first key of the chunk
+  // the next batch's loads are issued before the current batch is summed (two batches in
+  // flight per row group)
+  int wn[R];
+#pragma unroll
+  for (int t = 0; t < R; ++t) wn[t] = __ldg(src + t * (D / 4));
   for (int bi = 0; bi < batches; ++bi) {
     int w[R];
 #pragma unroll
-    for (int t = 0; t < R; ++t) w[t] = __ldg(src + (bi * R + t) * (D / 4));
+    for (int t = 0; t < R; ++t) w[t] = wn[t];
+    if (bi + 1 < batches) {
+#pragma unroll
+      for (int t = 0; t < R; ++t) wn[t] = __ldg(src + ((bi + 1) * R + t) * (D / 4));
+    }
     int4 lv[R / 2];
 #pragma unroll
     for (int t = 0; t < R / 2; ++t) {
