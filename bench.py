@@ -317,7 +317,8 @@ def run_alhr(args, dist, rank, world):
     peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
     fwd_launch_s = t_fwd / args.steps
     achieved = fwd_bytes / fwd_launch_s / 1e9
-    traffic = profiled_traffic(args.workload)
+    rec = profiled_record(args.workload)
+    traffic = rec.get("dram_bytes_per_launch") if rec else None
     tree_launches = tree_build_launches(wl.bh, wl.n)
     line = {
         "metric": METRIC,
@@ -353,10 +354,13 @@ def run_alhr(args, dist, rank, world):
             "algorithmic_bytes_per_launch": fwd_bytes,
             "launch_ms": fwd_launch_s * 1e3,
             "traffic": traffic,
-            "note": ("algorithmic bytes count every row the path reads as if from DRAM; the "
-                     "working set of one step (tree, keys, values) is smaller than L2, so "
-                     "repeat reads of upper tree levels are served by L2 and achieved can "
-                     "exceed the DRAM peak; traffic is the DRAM bytes ncu measured"),
+            "issue": issue_rate(rec, fwd_launch_s),
+            "note": ("algorithmic bytes count every row the path reads as if from DRAM; "
+                     "queries run in (b, h, i) order, so the rows in use at any time (about "
+                     "one head's tree, keys and values) stay in L2, repeat reads are served "
+                     "there and achieved can exceed the DRAM peak; traffic is the DRAM bytes "
+                     "ncu measured (compulsory reads and the output); issue is the binding "
+                     "resource, the kernel's warp instructions against the GPU's issue slots"),
         },
         "stages_ms": {"tree_build": t_tree / args.steps * 1e3,
                       "forward": t_fwd / args.steps * 1e3,
@@ -372,6 +376,15 @@ def run_alhr(args, dist, rank, world):
         "wall_s_timed_region": wall,
     }
     return line
+
+
+def measured_hbm_peak() -> float:
+    """hbm_gbs of MEASURED_PEAKS.json (the measured copy bandwidth), else the fallback 6650."""
+    try:
+        with open(os.path.join(HERE, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"])
+    except (OSError, KeyError, ValueError):
+        return 6650.0
 
 
 def tree_build_launches(bh: int, n: int) -> int:
@@ -404,10 +417,11 @@ def run_stages(args):
     """Per-stage split of one step (tree build, predictor, route, unfused attend, and the fused
     forward that does the last three in one kernel), then the fused forward against N at fixed
     batch and heads (prefill of every position), with the fitted log-log exponent of its time."""
-    from tree_routed_sparse_b200 import alhr, synth
+    from tree_routed_sparse_b200 import alhr, metrics, synth
     dev = torch.device("cuda", 0)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     reps = max(args.steps, 5)
+    peak = measured_hbm_peak()
 
     def stages(wl):
         vb = max(-wl.qk_lo, wl.qk_hi)
@@ -433,25 +447,35 @@ def run_stages(args):
                                   reps, flush)
         t["fused_forward"] = _event_time(
             lambda: alhr.forward(Q, K, V, tree, W=W, budget_override=bo, out=out, **kw), reps, flush)
+        full = alhr.forward(Q, K, V, tree, W=W, budget_override=bo, want_count=True,
+                            want_expansions=True, want_budget=True, **kw)
+        pos = np.broadcast_to(np.arange(wl.q_start, wl.q_start + wl.nq), (wl.bh, wl.nq))
+        fb = metrics.forward_bytes(pos, wl.n, wl.d, wl.window, full["count"].cpu().numpy(),
+                                   full["expansions"].cpu().numpy(), full["budget"].cpu().numpy(),
+                                   wl.predictor, wl.max_keys, value_bound=vb)
         keys = float(count.float().mean())
-        del inp, tree, out, idx, count, budget
+        del inp, tree, out, idx, count, budget, full
         torch.cuda.empty_cache()
-        return t, keys
+        return t, keys, fb
 
     base = synth.WORKLOADS[args.workload]
-    t, keys = stages(base)
+    t, keys, fb = stages(base)
     report = {"report": "stages", "workload": describe(base), "reps": reps,
               "stage_ms": {k: v * 1e3 for k, v in t.items()}, "mean_keys_per_query": keys,
+              "fused_forward_algorithmic_bytes": fb,
+              "fused_forward_GBps": fb / t["fused_forward"] / 1e9, "peak_GBps": peak,
               "scaling": []}
     sweep = [1024, 4096, 16384, 65536]
     for n in sweep:
         wl = base.replace(n=n, nq=n, q_start=0)
-        t, keys = stages(wl)
+        t, keys, fb = stages(wl)
         q = wl.bh * wl.nq
         report["scaling"].append({"n": n, "queries": q, "fused_forward_ms": t["fused_forward"] * 1e3,
                                   "tree_build_ms": t["tree_build"] * 1e3,
                                   "ns_per_query": t["fused_forward"] / q * 1e9,
-                                  "mean_keys_per_query": keys})
+                                  "mean_keys_per_query": keys,
+                                  "fused_forward_GBps": fb / t["fused_forward"] / 1e9,
+                                  "frac_of_copy_peak": fb / t["fused_forward"] / 1e9 / peak})
     xs = np.log([e["n"] for e in report["scaling"]])
     ys = np.log([e["fused_forward_ms"] for e in report["scaling"]])
     report["loglog_exponent_fused_forward_vs_n"] = float(np.polyfit(xs, ys, 1)[0])
@@ -478,12 +502,7 @@ def run_tree(args):
         run()
     t = _event_time(run, max(args.steps, 3), flush)
     nbytes = metrics.tree_bytes(wl.bh, wl.n, wl.d, vb)  # keys read + tree rows written
-    peak = 6650.0
-    try:
-        with open(os.path.join(HERE, "MEASURED_PEAKS.json")) as f:
-            peak = float(json.load(f)["hbm_gbs"])
-    except (OSError, KeyError, ValueError):
-        pass
+    peak = measured_hbm_peak()
     print(json.dumps({"report": "tree_build", "workload": describe(wl), "ms": t * 1e3,
                       "algorithmic_bytes": nbytes, "GBps": nbytes / t / 1e9,
                       "frac_of_copy_peak": nbytes / t / 1e9 / peak, "peak_GBps": peak,
@@ -520,10 +539,10 @@ def run_labels(args):
                       "gpu": torch.cuda.get_device_name(dev)}))
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per launch of the fused kernel from the committed ncu summary, if that
-    summary was taken on the fused kernel's source (query_kernels.cu and the headers) as it is
-    now; else None."""
+def profiled_record(workload: str):
+    """The committed ncu record of the fused kernel on this workload (DRAM bytes and warp
+    instructions per launch), if it was taken on the fused kernel's source (query_kernels.cu and
+    the headers) as it is now; else None."""
     path = os.path.join(HERE, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -535,7 +554,24 @@ def profiled_traffic(workload: str):
     from tree_routed_sparse_b200 import build
     if rec.get("source_hash") != build.kernel_hash("query_kernels.cu"):
         return None
-    return rec.get("dram_bytes_per_launch")
+    return rec
+
+
+# warp-instruction issue slots per second of one B200: 148 SMs x 4 schedulers x max SM clock
+ISSUE_SLOTS_PER_S = 148 * 4 * 1965e6
+
+
+def issue_rate(rec, launch_s: float):
+    """The fused kernel's instruction issue against the GPU's issue slots: its warp
+    instructions per launch (from the ncu record) over the live launch time, as a fraction of
+    148 SMs x 4 schedulers x 1965 MHz. None without a current record."""
+    if not rec or "warp_instructions_per_launch" not in rec:
+        return None
+    achieved = rec["warp_instructions_per_launch"] / launch_s
+    return {"warp_instructions_per_launch": rec["warp_instructions_per_launch"],
+            "achieved_per_s": achieved, "peak_per_s": ISSUE_SLOTS_PER_S,
+            "frac": achieved / ISSUE_SLOTS_PER_S,
+            "source": "instruction count from profiles/traffic.json (ncu), live launch time"}
 
 
 def main():

@@ -48,6 +48,7 @@ def _slice_inputs(inp, wl, b, h):
     ("tiny_prefill_n1024", [(0, 0)]),
     ("prefill_b4h8_n4096", [(0, 0), (3, 7)]),
     ("prefill_b2h8_n16384", [(0, 3), (1, 7)]),
+    ("prefill_b2h8_n65536", [(0, 5), (1, 2)]),
     ("recall_b2h4_n16384_d128", [(0, 0), (1, 3)]),
     ("decode_s64h8_n262144_d128", [(0, 0), (5, 1), (17, 2), (31, 3), (40, 4), (50, 5),
                                    (62, 6), (63, 7)]),

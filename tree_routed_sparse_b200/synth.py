@@ -152,6 +152,9 @@ WORKLOADS = {
     # T=16K, same distributions and predictor, exact int32 scores
     "prefill_b2h8_n16384": Workload("prefill_b2h8_n16384", 2, 8, 16384, 64, 0, 16384,
                                     score_bits=32),
+    # T=64K, same distributions: the working set (tree 268 MB, keys, values) exceeds L2
+    "prefill_b2h8_n65536": Workload("prefill_b2h8_n65536", 2, 8, 65536, 64, 0, 65536,
+                                    score_bits=32),
     # T=16K associative-recall shape: 256 planted pairs per sequence, int64 scores
     "recall_b2h4_n16384_d128": Workload("recall_b2h4_n16384_d128", 2, 4, 16384, 128, 0,
                                         16384, score_bits=64, plant_pairs=256),
