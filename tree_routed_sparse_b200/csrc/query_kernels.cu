@@ -167,7 +167,9 @@ __device__ __forceinline__ void narrow_child_pass(WarpBuf<S>& B, const char* Th,
 #pragma unroll
   for (int u = 0; u < US; ++u) {
     const int xi = base + u * RPI + grp;
-    const S left = group_sum<S, TPR>(S(dot_tree16(q, w[u])));
+    // the whole row's score fits in int32 (|q| <= 127, |x| <= 32767, d = 128), so the group
+    // sum runs in int32 and is widened once
+    const S left = S(group_sum<int, TPR>(dot_tree16(q, w[u])));
     if (xi < end && sub == 0) B.xleft[xi] = left;
   }
 }
