@@ -366,11 +366,69 @@ __device__ __noinline__ int tie_cut(TieStarts<NS> ts, int need) {
   }
   return lo2;
 }
-//
+// The threshold of the top r among the lane's NS candidate scores (kLow marks an empty slot):
+// the r-th largest score thr, and the cut on start positions among the candidates tied at thr
+// (candidates with score thr and start <= cut are kept; cut = INT_MAX when no tie straddles).
+// Exact: thr is found by bisection on the integer score; candidates tied at thr are then cut by
+// bisection on their start position (starts are distinct).
+template <typename T, int NS>
+__device__ __forceinline__ void top_r_threshold(const T (&sc)[NS], const int (&ds)[NS], int r,
+                                                T& thr, int& cut) {
+  constexpr T kLow = ScoreLimits<T>::lowest;
+  T mn = ScoreLimits<T>::highest, mx = kLow;
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    if (sc[s] != kLow) {
+      mn = sc[s] < mn ? sc[s] : mn;
+      mx = sc[s] > mx ? sc[s] : mx;
+    }
+  }
+  T lo = warp_min<T>(mn);
+  T hi = warp_max<T>(mx);
+  // Bisection for the largest T with #{score >= T} >= r. It stops as soon as a midpoint has
+  // exactly r candidates at or above it: that set is the top r (nothing at or above the
+  // midpoint is left out, so no tie can straddle the cut), which takes about log2(C) probes
+  // instead of log2(score range).
+  bool exact = false;
+  for (int guard = 0; guard < 70 && lo < hi; ++guard) {
+    const T mid = T((long long)lo + (((long long)hi - (long long)lo + 1) >> 1));
+    int c = 0;
+#pragma unroll
+    for (int s = 0; s < NS; ++s) c += sc[s] >= mid ? 1 : 0;
+    c = __reduce_add_sync(kFull, c);
+    if (c == r) {
+      lo = mid;
+      exact = true;
+      break;
+    }
+    if (c > r) lo = mid; else hi = mid - 1;
+  }
+  thr = lo;
+  int need = 0, eq = 0;
+  if (!exact) {
+    int gt = 0;
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      gt += sc[s] > lo ? 1 : 0;
+      eq += sc[s] == lo ? 1 : 0;
+    }
+    gt = __reduce_add_sync(kFull, gt);
+    eq = __reduce_add_sync(kFull, eq);
+    need = r - gt;
+  }
+  cut = 0x7fffffff;
+  if (!exact && need < eq) {
+    TieStarts<NS> ts;
+#pragma unroll
+    for (int s = 0; s < NS; ++s) ts.v[s] = sc[s] == lo ? desc_start(ds[s]) : 0x7fffffff;
+    cut = tie_cut<NS>(ts, need);
+  }
+}
+
 // Keeps, among the C candidates (r < C <= 32*NS), the r with the largest score, ties to the
-// lower start, and packs them into the front of the buffer. Exact: the r-th largest score T is
-// found by bisection on the integer score; candidates tied at T are then cut by bisection on
-// their start position (starts are distinct).
+// lower start, and packs them into the front of the buffer. With 64-bit scores the threshold
+// search runs on 32-bit copies whenever every candidate's score fits in 32 bits (one vote per
+// call; the same set either way).
 template <typename S, int NS, bool NORM>
 __device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int lane,
                                                 int norm_l) {
@@ -386,61 +444,40 @@ __device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int
     // ranking by means: q . sum / 2^level, scaled by 2^L to stay an exact integer
     if (NORM && norm_l && ok) sc[s] = sc[s] * (S(1) << (norm_l - desc_level(ds[s])));
   }
-  S mn = ScoreLimits<S>::highest, mx = kLow;
+  bool keep[NS];
+  bool narrow = false;
+  if constexpr (sizeof(S) == 8) {
+    bool fits = true;
 #pragma unroll
-  for (int s = 0; s < NS; ++s) {
-    if (sc[s] != kLow) {
-      mn = sc[s] < mn ? sc[s] : mn;
-      mx = sc[s] > mx ? sc[s] : mx;
-    }
+    for (int s = 0; s < NS; ++s)
+      fits &= sc[s] == kLow || (sc[s] > S(ScoreLimits<int>::lowest) &&
+                                sc[s] <= S(ScoreLimits<int>::highest));
+    narrow = __all_sync(kFull, fits);
   }
-  S lo = warp_min<S>(mn);
-  S hi = warp_max<S>(mx);
-  // Bisection for the largest T with #{score >= T} >= r. It stops as soon as a midpoint has
-  // exactly r candidates at or above it: that set is the top r (nothing at or above the
-  // midpoint is left out, so no tie can straddle the cut), which takes about log2(C) probes
-  // instead of log2(score range).
-  bool exact = false;
-  for (int guard = 0; guard < 70 && lo < hi; ++guard) {
-    const S mid = S((long long)lo + (((long long)hi - (long long)lo + 1) >> 1));
-    int c = 0;
+  if (narrow) {
+    int s32[NS];
 #pragma unroll
-    for (int s = 0; s < NS; ++s) c += sc[s] >= mid ? 1 : 0;
-    c = __reduce_add_sync(kFull, c);
-    if (c == r) {
-      lo = mid;
-      exact = true;
-      break;
-    }
-    if (c > r) lo = mid; else hi = mid - 1;
-  }
-  const S T = lo;
-  int need = 0, eq = 0;
-  if (!exact) {
-    int gt = 0;
+    for (int s = 0; s < NS; ++s) s32[s] = sc[s] == kLow ? ScoreLimits<int>::lowest : int(sc[s]);
+    int thr, cut;
+    top_r_threshold<int, NS>(s32, ds, r, thr, cut);
 #pragma unroll
-    for (int s = 0; s < NS; ++s) {
-      gt += sc[s] > T ? 1 : 0;
-      eq += sc[s] == T ? 1 : 0;
-    }
-    gt = __reduce_add_sync(kFull, gt);
-    eq = __reduce_add_sync(kFull, eq);
-    need = r - gt;
-  }
-  int U = 0x7fffffff;
-  if (!exact && need < eq) {
-    TieStarts<NS> ts;
+    for (int s = 0; s < NS; ++s)
+      keep[s] = s32[s] != ScoreLimits<int>::lowest &&
+                (s32[s] > thr || (s32[s] == thr && desc_start(ds[s]) <= cut));
+  } else {
+    S thr;
+    int cut;
+    top_r_threshold<S, NS>(sc, ds, r, thr, cut);
 #pragma unroll
-    for (int s = 0; s < NS; ++s) ts.v[s] = sc[s] == T ? desc_start(ds[s]) : 0x7fffffff;
-    U = tie_cut<NS>(ts, need);
+    for (int s = 0; s < NS; ++s)
+      keep[s] = sc[s] != kLow && (sc[s] > thr || (sc[s] == thr && desc_start(ds[s]) <= cut));
   }
   __syncwarp();
   int base = 0;
 #pragma unroll
   for (int s = 0; s < NS; ++s) {
-    const bool keep = sc[s] != kLow && (sc[s] > T || (sc[s] == T && desc_start(ds[s]) <= U));
-    const unsigned bal = __ballot_sync(kFull, keep);
-    if (keep) {
+    const unsigned bal = __ballot_sync(kFull, keep[s]);
+    if (keep[s]) {
       const int pos = base + __popc(bal & lanemask_lt(lane));
       B.cdesc[pos] = ds[s];
       B.cscore[pos] = (NORM && norm_l) ? S(sc[s] >> (norm_l - desc_level(ds[s]))) : sc[s];
