@@ -86,7 +86,7 @@ typedef enum {
 
 /* Problem sizes, shared by every entry point. */
 typedef struct {
-  int32_t batch;       /* >= 1                                                            */
+  int32_t batch;       /* >= 1; batch * heads < 2^31 (else ALHR_ERR_UNSUPPORTED)          */
   int32_t heads;       /* >= 1                                                            */
   int32_t n;           /* keys per (b,h): a power of two, 2 <= n <= 2^20                  */
   int32_t d;           /* head dimension: 64 or 128                                       */

@@ -124,6 +124,8 @@ def test_score_width_choice(A):
     assert sb(score_bits=64) == 64
     assert sb(d=96) == -2 and sb(n=1000) == -1 and sb(window=33) == -2 and sb(max_keys=97) == -2
     assert sb(max_keys=0) == -1 and sb(q_start=1) == -1 and sb(score_bits=16) == -1
+    assert sb(batch=65536, heads=32768) == -2         # batch * heads must stay below 2^31
+    assert sb(batch=65535, heads=32768) == 32
     # ranked by means, a key's ranking value is q . k * n: the bound doubles
     assert sb(n=65536, d=128) == 32                    # 128 * 256 * 2^15 = 2^30
     assert sb(n=65536, d=128, score_norm=1) == 64      # 128 * 256 * 2^16 = 2^31

@@ -28,6 +28,7 @@ int value_bound_of(const alhr_dims* d) { return d->value_bound == 0 ? 16 : d->va
 alhr_status check_common(const alhr_dims* d) {
   if (!d) return ALHR_ERR_INVALID_ARG;
   if (d->batch < 1 || d->heads < 1) return ALHR_ERR_INVALID_ARG;
+  if (int64_t(d->batch) * d->heads > int64_t(INT32_MAX)) return ALHR_ERR_UNSUPPORTED;
   if (!pow2_in_range(d->n)) return ALHR_ERR_INVALID_ARG;
   if (d->d != 64 && d->d != 128) return ALHR_ERR_UNSUPPORTED;
   if (d->value_bound < 0 || d->value_bound > 127) return ALHR_ERR_INVALID_ARG;

@@ -69,6 +69,29 @@ struct QueryArgs {
 
 __device__ __forceinline__ int sx8(int w, int byte) { return (w << (24 - 8 * byte)) >> 24; }
 
+// A warp's walk over the flat query index qi = bh * nq + r in steps of `stride`, keeping
+// (bh, r) up to date with one division at the start instead of one per query.
+struct QueryCursor {
+  long long qi, bh, step_bh;
+  int r, step_r;
+  __device__ __forceinline__ QueryCursor(long long first, int nq, long long stride) {
+    qi = first;
+    bh = first / nq;
+    r = int(first - bh * nq);
+    step_bh = stride / nq;
+    step_r = int(stride - step_bh * nq);
+  }
+  __device__ __forceinline__ void advance(long long stride, int nq) {
+    qi += stride;
+    bh += step_bh;
+    r += step_r;  // r, step_r < nq, so one carry at most
+    if (r >= nq) {
+      r -= nq;
+      ++bh;
+    }
+  }
+};
+
 // Byte offset of row j of tree level l (>= 1) inside a block of the layout of tree_layout.h,
 // from scalars only (levels 1 .. l-1 hold n - (n >> (l-1)) rows, the first n - (n >> narrow) of
 // them int16 rows of 2d bytes, the rest int32 rows of 4d bytes).
@@ -366,6 +389,18 @@ __device__ __noinline__ int tie_cut(TieStarts<NS> ts, int need) {
   }
   return lo2;
 }
+// Upper midpoint of [lo, hi] (lo < hi), exact.
+template <typename T>
+__device__ __forceinline__ T upper_mid(T lo, T hi) {
+  return T((long long)lo + (((long long)hi - (long long)lo + 1) >> 1));
+}
+// 32-bit scores: valid scores are above INT_MIN (the empty-slot mark), so hi - lo + 1 < 2^32
+// and the unsigned difference is exact.
+template <>
+__device__ __forceinline__ int upper_mid<int>(int lo, int hi) {
+  return lo + int((unsigned(hi) - unsigned(lo) + 1u) >> 1);
+}
+
 // The threshold of the top r among the lane's NS candidate scores (kLow marks an empty slot):
 // the r-th largest score thr, and the cut on start positions among the candidates tied at thr
 // (candidates with score thr and start <= cut are kept; cut = INT_MAX when no tie straddles).
@@ -391,7 +426,7 @@ __device__ __forceinline__ void top_r_threshold(const T (&sc)[NS], const int (&d
   // instead of log2(score range).
   bool exact = false;
   for (int guard = 0; guard < 70 && lo < hi; ++guard) {
-    const T mid = T((long long)lo + (((long long)hi - (long long)lo + 1) >> 1));
+    const T mid = upper_mid<T>(lo, hi);
     int c = 0;
 #pragma unroll
     for (int s = 0; s < NS; ++s) c += sc[s] >= mid ? 1 : 0;

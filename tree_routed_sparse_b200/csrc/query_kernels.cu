@@ -266,9 +266,13 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
   const int norm_l = VAR ? a.norm_l : 0;          // ranking by means (0: by sums)
   const long long stride = (long long)gridDim.x * NW;
 
-  for (long long qi = (long long)blockIdx.x * NW + warp; qi < a.num_queries; qi += stride) {
-    const long long bh = qi / a.nq;
-    const int i = a.q_start + int(qi - bh * a.nq);
+  for (QueryCursor cur((long long)blockIdx.x * NW + warp, a.nq, stride); cur.qi < a.num_queries;
+       cur.advance(stride, a.nq)) {
+    const long long qi = cur.qi;
+    // (bh, position) from the cursor in the int32-score kernels; the int64-score kernels, at a
+    // tighter register budget, measured faster dividing once per query
+    const long long bh = sizeof(S) == 4 ? cur.bh : qi / a.nq;
+    const int i = a.q_start + (sizeof(S) == 4 ? cur.r : int(qi - bh * a.nq));
     const int8_t* Kh = a.K + bh * (long long)n * D;
     const char* Th = a.tree + bh * tree_block;
 
@@ -717,9 +721,11 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(const QueryArgs a) 
   WarpBuf<int>& B = wbuf[warp];
   const int n = a.n;
   const long long stride = (long long)gridDim.x * kWarps;
-  for (long long qi = (long long)blockIdx.x * kWarps + warp; qi < a.num_queries; qi += stride) {
-    const long long bh = qi / a.nq;
-    const int i = a.q_start + int(qi - bh * a.nq);
+  for (QueryCursor cur((long long)blockIdx.x * kWarps + warp, a.nq, stride);
+       cur.qi < a.num_queries; cur.advance(stride, a.nq)) {
+    const long long qi = cur.qi;
+    const long long bh = cur.bh;
+    const int i = a.q_start + cur.r;
     const int8_t* Kh = a.K + bh * (long long)n * D;
     const uint16_t* Vh = a.V + bh * (long long)n * D;
     RowQ q;
