@@ -74,6 +74,35 @@ def test_update_large_ranges_equal_full_build(alhr, synth, n, d, vb):
         _check_update(alhr, synth, 2, 2, n, d, vb, lo, hi, seed=31 * n + d + k)
 
 
+def test_update_large_build_plan(alhr, synth):
+    """A range rebuild large enough (batch * heads * keys >= 2^24) for the build's large-size
+    launch plan (7 levels per streaming row group), with chunks starting mid-sequence: equal to a
+    full build, and to the oracle on two blocks (copied to the host block by block)."""
+    B, H, n, d, vb = 64, 8, 65536, 64, 16
+    lo, hi = 1000, 41000  # 512 blocks x 40,000 keys; first rebuilt chunk starts at key 896
+    need = 2 * B * H * n * d + 2 * B * H * alhr.tree_bytes(n, d, vb)
+    free, _ = torch.cuda.mem_get_info()
+    if need > free - (2 << 30):
+        pytest.skip(f"needs {need / 2**30:.1f} GiB")
+    K_old = synth.uniform_int8(3, synth.TID_K, (B, H, n, d), -vb, vb, "cuda")
+    tree = alhr.build_tree(K_old, value_bound=vb)
+    K = K_old.clone()
+    del K_old
+    K[:, :, lo:hi] = synth.uniform_int8(3, TID_NEW, (B, H, hi - lo, d), -vb, vb, "cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    alhr.update_tree(K, tree, lo, hi, value_bound=vb, dev_err=err)
+    full = alhr.build_tree(K, value_bound=vb)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(tree, full)
+    del full
+    for b, h in [(0, 0), (B - 1, H - 1)]:
+        got = decode_tree(tree[b, h].cpu().numpy(), n, d, vb)
+        assert np.array_equal(got, orc.build_tree(K[b, h].cpu().numpy())), (b, h)
+    del tree, K
+    torch.cuda.empty_cache()
+
+
 def test_update_empty_range_changes_nothing(alhr, synth):
     K = synth.uniform_int8(5, synth.TID_K, (1, 2, 256, 64), -16, 16, "cuda")
     tree = alhr.build_tree(K)
