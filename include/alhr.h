@@ -149,7 +149,7 @@ ALHR_API const char* alhr_build_info(void);
  *   ALHR_LAUNCH_AUTO (default): latency shape when a launch has at most 8 queries per SM of the
  *     device (decode and other small launches), throughput shape above.
  *   ALHR_LAUNCH_THROUGHPUT: several CTAs per SM, one or two tree rows in flight per lane group.
- *   ALHR_LAUNCH_LATENCY: one CTA per SM, up to eight rows in flight per lane group.
+ *   ALHR_LAUNCH_LATENCY: one CTA per SM, up to twelve rows in flight per lane group.
  * alhr_set_launch_mode returns ALHR_ERR_INVALID_ARG (and changes nothing) for any other value.
  */
 typedef enum {

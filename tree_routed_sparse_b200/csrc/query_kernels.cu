@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
   constexpr int TPR = Lay<D>::TPR;
   constexpr int RPI = Lay<D>::RPI;
   // tree rows per group per pass (at d = 128: int16 rows; int32 rows take UW)
-  constexpr int U = LAT ? (D == 128 ? 8 : 4) : tree_rows_in_flight<S, D>();
+  constexpr int U = LAT ? (D == 128 ? 12 : 4) : tree_rows_in_flight<S, D>();
   constexpr int UK = LAT ? 8 : 1;  // key rows per group per pass
   constexpr int UW = LAT ? 4 : 1;  // d = 128: int32 tree rows per group per pass
   constexpr int UV = LAT ? 8 : 2;  // value-row passes in flight
