@@ -367,7 +367,7 @@ template <int D>
 cudaError_t launch_labels_d(const int8_t* Q, const int8_t* K, int32_t* labels, int32_t* scores,
                             int n, int q_start, int nq, int k, long long bh, uint32_t* dev_err,
                             cudaStream_t st) {
-  static bool configured[128] = {};
+  static thread_local bool configured[128] = {};  // per host thread: no shared state
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 128 || !configured[dev]) {

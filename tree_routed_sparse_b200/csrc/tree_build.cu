@@ -371,7 +371,7 @@ cudaError_t build_tree_d(const int8_t* K, char* tree, const TreeLayout& tl, long
   const int L = tl.L;
   const size_t smem_max = size_t(1 << kChunkLog) * D * sizeof(int);
   // the opt-in above 48 KB of dynamic shared memory is a per-device function attribute
-  static bool configured[128] = {};
+  static thread_local bool configured[128] = {};  // per host thread: no shared state
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 128 || !configured[dev]) {
