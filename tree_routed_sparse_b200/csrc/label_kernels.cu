@@ -273,10 +273,25 @@ __global__ void __launch_bounds__(kLThreads, D == 64 ? 4 : 3)
   int epoch = 0;                   // key base of the queued entries
   for (int t = 0; t < ntiles; ++t) {
     const int b = t & 1;
-    // 1. MMA t done: its accumulator is ready and its key buffer is free
+    // 1. MMA t done (as this thread sees it): its accumulator is ready, its key buffer free
     bool ok = false;
     for (uint32_t w = 0; w < kWaitLimit && !ok; ++w)
       ok = mbar_try_wait(smem_u32(mbar + b), (phases >> b) & 1u);
+    phases ^= 1u << b;
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    // 2. key tile t + 2 into the freed buffer (its own cp.async group)
+    if (ok && t + 2 < ntiles) {
+      const int k2 = (t + 2) * kNT;
+      load_tile<D, kNT>(sK + b * L::k_bytes, Kh, k2, min(kNT, n - k2), tid);
+    }
+    // 3. the tile's one CTA barrier: every thread's copies of key tile t + 1 have landed, every
+    //    thread has read accumulator (t + 1) & 1 (tile t - 1, in the previous iteration), and
+    //    a wait that ran out on any thread stops all of them here together
+    if (t + 1 < ntiles) {
+      if (t + 2 < ntiles) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+      else asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    }
     if (__syncthreads_or(!ok)) {
       if (tid == 0) {
         *abort_flag = 1;
@@ -284,22 +299,7 @@ __global__ void __launch_bounds__(kLThreads, D == 64 ? 4 : 3)
       }
       break;
     }
-    phases ^= 1u << b;
-    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-    // 2. key tile t + 2 into the freed buffer (its own cp.async group)
-    if (t + 2 < ntiles) {
-      const int k2 = (t + 2) * kNT;
-      load_tile<D, kNT>(sK + b * L::k_bytes, Kh, k2, min(kNT, n - k2), tid);
-    }
-    // 3. key tile t + 1 has landed: start its MMA into the other accumulator (read back in the
-    //    previous iteration, before that iteration's closing barrier)
-    if (t + 1 < ntiles) {
-      if (t + 2 < ntiles) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
-      else asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-      __syncthreads();
-      if (tid == 0) issue_mma(t + 1);
-    }
+    if (t + 1 < ntiles && tid == 0) issue_mma(t + 1);
     // 4. this thread's row of scores for tile t, 64 columns as two loads of 32
     uint32_t v0[32], v1[32];
     const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + b * kNT;
@@ -338,9 +338,9 @@ __global__ void __launch_bounds__(kLThreads, D == 64 ? 4 : 3)
     if (__any_sync(0xffffffffu, qp - qbase > (L::kQueue - 32) * kLThreads))
       qp = flush_queue(qbase, qp, epoch, s, ix);
     qp = queue_chunk(v1, lim - 32, s[kListK - 1], k0 + 32 - epoch, qp, rowp);
-    // 5. accumulator t & 1 is read: the MMA of tile t + 2 may overwrite it
+    // 5. accumulator t & 1 is read; the next iteration's barrier orders this before the MMA of
+    //    tile t + 2 overwrites it
     asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-    __syncthreads();
   }
 
   qp = flush_queue(qbase, qp, epoch, s, ix);
