@@ -52,6 +52,10 @@ def parse():
     ap.add_argument("--stages", action="store_true",
                     help="instead of the bench line: per-stage times of the workload through the "
                          "unfused entry points, and fused-forward time against N (1 GPU)")
+    ap.add_argument("--launch-mode", default="auto", choices=["auto", "throughput", "latency"],
+                    help="with --stages: launch shape of the per-query kernels")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="with --stages: only the workload's own stage split (no sweep over N)")
     ap.add_argument("--tree", action="store_true",
                     help="instead of the bench line: time the tree build (alhr_build_tree) on "
                          "the workload's keys (1 GPU)")
@@ -422,6 +426,7 @@ def run_stages(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     reps = max(args.steps, 5)
     peak = measured_hbm_peak()
+    alhr.set_launch_mode(args.launch_mode)
 
     def stages(wl):
         vb = max(-wl.qk_lo, wl.qk_hi)
@@ -461,11 +466,12 @@ def run_stages(args):
     base = synth.WORKLOADS[args.workload]
     t, keys, fb = stages(base)
     report = {"report": "stages", "workload": describe(base), "reps": reps,
+              "launch_mode": args.launch_mode,
               "stage_ms": {k: v * 1e3 for k, v in t.items()}, "mean_keys_per_query": keys,
               "fused_forward_algorithmic_bytes": fb,
               "fused_forward_GBps": fb / t["fused_forward"] / 1e9, "peak_GBps": peak,
               "scaling": []}
-    sweep = [1024, 4096, 16384, 65536]
+    sweep = [] if args.no_sweep else [1024, 4096, 16384, 65536]
     for n in sweep:
         wl = base.replace(n=n, nq=n, q_start=0)
         t, keys, fb = stages(wl)
@@ -476,9 +482,10 @@ def run_stages(args):
                                   "mean_keys_per_query": keys,
                                   "fused_forward_GBps": fb / t["fused_forward"] / 1e9,
                                   "frac_of_copy_peak": fb / t["fused_forward"] / 1e9 / peak})
-    xs = np.log([e["n"] for e in report["scaling"]])
-    ys = np.log([e["fused_forward_ms"] for e in report["scaling"]])
-    report["loglog_exponent_fused_forward_vs_n"] = float(np.polyfit(xs, ys, 1)[0])
+    if sweep:
+        xs = np.log([e["n"] for e in report["scaling"]])
+        ys = np.log([e["fused_forward_ms"] for e in report["scaling"]])
+        report["loglog_exponent_fused_forward_vs_n"] = float(np.polyfit(xs, ys, 1)[0])
     report["gpu"] = torch.cuda.get_device_name(dev)
     print(json.dumps(report))
 
