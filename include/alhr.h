@@ -16,7 +16,9 @@
  *     [README §Results and Variables: the caps are 96 keys and 32 budget classes];
  *   - the neighbour window is w keys (16 in the README's setting).
  *
- * Memory layouts (all row-major, contiguous, device memory, 16-byte aligned base pointers):
+ * Memory layouts (all row-major, contiguous, device memory, 16-byte aligned base pointers; the
+ * tree 32-byte aligned, since its rows are read 32 bytes at a time — cudaMalloc and torch
+ * allocations are 256-byte aligned):
  *   Q      int8     [batch][heads][nq][d]        row t is the query at position q_start+t
  *   K      int8     [batch][heads][n][d]
  *   V      uint16   [batch][heads][n][d]         bf16 bit patterns

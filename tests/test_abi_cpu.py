@@ -138,6 +138,7 @@ def test_entry_points_reject_bad_arguments_before_launch(A):
     L = A.lib()
     fake = ctypes.c_void_p(0x10000)     # never dereferenced: every call below fails its checks
     odd = ctypes.c_void_p(0x10008)      # not 16-byte aligned
+    odd32 = ctypes.c_void_p(0x10010)    # 16-byte but not 32-byte aligned (enough but for a tree)
     null = None
     d = ctypes.byref(_dims(A))
     assert L.alhr_build_tree(None, fake, fake, null, null) == 1
@@ -163,6 +164,14 @@ def test_entry_points_reject_bad_arguments_before_launch(A):
         assert L.alhr_update_tree(d, fake, fake, lo, hi, null, null) == 1, (lo, hi)
     assert L.alhr_update_tree(d, null, fake, 0, 1, null, null) == 1
     assert L.alhr_update_tree(d, fake, odd, 0, 1, null, null) == 1
+    # the tree is read 32 bytes at a time: a 16-byte aligned tree is refused everywhere
+    assert L.alhr_build_tree(d, fake, odd32, null, null) == 1
+    assert L.alhr_update_tree(d, fake, odd32, 0, 1, null, null) == 1
+    assert L.alhr_tree_unpack(d, odd32, fake, null) == 1
+    assert L.alhr_forward(d, fake, fake, fake, odd32, fake, null, fake, null, null, null, null,
+                          null, null) == 1
+    assert L.alhr_route(d, fake, fake, odd32, fake, fake, fake, null, null, null) == 1
+    assert L.alhr_predict_budget(d, fake, fake, odd32, fake, fake, null, null) == 1
     assert L.alhr_update_tree(ctypes.byref(_dims(A, d=32)), fake, fake, 0, 1, null, null) == 2
     # nothing to do: no pointer is needed
     assert L.alhr_update_tree(d, null, null, 5, 5, null, null) == 0

@@ -21,6 +21,8 @@ int log2_exact(int32_t n) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// the tree is read with 32-byte loads
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 int value_bound_of(const alhr_dims* d) { return d->value_bound == 0 ? 16 : d->value_bound; }
 
@@ -144,7 +146,7 @@ alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, void* tree,
                             uint32_t* dev_err, void* stream) {
   const alhr_status s = check_common(dims);
   if (s != ALHR_OK) return s;
-  if (!K || !tree || !aligned16(K) || !aligned16(tree)) return ALHR_ERR_INVALID_ARG;
+  if (!K || !tree || !aligned16(K) || !aligned32(tree)) return ALHR_ERR_INVALID_ARG;
   const long long bh = (long long)dims->batch * dims->heads;
   const alhr::TreeLayout tl = alhr::make_tree_layout(dims->n, dims->d, dims->value_bound);
   return from_cuda(alhr::launch_build_tree(K, static_cast<char*>(tree), tl, bh,
@@ -173,7 +175,7 @@ alhr_status alhr_update_tree(const alhr_dims* dims, const int8_t* K, void* tree,
   if (s != ALHR_OK) return s;
   if (lo < 0 || hi < lo || hi > dims->n) return ALHR_ERR_INVALID_ARG;
   if (lo == hi) return ALHR_OK;
-  if (!K || !tree || !aligned16(K) || !aligned16(tree)) return ALHR_ERR_INVALID_ARG;
+  if (!K || !tree || !aligned16(K) || !aligned32(tree)) return ALHR_ERR_INVALID_ARG;
   const long long bh = (long long)dims->batch * dims->heads;
   const alhr::TreeLayout tl = alhr::make_tree_layout(dims->n, dims->d, dims->value_bound);
   return from_cuda(alhr::launch_update_tree(K, static_cast<char*>(tree), tl, bh, lo, hi,
@@ -185,7 +187,7 @@ alhr_status alhr_tree_unpack(const alhr_dims* dims, const void* tree, int32_t* n
                              void* stream) {
   const alhr_status s = check_common(dims);
   if (s != ALHR_OK) return s;
-  if (!tree || !nodes || !aligned16(tree) || !aligned16(nodes)) return ALHR_ERR_INVALID_ARG;
+  if (!tree || !nodes || !aligned32(tree) || !aligned16(nodes)) return ALHR_ERR_INVALID_ARG;
   const long long bh = (long long)dims->batch * dims->heads;
   const alhr::TreeLayout tl = alhr::make_tree_layout(dims->n, dims->d, dims->value_bound);
   return from_cuda(alhr::launch_tree_unpack(static_cast<const char*>(tree), tl, bh, nodes,
@@ -201,7 +203,7 @@ alhr_status alhr_predict_budget(const alhr_dims* dims, const int8_t* Q, const in
   if (s != ALHR_OK) return s;
   if (dims->nq == 0) return ALHR_OK;  // nothing to read or write
   if (!Q || !K || !tree || !W || !budget) return ALHR_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(tree) || !aligned16(W)) return ALHR_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned32(tree) || !aligned16(W)) return ALHR_ERR_INVALID_ARG;
   alhr::QueryArgs a = base_args(dims);
   a.Q = Q; a.K = K; a.tree = static_cast<const char*>(tree); a.W = W; a.budget_out = budget; a.dev_err = dev_err;
   return from_cuda(alhr::launch_predict(a, dims->d, bits, static_cast<cudaStream_t>(stream)));
@@ -216,7 +218,7 @@ alhr_status alhr_route(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
   if (s != ALHR_OK) return s;
   if (dims->nq == 0) return ALHR_OK;  // nothing to read or write
   if (!Q || !K || !tree || !budget || !idx || !count) return ALHR_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(tree)) return ALHR_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned32(tree)) return ALHR_ERR_INVALID_ARG;
   alhr::QueryArgs a = base_args(dims);
   a.Q = Q; a.K = K; a.tree = static_cast<const char*>(tree); a.budget_in = budget;
   a.idx_out = idx; a.count_out = count; a.exp_out = expansions; a.dev_err = dev_err;
@@ -248,7 +250,7 @@ alhr_status alhr_forward(const alhr_dims* dims, const int8_t* Q, const int8_t* K
   if (dims->nq == 0) return ALHR_OK;  // nothing to read or write
   if (!Q || !K || !V || !tree || !out) return ALHR_ERR_INVALID_ARG;
   if (!W && !budget_override) return ALHR_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(tree) || !aligned16(out))
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned32(tree) || !aligned16(out))
     return ALHR_ERR_INVALID_ARG;
   if (!budget_override && !aligned16(W)) return ALHR_ERR_INVALID_ARG;
   alhr::QueryArgs a = base_args(dims);

@@ -1,7 +1,7 @@
 // alhr_device.cuh -- device building blocks of the warp-per-query ALHR path (sm_100a).
 //
 // One warp owns one query. Rows are scored in "row groups": TPR = d/16 consecutive lanes share a
-// row and each lane holds 16 of its dims (dims 4*(sub + TPR*v) + e for v, e < 4, sub = lane %
+// row and each lane holds 16 of its dims (dims 8*(sub + TPR*v) + e for v < 2, e < 8, sub = lane %
 // TPR), so one warp pass scores RPI = 32/TPR rows (8 at d=64, 4 at d=128): a tree row (int32) is
 // four 16-byte loads and 16 multiply-adds per lane, a key row (int8) four 4-byte loads and four
 // dp4a per lane, and a row score costs log2(TPR) shuffles. The value rows of the final weighted
@@ -105,36 +105,32 @@ __device__ __forceinline__ int tree_row_offset(int n, int narrow, int level, int
   return off + j * (is_narrow ? 2 * D : 4 * D);
 }
 
-// The query in the row-group layouts. Key rows and int32 tree rows: lane `sub` of a group holds
-// dims 4m .. 4m+3 for m = sub + TPR*v, v < 4 (qp: packed words for dp4a, qn: the same 16 values
-// sign-extended for int32 multiply-adds). int16 tree rows: the lane holds dims 8c .. 8c+7 for
-// c = sub + TPR*v, v < 2 (qw: the matching packed words for dp2a).
+// The query in the row-group layout shared by every row kind: lane `sub` of a group holds the
+// 16 dims 8c .. 8c+7 of the two chunks c = sub + TPR*v, v < 2 (qp: the four packed words, dims
+// 4j .. 4j+3 of the lane's 16 in word j, for dp4a against key rows and dp2a against int16 rows;
+// qn: the same 16 values sign-extended, qn[4j + e] = dim e of word j, for int32 rows).
 struct RowQ {
   int qp[4];
   int qn[16];
-  int qw[4];
 };
 
 template <int D>
 __device__ __forceinline__ void load_rowq(const int8_t* qrow, int sub, RowQ& q) {
   constexpr int TPR = Lay<D>::TPR;
-  const int* p = reinterpret_cast<const int*>(qrow) + sub;
-#pragma unroll
-  for (int v = 0; v < 4; ++v) {
-    q.qp[v] = __ldg(p + TPR * v);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) q.qn[4 * v + e] = sx8(q.qp[v], e);
-  }
-  const int2* p2 = reinterpret_cast<const int2*>(qrow) + sub;
+  const int2* p = reinterpret_cast<const int2*>(qrow) + sub;
 #pragma unroll
   for (int v = 0; v < 2; ++v) {
-    const int2 t = __ldg(p2 + TPR * v);
-    q.qw[2 * v] = t.x;
-    q.qw[2 * v + 1] = t.y;
+    const int2 t = __ldg(p + TPR * v);
+    q.qp[2 * v] = t.x;
+    q.qp[2 * v + 1] = t.y;
   }
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) q.qn[4 * j + e] = sx8(q.qp[j], e);
 }
 
-// An int16 tree row (2d bytes) in its row-group layout: two 16-byte loads per lane, 8 words of
+// An int16 tree row (2d bytes) in its row-group layout: one 16-byte load per chunk, 8 words of
 // two int16 each.
 template <int D>
 __device__ __forceinline__ void ld_tree16(const char* row, int sub, int (&w)[8]) {
@@ -157,53 +153,59 @@ __device__ __forceinline__ int dot_tree16(const RowQ& q, const int (&w)[8]) {
   int t = 0;
 #pragma unroll
   for (int v = 0; v < 2; ++v) {
-    s = __dp2a_lo(w[4 * v + 0], q.qw[2 * v], s);
-    t = __dp2a_hi(w[4 * v + 1], q.qw[2 * v], t);
-    s = __dp2a_lo(w[4 * v + 2], q.qw[2 * v + 1], s);
-    t = __dp2a_hi(w[4 * v + 3], q.qw[2 * v + 1], t);
+    s = __dp2a_lo(w[4 * v + 0], q.qp[2 * v], s);
+    t = __dp2a_hi(w[4 * v + 1], q.qp[2 * v], t);
+    s = __dp2a_lo(w[4 * v + 2], q.qp[2 * v + 1], s);
+    t = __dp2a_hi(w[4 * v + 3], q.qp[2 * v + 1], t);
   }
   s += t;
   return s;
 }
 
-// An int16 tree row read in the int32 row layout (dims 4m .. 4m+3, m = sub + TPR*v), widened;
-// used where rows of different widths are summed (the causal key sum).
+// An int16 tree row widened to the lane's 16 int32 values (one 16-byte load per chunk); used
+// where rows of different widths are summed (the causal key sum).
 template <int D>
 __device__ __forceinline__ void ld_tree16_as32(const char* row, int sub, int (&x)[16]) {
   constexpr int TPR = Lay<D>::TPR;
-  const uint2* p = reinterpret_cast<const uint2*>(row) + sub;
+  const uint4* p = reinterpret_cast<const uint4*>(row) + sub;
 #pragma unroll
-  for (int v = 0; v < 4; ++v) {
-    const uint2 t = __ldg(p + TPR * v);
-    x[4 * v + 0] = int(t.x << 16) >> 16;
-    x[4 * v + 1] = int(t.x) >> 16;
-    x[4 * v + 2] = int(t.y << 16) >> 16;
-    x[4 * v + 3] = int(t.y) >> 16;
+  for (int v = 0; v < 2; ++v) {
+    const uint4 t = __ldg(p + TPR * v);
+    const unsigned w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      x[8 * v + 2 * h] = int(w[h] << 16) >> 16;
+      x[8 * v + 2 * h + 1] = int(w[h]) >> 16;
+    }
   }
 }
 
-// A tree row (int32) in the row-group layout.
+// A tree row (int32) in the row-group layout: one 32-byte load per chunk (rows are 32-byte
+// aligned: the tree buffer is, and every row is a multiple of 256 bytes).
 template <int D>
 __device__ __forceinline__ void ld_tree(const char* row, int sub, int (&x)[16]) {
   constexpr int TPR = Lay<D>::TPR;
-  const int4* p = reinterpret_cast<const int4*>(row) + sub;
 #pragma unroll
-  for (int v = 0; v < 4; ++v) {
-    const int4 t = __ldg(p + TPR * v);
-    x[4 * v + 0] = t.x;
-    x[4 * v + 1] = t.y;
-    x[4 * v + 2] = t.z;
-    x[4 * v + 3] = t.w;
+  for (int v = 0; v < 2; ++v) {
+    const char* p = row + 32 * (sub + TPR * v);
+    asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+                 : "=r"(x[8 * v + 0]), "=r"(x[8 * v + 1]), "=r"(x[8 * v + 2]), "=r"(x[8 * v + 3]),
+                   "=r"(x[8 * v + 4]), "=r"(x[8 * v + 5]), "=r"(x[8 * v + 6]), "=r"(x[8 * v + 7])
+                 : "l"(p));
   }
 }
 
-// A key row (int8) in the row-group layout, as packed words.
+// A key row (int8) in the row-group layout, as packed words: one 8-byte load per chunk.
 template <int D>
 __device__ __forceinline__ void ld_key(const int8_t* row, int sub, int (&xp)[4]) {
   constexpr int TPR = Lay<D>::TPR;
-  const int* p = reinterpret_cast<const int*>(row) + sub;
+  const int2* p = reinterpret_cast<const int2*>(row) + sub;
 #pragma unroll
-  for (int v = 0; v < 4; ++v) xp[v] = __ldg(p + TPR * v);
+  for (int v = 0; v < 2; ++v) {
+    const int2 t = __ldg(p + TPR * v);
+    xp[2 * v] = t.x;
+    xp[2 * v + 1] = t.y;
+  }
 }
 
 template <typename S>
