@@ -353,13 +353,49 @@ struct ScoreLimits<long long> {
   static constexpr long long highest = 9223372036854775807LL;
 };
 
+// A node of the frontier or a candidate: its descriptor and its score.
+template <typename S>
+struct Cand {
+  int desc;
+  S score;
+};
+
+// N nodes in shared memory. With int32 scores each node is one 8-byte record, so one access
+// moves both fields; with int64 scores descriptors and scores are kept apart (a 16-byte padded
+// record measured slower).
+template <typename S, int N>
+struct CandArray {
+  int d[N];
+  S s[N];
+  __device__ __forceinline__ Cand<S> get(int e) const { return Cand<S>{d[e], s[e]}; }
+  __device__ __forceinline__ void put(int e, int desc, S score) {
+    d[e] = desc;
+    s[e] = score;
+  }
+  __device__ __forceinline__ int desc(int e) const { return d[e]; }
+  __device__ __forceinline__ S score(int e) const { return s[e]; }
+  __device__ __forceinline__ void set_desc(int e, int v) { d[e] = v; }
+  __device__ __forceinline__ void set_score(int e, S v) { s[e] = v; }
+};
+template <int N>
+struct CandArray<int, N> {
+  int2 c[N];  // (desc, score)
+  __device__ __forceinline__ Cand<int> get(int e) const {
+    const int2 v = c[e];
+    return Cand<int>{v.x, v.y};
+  }
+  __device__ __forceinline__ void put(int e, int desc, int score) { c[e] = make_int2(desc, score); }
+  __device__ __forceinline__ int desc(int e) const { return c[e].x; }
+  __device__ __forceinline__ int score(int e) const { return c[e].y; }
+  __device__ __forceinline__ void set_desc(int e, int v) { c[e].x = v; }
+  __device__ __forceinline__ void set_score(int e, int v) { c[e].y = v; }
+};
+
 // Per-warp scratch of one query (shared memory).
 template <typename S>
 struct WarpBuf {
-  int cdesc[kMaxCand];       // frontier / candidates
-  S cscore[kMaxCand];
-  int xdesc[kMaxFrontier];   // nodes expanded this step
-  S xscore[kMaxFrontier];
+  CandArray<S, kMaxCand> cand;       // frontier / candidates
+  CandArray<S, kMaxFrontier> xnode;  // nodes expanded this step
   int xrow[kMaxFrontier];    // byte offset of each expanded node's left child row (tree
                              // block or key rows of the head)
   S xleft[kMaxFrontier];     // score of that left child
@@ -476,8 +512,10 @@ __device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int
   for (int s = 0; s < NS; ++s) {
     const int e = lane + 32 * s;
     const bool ok = e < C;
-    sc[s] = ok ? B.cscore[e] : kLow;
-    ds[s] = ok ? B.cdesc[e] : 0;
+    Cand<S> cd{0, kLow};
+    if (ok) cd = B.cand.get(e);
+    sc[s] = cd.score;
+    ds[s] = cd.desc;
     // ranking by means: q . sum / 2^level, scaled by 2^L to stay an exact integer
     if (NORM && norm_l && ok) sc[s] = sc[s] * (S(1) << (norm_l - desc_level(ds[s])));
   }
@@ -516,8 +554,8 @@ __device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int
     const unsigned bal = __ballot_sync(kFull, keep[s]);
     if (keep[s]) {
       const int pos = base + __popc(bal & lanemask_lt(lane));
-      B.cdesc[pos] = ds[s];
-      B.cscore[pos] = (NORM && norm_l) ? S(sc[s] >> (norm_l - desc_level(ds[s]))) : sc[s];
+      B.cand.put(pos, ds[s],
+                 (NORM && norm_l) ? S(sc[s] >> (norm_l - desc_level(ds[s]))) : sc[s]);
     }
     base += __popc(bal);
   }

@@ -30,15 +30,14 @@ namespace alhr {
 
 enum Mode : int { kForwardPredict = 0, kForwardOverride = 1, kRouteOnly = 2, kPredictOnly = 3 };
 
-// Writes the two children of expanded node x (descriptor pd, score ps; left score `left`).
+// Writes the two children of expanded node x (the node p; its left child's score `left`).
 template <typename S>
-__device__ __forceinline__ void put_children(WarpBuf<S>& B, int nl, int x, int pd, S ps, S left) {
-  const int cl = desc_level(pd) - 1;
-  const int st = desc_start(pd);
-  B.cdesc[nl + 2 * x] = make_desc(st, cl);
-  B.cscore[nl + 2 * x] = left;
-  B.cdesc[nl + 2 * x + 1] = make_desc(st + (1 << cl), cl);
-  B.cscore[nl + 2 * x + 1] = ps - left;
+__device__ __forceinline__ void put_children(WarpBuf<S>& B, int nl, int x, Cand<S> p, S left) {
+  const int cl = desc_level(p.desc) - 1;
+  const int st = desc_start(p.desc);
+  const S ps = p.score;
+  B.cand.put(nl + 2 * x, make_desc(st, cl), left);
+  B.cand.put(nl + 2 * x + 1, make_desc(st + (1 << cl), cl), ps - left);
 }
 
 // Dynamic shared memory of a query kernel: the predictor weights (the G half widened to
@@ -117,7 +116,7 @@ __device__ __noinline__ int expand_buckets(WarpBuf<S>& B, int nf, const int8_t* 
     const int e = lane + 32 * s;
     int sz = 0, st = 0;
     if (e < nf) {
-      const int ds = B.cdesc[e];
+      const int ds = B.cand.desc(e);
       sz = 1 << desc_level(ds);
       st = desc_start(ds);
     }
@@ -138,8 +137,7 @@ __device__ __noinline__ int expand_buckets(WarpBuf<S>& B, int nf, const int8_t* 
     if (k < total) ld_key<D>(Kh + (long long)B.xrow[k] * D, sub, xp);
     const int sc = group_sum<int, TPR>(dot_key(q, xp));
     if (k < total && sub == 0) {
-      B.cdesc[k] = make_desc(B.xrow[k], 0);
-      B.cscore[k] = S(sc);
+      B.cand.put(k, make_desc(B.xrow[k], 0), S(sc));
     }
   }
   __syncwarp();
@@ -184,9 +182,9 @@ __device__ __noinline__ void write_selection(const WarpBuf<S>& B, int nf, int ns
   for (int s = 0; s < kFrontSlots; ++s) {
     const int e = lane + 32 * s;
     if (e < nf) {
-      const int st = desc_start(B.cdesc[e]);
+      const int st = desc_start(B.cand.desc(e));
       int rank = 0;
-      for (int f = 0; f < nf; ++f) rank += desc_start(B.cdesc[f]) < st ? 1 : 0;
+      for (int f = 0; f < nf; ++f) rank += desc_start(B.cand.desc(f)) < st ? 1 : 0;
       io[rank] = st;
     }
   }
@@ -366,8 +364,7 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
             if (k < nA && sub == 0) {
               const int pd = B.plist[k];
               if (pd & kFlagRoot) {
-                B.cdesc[k] = pd & ~(kFlagRoot | kFlagG);
-                B.cscore[k] = rsc[ps][u];
+                B.cand.put(k, pd & ~(kFlagRoot | kFlagG), rsc[ps][u]);
               }
             }
           }
@@ -400,8 +397,7 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
         }
         sc = group_sum<S, TPR>(sc);
         if (active && sub == 0 && (pd & kFlagRoot)) {
-          B.cdesc[k] = pd & ~(kFlagRoot | kFlagG);  // common roots are the first ones
-          B.cscore[k] = sc;
+          B.cand.put(k, pd & ~(kFlagRoot | kFlagG), sc);  // common roots are the first ones
         }
       }
       if constexpr (!LAT) {
@@ -476,8 +472,7 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
             const int k = base + u * RPI + grp;
             const S sc = group_sum<S, TPR>(dot_tree<S>(q, x[u]));
             if (k < nB && sub == 0) {
-              B.cdesc[n_common + k] = B.plist[k];
-              B.cscore[n_common + k] = sc;
+              B.cand.put(n_common + k, B.plist[k], sc);
             }
           }
         }
@@ -506,8 +501,7 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
         }
         sc = group_sum<S, TPR>(sc);
         if (active && sub == 0) {
-          B.cdesc[n_common + k] = pd;
-          B.cscore[n_common + k] = sc;
+          B.cand.put(n_common + k, pd, sc);
         }
       }
       nf = __popc(Mu);
@@ -530,8 +524,9 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
           if (32 * s < nf) {  // warp-uniform: only the slots the frontier occupies
             const int e = lane + 32 * s;
             if (e < nf) {
-              fd[s] = B.cdesc[e];
-              fs[s] = B.cscore[e];
+              const Cand<S> cd = B.cand.get(e);
+              fd[s] = cd.desc;
+              fs[s] = cd.score;
               const int lv = desc_level(fd[s]);
               cat[s] = lv <= bucket ? 1 : (lv == 1 ? 4 : ((!kNarrow || lv - 1 > narrow) ? 2 : 3));
             }
@@ -574,13 +569,11 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
                                                          : ok + __popc(bk_[s] & below));
               const int cl = desc_level(fd[s]) - 1;
               const int st = desc_start(fd[s]);
-              B.xdesc[pos] = fd[s];
-              B.xscore[pos] = fs[s];
+              B.xnode.put(pos, fd[s], fs[s]);
               B.xrow[pos] = cat[s] == 4 ? st * D : tree_row_offset<D>(n, narrow, cl, st >> cl);
             } else if (cat[s] == 1) {
               const int pos = ol + __popc(bl_[s] & below);
-              B.cdesc[pos] = fd[s];
-              B.cscore[pos] = fs[s];
+              B.cand.put(pos, fd[s], fs[s]);
             }
             ow += __popc(bw_[s]);
             on += __popc(bn_[s]);
@@ -623,7 +616,7 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
         __syncwarp();
         // both children of every expanded node, one node per lane
         for (int x0 = lane; x0 < nx; x0 += 32)
-          put_children<S>(B, nl, x0, B.xdesc[x0], B.xscore[x0], B.xleft[x0]);
+          put_children<S>(B, nl, x0, B.xnode.get(x0), B.xleft[x0]);
         const int C = nl + 2 * nx;
         if (C > keep) {
           select_top_r<S, VAR>(B, C, keep, lane, norm_l);
@@ -678,8 +671,10 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
 #pragma unroll
       for (int s = 0; s < kFrontSlots; ++s) {
         const int e = lane + 32 * s;
-        sr[s] = e < nf ? float(B.cscore[e]) * scale : -INFINITY;
-        kr[s] = e < nf ? desc_start(B.cdesc[e]) : 0;
+        Cand<S> cd{0, S(0)};
+        if (e < nf) cd = B.cand.get(e);
+        sr[s] = e < nf ? float(cd.score) * scale : -INFINITY;
+        kr[s] = desc_start(cd.desc);
       }
       float m = sw;
 #pragma unroll
@@ -748,23 +743,23 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(const QueryArgs a) 
       key[s] = e < cnt ? __ldg(a.idx_in + qi * a.max_keys + e) : -1;
       ok[s] = e < cnt && key[s] >= 0 && key[s] <= i;
       bad |= e < cnt && !ok[s];
-      if (e < cnt) B.cdesc[e] = ok[s] ? key[s] : -1;
+      if (e < cnt) B.cand.set_desc(e, ok[s] ? key[s] : -1);
     }
     if (__any_sync(kFull, bad) && lane == 0) flag(a.dev_err, ALHR_DEVERR_INDEX);
     __syncwarp();
     for (int base = 0; base < cnt; base += RPI) {
       const int x = base + grp;
-      const int kk = x < cnt ? B.cdesc[x] : -1;
+      const int kk = x < cnt ? B.cand.desc(x) : -1;
       int xp[4] = {0, 0, 0, 0};
       if (kk >= 0) ld_key<D>(Kh + (long long)kk * D, sub, xp);
       const int s = group_sum<int, TPR>(dot_key(q, xp));
-      if (x < cnt && sub == 0) B.cscore[x] = s;
+      if (x < cnt && sub == 0) B.cand.set_score(x, s);
     }
     __syncwarp();
     float sc[kFrontSlots];
 #pragma unroll
     for (int s = 0; s < kFrontSlots; ++s)
-      sc[s] = ok[s] ? float(B.cscore[lane + 32 * s]) * a.scale : -INFINITY;
+      sc[s] = ok[s] ? float(B.cand.score(lane + 32 * s)) * a.scale : -INFINITY;
     float m = -INFINITY;
 #pragma unroll
     for (int s = 0; s < kFrontSlots; ++s) m = fmaxf(m, sc[s]);
