@@ -126,9 +126,9 @@ __global__ void __launch_bounds__(kTreeThreads)
 // load per key). The chunk is read in batches of 2^P keys, all loads of a batch issued before
 // any sum and one batch ahead; levels 1 .. P above a batch are summed in registers, and levels
 // P+1 .. m are carried from batch to batch in a per-lane stack that works like a binary counter
-// on the batch index.
-// Every node is written once, as soon as the last key beneath it has been read, and no shared
-// memory or barrier is involved, so many batches of many warps are in flight at once.
+// on the batch index. Every node is written once, as soon as the last key beneath it has been
+// read, and no shared memory or barrier is involved, so many batches of many warps are in flight
+// at once.
 template <int D, int P>
 __global__ void __launch_bounds__(kTreeThreads)
     tree_stream_kernel(const int8_t* __restrict__ K, char* __restrict__ tree, const TreeLayout tl,
