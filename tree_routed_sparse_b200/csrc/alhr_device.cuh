@@ -1,8 +1,8 @@
 // alhr_device.cuh -- device building blocks of the warp-per-query ALHR path (sm_100a).
 //
 // One warp owns one query. Rows are scored in "row groups": TPR = d/16 consecutive lanes share a
-// row and each lane holds 16 of its dims (dims 8*(sub + TPR*v) + e for v < 2, e < 8, sub = lane %
-// TPR), so one warp pass scores RPI = 32/TPR rows (8 at d=64, 4 at d=128): a tree row (int32) is
+// row and each lane holds 16 of its dims (see the row-group layout below), so one warp pass
+// scores RPI = 32/TPR rows (8 at d=64, 4 at d=128): a tree row (int32) is
 // four 16-byte loads and 16 multiply-adds per lane, a key row (int8) four 4-byte loads and four
 // dp4a per lane, and a row score costs log2(TPR) shuffles. The value rows of the final weighted
 // sum use the plain layout instead: lane l owns dims [l*d/32, (l+1)*d/32) of every value row.
@@ -105,44 +105,80 @@ __device__ __forceinline__ int tree_row_offset(int n, int narrow, int level, int
   return off + j * (is_narrow ? 2 * D : 4 * D);
 }
 
-// The query in the row-group layout shared by every row kind: lane `sub` of a group holds the
-// 16 dims 8c .. 8c+7 of the two chunks c = sub + TPR*v, v < 2 (qp: the four packed words, dims
-// 4j .. 4j+3 of the lane's 16 in word j, for dp4a against key rows and dp2a against int16 rows;
-// qn: the same 16 values sign-extended, qn[4j + e] = dim e of word j, for int32 rows).
+// The row-group layout, shared by every row kind (TPR = d/16 lanes per row, sub = lane % TPR):
+// at d = 128 lane `sub` holds the 16 consecutive dims 16*sub .. 16*sub+15 of a row; at d = 64
+// it holds the two 8-dim chunks 8c .. 8c+7, c = sub and sub + TPR. Either way the lane's dims
+// come as four 4-dim words j = 0..3 (dims 4j .. 4j+3 of the lane's 16). Consecutive dims mean
+// fewer, wider loads (one 32-byte load for an int16 row, one 16-byte load for a key row);
+// chunks measured faster at d = 64, where they keep the fused kernel within its registers.
+template <int D>
+constexpr bool kBlockLayout = (D == 128);
+
+// The query in the row-group layout (qp: the lane's four packed words, for dp4a against key
+// rows and dp2a against int16 rows; qn: the same 16 values sign-extended, qn[4j + e] = dim e of
+// word j, for int32 rows).
 struct RowQ {
   int qp[4];
   int qn[16];
 };
 
+// 32 bytes from global memory in one load (sm_100; p 32-byte aligned).
+__device__ __forceinline__ void ldg32B(const void* p, int (&w)[8]) {
+  asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]),
+                 "=r"(w[6]), "=r"(w[7])
+               : "l"(p));
+}
+
+// The lane's four words of an int8 row (a query or a key): one 16-byte load (d = 128) or two
+// 8-byte loads (d = 64).
+template <int D>
+__device__ __forceinline__ void ld_bytes16(const int8_t* row, int sub, int (&w)[4]) {
+  constexpr int TPR = Lay<D>::TPR;
+  if constexpr (kBlockLayout<D>) {
+    const int4 t = __ldg(reinterpret_cast<const int4*>(row) + sub);
+    w[0] = t.x;
+    w[1] = t.y;
+    w[2] = t.z;
+    w[3] = t.w;
+  } else {
+    const int2* p = reinterpret_cast<const int2*>(row) + sub;
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const int2 t = __ldg(p + TPR * v);
+      w[2 * v] = t.x;
+      w[2 * v + 1] = t.y;
+    }
+  }
+}
+
 template <int D>
 __device__ __forceinline__ void load_rowq(const int8_t* qrow, int sub, RowQ& q) {
-  constexpr int TPR = Lay<D>::TPR;
-  const int2* p = reinterpret_cast<const int2*>(qrow) + sub;
-#pragma unroll
-  for (int v = 0; v < 2; ++v) {
-    const int2 t = __ldg(p + TPR * v);
-    q.qp[2 * v] = t.x;
-    q.qp[2 * v + 1] = t.y;
-  }
+  ld_bytes16<D>(qrow, sub, q.qp);
 #pragma unroll
   for (int j = 0; j < 4; ++j)
 #pragma unroll
     for (int e = 0; e < 4; ++e) q.qn[4 * j + e] = sx8(q.qp[j], e);
 }
 
-// An int16 tree row (2d bytes) in its row-group layout: one 16-byte load per chunk, 8 words of
-// two int16 each.
+// An int16 tree row (2d bytes) in its row-group layout: 8 words of two int16 each, word k
+// holding dims 2k, 2k+1 of the lane's 16 (one 32-byte load at d = 128, two 16-byte loads at
+// d = 64; rows are 32-byte aligned: the tree buffer is, and every row is a multiple of 256 bytes).
 template <int D>
 __device__ __forceinline__ void ld_tree16(const char* row, int sub, int (&w)[8]) {
   constexpr int TPR = Lay<D>::TPR;
-  const int4* p = reinterpret_cast<const int4*>(row) + sub;
+  if constexpr (kBlockLayout<D>) {
+    ldg32B(row + 32 * sub, w);
+  } else {
+    const int4* p = reinterpret_cast<const int4*>(row) + sub;
 #pragma unroll
-  for (int v = 0; v < 2; ++v) {
-    const int4 t = __ldg(p + TPR * v);
-    w[4 * v + 0] = t.x;
-    w[4 * v + 1] = t.y;
-    w[4 * v + 2] = t.z;
-    w[4 * v + 3] = t.w;
+    for (int v = 0; v < 2; ++v) {
+      const int4 t = __ldg(p + TPR * v);
+      w[4 * v + 0] = t.x;
+      w[4 * v + 1] = t.y;
+      w[4 * v + 2] = t.z;
+      w[4 * v + 3] = t.w;
+    }
   }
 }
 
@@ -152,60 +188,63 @@ __device__ __forceinline__ int dot_tree16(const RowQ& q, const int (&w)[8]) {
   // two independent accumulator chains (the intrinsic is not reassociated by the compiler)
   int t = 0;
 #pragma unroll
-  for (int v = 0; v < 2; ++v) {
-    s = __dp2a_lo(w[4 * v + 0], q.qp[2 * v], s);
-    t = __dp2a_hi(w[4 * v + 1], q.qp[2 * v], t);
-    s = __dp2a_lo(w[4 * v + 2], q.qp[2 * v + 1], s);
-    t = __dp2a_hi(w[4 * v + 3], q.qp[2 * v + 1], t);
+  for (int j = 0; j < 4; ++j) {
+    s = __dp2a_lo(w[2 * j], q.qp[j], s);
+    t = __dp2a_hi(w[2 * j + 1], q.qp[j], t);
   }
   s += t;
   return s;
 }
 
-// An int16 tree row widened to the lane's 16 int32 values (one 16-byte load per chunk); used
-// where rows of different widths are summed (the causal key sum).
+// An int16 tree row widened to the lane's 16 int32 values; used where rows of different widths
+// are summed (the causal key sum).
 template <int D>
 __device__ __forceinline__ void ld_tree16_as32(const char* row, int sub, int (&x)[16]) {
-  constexpr int TPR = Lay<D>::TPR;
-  const uint4* p = reinterpret_cast<const uint4*>(row) + sub;
+  int w[8];
+  ld_tree16<D>(row, sub, w);
 #pragma unroll
-  for (int v = 0; v < 2; ++v) {
-    const uint4 t = __ldg(p + TPR * v);
-    const unsigned w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      x[8 * v + 2 * h] = int(w[h] << 16) >> 16;
-      x[8 * v + 2 * h + 1] = int(w[h]) >> 16;
-    }
+  for (int k = 0; k < 8; ++k) {
+    x[2 * k] = (w[k] << 16) >> 16;
+    x[2 * k + 1] = w[k] >> 16;
   }
 }
 
-// A tree row (int32) in the row-group layout: one 32-byte load per chunk (rows are 32-byte
-// aligned: the tree buffer is, and every row is a multiple of 256 bytes).
+// A tree row (int32) in the row-group layout: two 32-byte loads per lane.
 template <int D>
 __device__ __forceinline__ void ld_tree(const char* row, int sub, int (&x)[16]) {
   constexpr int TPR = Lay<D>::TPR;
+  int w0[8], w1[8];
+  if constexpr (kBlockLayout<D>) {
+    ldg32B(row + 64 * sub, w0);
+    ldg32B(row + 64 * sub + 32, w1);
+  } else {
+    ldg32B(row + 32 * sub, w0);
+    ldg32B(row + 32 * (sub + TPR), w1);
+  }
 #pragma unroll
-  for (int v = 0; v < 2; ++v) {
-    const char* p = row + 32 * (sub + TPR * v);
-    asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
-                 : "=r"(x[8 * v + 0]), "=r"(x[8 * v + 1]), "=r"(x[8 * v + 2]), "=r"(x[8 * v + 3]),
-                   "=r"(x[8 * v + 4]), "=r"(x[8 * v + 5]), "=r"(x[8 * v + 6]), "=r"(x[8 * v + 7])
-                 : "l"(p));
+  for (int k = 0; k < 8; ++k) {
+    x[k] = w0[k];
+    x[8 + k] = w1[k];
   }
 }
 
-// A key row (int8) in the row-group layout, as packed words: one 8-byte load per chunk.
+// A key row (int8) in the row-group layout, as the lane's four packed words.
 template <int D>
 __device__ __forceinline__ void ld_key(const int8_t* row, int sub, int (&xp)[4]) {
+  ld_bytes16<D>(row, sub, xp);
+}
+
+// Slot of word m (dims 4m .. 4m+3) of a predictor weight row in shared memory, and the slot of
+// word j of the lane `sub`: words are grouped by their position in the lane's 16 dims, so the
+// lanes of a row group read consecutive slots.
+template <int D>
+__device__ __forceinline__ int w_slot(int m) {
+  return kBlockLayout<D> ? (m & 3) * (D / 16) + (m >> 2) : (m & 1) * (D / 8) + (m >> 1);
+}
+template <int D>
+__device__ __forceinline__ int w_lane_slot(int sub, int j) {
   constexpr int TPR = Lay<D>::TPR;
-  const int2* p = reinterpret_cast<const int2*>(row) + sub;
-#pragma unroll
-  for (int v = 0; v < 2; ++v) {
-    const int2 t = __ldg(p + TPR * v);
-    xp[2 * v] = t.x;
-    xp[2 * v + 1] = t.y;
-  }
+  return kBlockLayout<D> ? j * (D / 16) + sub : (j & 1) * (D / 8) + sub + TPR * (j >> 1);
 }
 
 template <typename S>

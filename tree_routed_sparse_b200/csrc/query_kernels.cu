@@ -42,8 +42,9 @@ __device__ __forceinline__ void put_children(WarpBuf<S>& B, int nl, int x, Cand<
 
 // Dynamic shared memory of a query kernel: the predictor weights (the G half widened to
 // int32, then the q half as packed int8 words; within a class row the 4-dim words are stored
-// even words first, then odd ones, and rows are padded, so that the row groups, which read
-// different classes at once, hit different banks) followed by one WarpBuf per warp.
+// grouped by their position in a lane's 16 dims, and rows are padded, so that the row groups,
+// which read different classes at once, hit different banks) followed by one WarpBuf per
+// warp.
 template <int D>
 struct WLayout {
   static constexpr int g_stride = D + 16;     // ints per class row of the G half
@@ -246,17 +247,15 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
   const int grp = lane / TPR;
   const int sub = lane % TPR;
   if constexpr (kUsesW) {
-    // word m (dims 4m .. 4m+3) of a class row is stored at slot (m & 1) * D/8 + (m >> 1): the
-    // lanes of a row group, which read the same half of consecutive 8-dim chunks, then read
-    // consecutive slots
+    // word m (dims 4m .. 4m+3) of a class row goes to slot w_slot<D>(m), so that the lanes of
+    // a row group read consecutive slots
     for (int k = threadIdx.x; k < 32 * D / 4; k += blockDim.x) {
       const int c = k / (D / 4), m = k - c * (D / 4);
-      sWq[c * QS + (m & 1) * (D / 8) + (m >> 1)] =
-          __ldg(reinterpret_cast<const int*>(a.W + c * 2 * D) + m);
+      sWq[c * QS + w_slot<D>(m)] = __ldg(reinterpret_cast<const int*>(a.W + c * 2 * D) + m);
     }
     for (int k = threadIdx.x; k < 32 * D; k += blockDim.x) {
-      const int c = k / D, t = k - c * D, m = t >> 2;
-      sWg[c * GS + 4 * ((m & 1) * (D / 8) + (m >> 1)) + (t & 3)] = a.W[c * 2 * D + D + t];
+      const int c = k / D, t = k - c * D;
+      sWg[c * GS + 4 * w_slot<D>(t >> 2) + (t & 3)] = a.W[c * 2 * D + D + t];
     }
     __syncthreads();
   }
@@ -416,9 +415,7 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
         long long sg = 0;
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          // word v of the lane's dims is word 2(sub + TPR (v >> 1)) + (v & 1) of the row, at
-          // slot (v & 1) * D/8 + sub + TPR (v >> 1)
-          const int m = (v & 1) * (D / 8) + sub + TPR * (v >> 1);
+          const int m = w_lane_slot<D>(sub, v);  // slot of the lane's word v
           sq = __dp4a(sWq[c * QS + m], q.qp[v], sq);
           const int4 wg = *reinterpret_cast<const int4*>(sWg + c * GS + 4 * m);
           sg += (long long)wg.x * G[4 * v] + (long long)wg.y * G[4 * v + 1] +
