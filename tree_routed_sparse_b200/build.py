@@ -10,6 +10,7 @@ from __future__ import annotations
 import glob
 import hashlib
 import os
+import re
 import subprocess
 import sys
 
@@ -47,17 +48,26 @@ def _hash() -> str:
 HEADERS = ["alhr_device.cuh", "internal.h", "tree_layout.h"]
 
 
+def code_only(text: str) -> str:
+    """C/C++/CUDA source without its comments and blank lines (the sources hold no string
+    literal with a comment marker)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_hash(source: str) -> str:
-    """Hash of one csrc/*.cu file, the headers every source includes and the flags: it
-    identifies the build of the kernels defined in that file, so a stored profiler record of
-    one kernel stays valid while only other files change."""
+    """Hash of the code (comments and blank lines left out) of one csrc/*.cu file, the headers
+    every source includes, and the flags: it identifies the kernels defined in that file, so a
+    stored profiler record of one kernel stays valid while only other files or comments
+    change."""
     h = hashlib.sha1()
     files = [os.path.join(PKG, "csrc", source)] + [
         os.path.join(PKG, "csrc", x) for x in HEADERS] + [os.path.join(ROOT, "include", "alhr.h")]
     for f in files:
         h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            h.update(code_only(fh.read()).encode())
     h.update(" ".join(FLAGS).encode())
     return h.hexdigest()
 

@@ -2,11 +2,11 @@
 //
 // One warp owns one query. Rows are scored in "row groups": TPR = d/16 consecutive lanes share a
 // row and each lane holds 16 of its dims (see the row-group layout below), so one warp pass
-// scores RPI = 32/TPR rows (8 at d=64, 4 at d=128): a tree row (int32) is
-// four 16-byte loads and 16 multiply-adds per lane, a key row (int8) four 4-byte loads and four
-// dp4a per lane, and a row score costs log2(TPR) shuffles. The value rows of the final weighted
-// sum use the plain layout instead: lane l owns dims [l*d/32, (l+1)*d/32) of every value row.
-// The frontier and the candidates of the descent live in a per-warp shared-memory buffer.
+// scores RPI = 32/TPR rows (8 at d=64, 4 at d=128): an int32 tree row is two 32-byte loads and
+// 16 multiply-adds per lane, an int16 tree row 8 dp2a, a key row four dp4a, and a row score
+// costs log2(TPR) shuffles. The value rows of the final weighted sum use value groups instead:
+// d/8 lanes share a value row, one 16-byte load of 8 bf16 each. The frontier and the
+// candidates of the descent live in a per-warp shared-memory buffer.
 #pragma once
 
 #include <cstdint>
