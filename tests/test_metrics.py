@@ -74,3 +74,17 @@ def test_bucket_keys_are_read_once_more():
     a = metrics.forward_bytes(pos, n, d, w, [16], none, [19], False, bucket_log=2)  # r = 3 < 4
     b = metrics.forward_bytes(pos, n, d, w, [16], none, [19], False)                # r = 3
     assert b - a == metrics._rows_bytes(np.array([500 - w + 1]), d, 0)[0]
+
+
+def test_tree_build_launch_count_follows_the_build_plan():
+    """bench.py's launch count of one alhr_build_tree: no streaming launch below 16 keys (one
+    shared-memory launch of up to 7 levels), else a streaming launch of 5 levels (7 from 2^24
+    keys in all) and one launch per further 7 levels."""
+    import bench
+    assert bench.tree_build_launches(1, 8) == 1           # 3 levels, one launch
+    assert bench.tree_build_launches(1, 16) == 1          # 4 levels streamed at once
+    assert bench.tree_build_launches(1, 32) == 1          # 5 levels streamed
+    assert bench.tree_build_launches(64, 256) == 2        # 5 streamed + 3
+    assert bench.tree_build_launches(16, 16384) == 3      # 5 + 7 + 2
+    assert bench.tree_build_launches(512, 262144) == 3    # 2^27 keys: 7 + 7 + 4
+    assert bench.tree_build_launches(1, 1 << 20) == 4     # 2^20 keys (small build): 5 + 7 + 7 + 1
