@@ -170,7 +170,8 @@ ALHR_API int32_t alhr_get_launch_mode(void);
  * For every (b,h) writes node(l, j) = sum_{t in [j*2^l, (j+1)*2^l)} K[t] for l = 1..log2 n,
  * exact, in the tree layout above. Only dims->batch, heads, n, d and value_bound are read.
  *   K       device, int8 [batch][heads][n][d], read only
- *   tree    device, batch*heads*alhr_tree_bytes(n, d, value_bound) bytes, fully overwritten
+ *   tree    device, 32-byte aligned, batch*heads*alhr_tree_bytes(n, d, value_bound) bytes,
+ *           fully overwritten
  *   dev_err device uint32 or NULL; ALHR_DEVERR_VALUE_RANGE if some |K| > value_bound (the
  *           narrow levels are then not exact)
  */
