@@ -51,6 +51,13 @@ MUTATIONS = {
     "labels_ties_to_higher_position": ("      return a.second < b.second;", "      return a.second > b.second;"),
     "labels_lowest_scores": ("      if (a.first != b.first) return a.first > b.first;",
                              "      if (a.first != b.first) return a.first < b.first;"),
+    "window_cut_far_first": (
+        "for (int64_t t = i; t >= 0 && t > int64_t(i) - w && int64_t(chosen.size()) < b_eff; --t)",
+        "for (int64_t t = std::max<int64_t>(0, int64_t(i) - w + 1); "
+        "t <= int64_t(i) && int64_t(chosen.size()) < b_eff; ++t)"),
+    "roots_smallest_first": ("for (int b = 62; b >= 0; --b) {", "for (int b = 0; b <= 62; ++b) {"),
+    "level_one_nodes_not_expanded": ("any_inner |= (nd.level > bucket_log);",
+                                     "any_inner |= (nd.level > bucket_log + 1);"),
 }
 
 PIN_TESTS = [
