@@ -58,12 +58,21 @@ MUTATIONS = {
     "roots_smallest_first": ("for (int b = 62; b >= 0; --b) {", "for (int b = 0; b <= 62; ++b) {"),
     "level_one_nodes_not_expanded": ("any_inner |= (nd.level > bucket_log);",
                                      "any_inner |= (nd.level > bucket_log + 1);"),
+    "roots_pruned_before_first_expansion": (
+        "    const bool norm = score_norm != 0;\n",
+        "    const bool norm = score_norm != 0;\n"
+        "    if (int64_t(frontier.size()) > keep) {\n"
+        "      std::sort(frontier.begin(), frontier.end(),\n"
+        "                [norm](const Node& a, const Node& b) { return ranks_before(a, b, norm); });\n"
+        "      frontier.resize(size_t(keep));\n"
+        "    }\n"),
 }
 
 PIN_TESTS = [
     ("golden_tree", lambda g: pins.test_golden_tree(g)),
     ("golden_causal", lambda g: pins.test_golden_causal_sums(g)),
     ("golden_routes", lambda g: pins.test_golden_routes(g)),
+    ("roots_not_pruned_first", lambda g: pins.test_roots_not_pruned_before_the_first_expansion(g)),
     ("golden_predictor", lambda g: pins.test_golden_predictor(g)),
     ("golden_forward", lambda g: pins.test_golden_forward_composition(g)),
     ("root_children", lambda g: pins.test_tree_root_and_children(64, 64)),

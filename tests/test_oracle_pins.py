@@ -63,6 +63,20 @@ def test_golden_routes(golden_n8):
         assert list(exp) == case["expansions"], case["why"]
 
 
+def test_roots_not_pruned_before_the_first_expansion(golden_n8):
+    """Hand-worked on the N=8, d=2 keys of the golden example, q = (1, 2), i = 7, w = 1, B = 2:
+    the window is {7}, r = 1, and the forest of [0, 7) has three roots, more than the beam:
+    [0,4) (sum (2,3), score 8), [4,6) (sum (1,3), score 7) and key 6 (score -4). The descent
+    expands every non-leaf root before it prunes (reading R6): [0,2) 3, [2,4) 5, key 4 9, key 5
+    -2, key 6 -4, of which key 4 is kept: selection {4, 7}, one level-2 and one level-1 node
+    expanded. Pruning the roots first would follow [0,4) down to key 3 instead."""
+    K = np.array(golden_n8["K"], dtype=np.int8)
+    nodes = orc.build_tree(K)
+    sel, exp = orc.route(K, nodes, np.array([1, 2], dtype=np.int8), 7, 2, 1, 96)
+    assert sel.tolist() == [4, 7]
+    assert list(exp) == [1, 1]
+
+
 def test_golden_predictor(golden_n8):
     for case in golden_n8["predictor"]:
         W = np.zeros((32, 4), dtype=np.int8)
