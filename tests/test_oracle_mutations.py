@@ -58,6 +58,15 @@ MUTATIONS = {
     "roots_smallest_first": ("for (int b = 62; b >= 0; --b) {", "for (int b = 0; b <= 62; ++b) {"),
     "level_one_nodes_not_expanded": ("any_inner |= (nd.level > bucket_log);",
                                      "any_inner |= (nd.level > bucket_log + 1);"),
+    "budget_classes_off_by_one": ("budget = 3 * (oracle_predict(d, q, G.data(), W, nullptr) + 1);",
+                                  "budget = 3 * oracle_predict(d, q, G.data(), W, nullptr) + 1;"),
+    "causal_sum_without_window": ("for (int u = 0; u <= i; ++u) s += K[int64_t(u) * d + t];",
+                                  "for (int u = 0; u <= i - 16; ++u) s += K[int64_t(u) * d + t];"),
+    "window_without_own_key": (
+        "for (int64_t t = i; t >= 0 && t > int64_t(i) - w && int64_t(chosen.size()) < b_eff; --t)",
+        "for (int64_t t = i - 1; t >= 0 && t >= int64_t(i) - w && int64_t(chosen.size()) < b_eff; --t)"),
+    "value_row_of_the_previous_key": ("const uint16_t* v = V + int64_t(sel[k]) * d;",
+                                  "const uint16_t* v = V + int64_t(sel[k] == 0 ? 0 : sel[k] - 1) * d;"),
     "roots_pruned_before_first_expansion": (
         "    const bool norm = score_norm != 0;\n",
         "    const bool norm = score_norm != 0;\n"
