@@ -3,15 +3,20 @@ configured workload (tree build + fused route/attend over every query), on N GPU
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl alhr|reference]
 
-N > 1 runs one process per GPU under torch.distributed.run (weak scaling: every rank processes
-its own full workload with its own seed; no collective on the data path). Prints one JSON line
-on rank 0. Inputs are seeded synthetic tensors generated on the device; L2 is flushed by a
-512 MiB write before every timed step; the timed region holds exactly K steps bracketed by a
-barrier and a device synchronisation; each step is timed with CUDA events on the launch stream
-and the job time is the maximum over ranks.
+N > 1 runs one process per GPU under torch.distributed.run (started by this script itself when
+WORLD_SIZE is not set). Weak scaling: the global batch holds N times the workload's sequences
+and rank k processes its contiguous share of the (b, h) blocks, drawn from the seeded generator
+at their flat index in the global batch; no collective on the data path (NCCL carries only the
+barrier and the max-over-ranks time). Prints one JSON line on rank 0. Inputs are seeded
+synthetic tensors generated on the device; L2 is flushed by a 512 MiB write before every timed
+step; the timed region holds exactly K steps bracketed by a barrier and a device
+synchronisation; each step is timed with CUDA events on the launch stream and the job time is
+the maximum over ranks.
 
 --impl reference times the oracle (the plain CPU reference that the tests use) on the host
-cores, on a bounded sample of the same workload, with the same metric.
+cores with the same metric: every step is one fully computed unit of the same workload (each
+(b, h) block's tree and every R-th query row, rotating the offset from step to step), timed
+as it runs; nothing is scaled.
 """
 from __future__ import annotations
 
@@ -20,6 +25,7 @@ import datetime
 import json
 import math
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -35,9 +41,13 @@ sys.path.insert(0, HERE)
 METRIC = "routed queries/sec and achieved HBM GB/s vs ~8 TB/s roofline, N=16384, 1 B200"
 DEFAULT_WORKLOAD = "prefill_b2h8_n16384"
 L2_FLUSH_BYTES = 512 << 20
+L2_NOTE = "flushed by a 512 MiB write before every timed GPU step (not timed)"
+# predictor classes kept live at the pages' operating point (rows of the higher classes are
+# zero): the budget is then 3 (c + 1) with c uniform over 0..19, about 31 keys per query
+OP_LIVE_CLASSES = 20
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=500)
@@ -45,6 +55,8 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="alhr", choices=["alhr", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--op-steps", type=int, default=100,
+                    help="launches timed at the operating point of about 30 keys per query")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--labels", action="store_true",
                     help="instead of the bench line: time the phase-2 label kernel "
@@ -61,26 +73,53 @@ def parse():
                          "the workload's keys (1 GPU)")
     ap.add_argument("--batch", type=int, default=0,
                     help="with --tree: replace the workload's batch (sequences)")
-    ap.add_argument("--cpu-sample-stride", type=int, default=4,
-                    help="CPU baseline: every k-th query row of every (b,h) block")
-    ap.add_argument("--ref-stride", type=int, default=64,
-                    help="--impl reference: every k-th query row of each step's block")
-    return ap.parse_args()
+    ap.add_argument("--cpu-steps", type=int, default=4,
+                    help="CPU baseline: oracle steps on all host cores (each as a reference step)")
+    ap.add_argument("--row-stride", type=int, default=16,
+                    help="oracle steps: every R-th query row of every (b,h) block, the first "
+                         "row rotating with the step")
+    ap.add_argument("--no-single-thread", action="store_true",
+                    help="CPU baseline: skip the single-threaded full-block timing")
+    return ap.parse_args(argv)
 
 
 def describe(wl) -> str:
     pred = (f"predictor W int8 U[{wl.w_lo},{wl.w_hi}] 32x{2 * wl.d}" if wl.predictor
             else f"fixed budget min(i+1,{wl.fixed_budget_cap})")
+    if wl.predictor and wl.live_classes < 32:
+        pred += f" with classes >= {wl.live_classes} zeroed"
     extra = f", {wl.plant_pairs} planted pairs/seq" if wl.plant_pairs else ""
     return (f"{wl.name}: batch {wl.batch}, heads {wl.heads}, N={wl.n}, d={wl.d}, "
             f"queries [{wl.q_start},{wl.q_start + wl.nq}), w={wl.window}, max_keys={wl.max_keys}, "
             f"Q/K int8 U[{wl.qk_lo},{wl.qk_hi}], V bf16 N(0,1), {pred}{extra}")
 
 
+def bench_config(wl) -> dict:
+    """The `config` object, identical in both arms: the per-GPU workload and the L2 policy."""
+    return {"workload": describe(wl), "l2": L2_NOTE}
+
+
 # ------------------------------------------------------------------ distributed plumbing
 
-def dist_setup(n_gpus):
+def free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def torchrun_command(argv: list[str], n: int, port: int) -> list[str]:
+    """The command that runs this script with the same arguments as n ranks, one per GPU."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__), *argv]
+
+
+def dist_setup(n_gpus: int):
+    """(dist module or None, rank, world) for a run under torch.distributed.run; the world size
+    must equal --gpus."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE {world}")
     if world > 1:
         import torch.distributed as dist
         local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -165,65 +204,86 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ oracle (CPU) timing
 
-def oracle_sample(wl, stride: int, blocks=None, inp=None) -> dict:
-    """The oracle as it stands, on the host cores, on a bounded sample of the workload: for
-    each listed (b,h) block, its whole tree and every `stride`-th query row. Blocks run on a
-    thread pool, one block per thread (the oracle itself is single-threaded; ctypes releases
-    the GIL). The sample's wall time is scaled to all query rows of the listed blocks, and
-    the value is queries of those blocks per extrapolated second."""
-    from concurrent.futures import ThreadPoolExecutor
-    from oracle import oracle as orc
-    from tree_routed_sparse_b200 import synth
-
-    orc.lib()
-    if inp is None:
-        inp = synth.make_inputs(wl, "cpu")
-    if blocks is None:
-        blocks = [(b, h) for b in range(wl.batch) for h in range(wl.heads)]
-    rows = np.arange(0, wl.nq, max(1, min(stride, wl.nq)), dtype=np.int32)
+def _host_blocks(inp):
+    """Per-(b,h) numpy views of host inputs."""
     Vbits = inp["V"].view(torch.int16).numpy().view(np.uint16)
     W = None if inp["W"] is None else inp["W"].numpy()
+    return Vbits, W
 
-    def run(bh):
-        b, h = bh
-        K = inp["K"][b, h].numpy()
-        Q = inp["Q"][b, h].numpy()
+
+def oracle_steps(wl, inp, steps: int, row_stride: int, first_step: int = 0) -> dict:
+    """The oracle as it stands on the host cores, step by step. Step s is one fully computed
+    unit of the workload: for every (b,h) block, its tree and the query rows r with
+    r = (first_step + s) mod R (mod R), R = min(row_stride, nq), so R consecutive steps cover
+    every row once. Blocks run on a thread pool, one block per thread (the oracle is
+    single-threaded; ctypes releases the GIL). Each step's wall time is measured as it runs;
+    the value is the queries computed over the summed step times."""
+    from concurrent.futures import ThreadPoolExecutor
+    from oracle import oracle as orc
+
+    orc.lib()
+    blocks = [(b, h) for b in range(wl.batch) for h in range(wl.heads)]
+    R = max(1, min(row_stride, wl.nq))
+    Vbits, W = _host_blocks(inp)
+
+    def run(arg):
+        (b, h), rows = arg
         bo = None if inp["budget_override"] is None else inp["budget_override"][b, h].numpy()
-        t0 = time.perf_counter()
-        nodes = orc.build_tree(K)
-        t1 = time.perf_counter()
-        orc.forward(Q, K, Vbits[b, h], nodes, W, bo, q_start=wl.q_start, window=wl.window,
-                    max_keys=wl.max_keys, rows=rows)
-        t2 = time.perf_counter()
-        return t1 - t0, t2 - t1
+        nodes = orc.build_tree(inp["K"][b, h].numpy())
+        orc.forward(inp["Q"][b, h].numpy(), inp["K"][b, h].numpy(), Vbits[b, h], nodes, W, bo,
+                    q_start=wl.q_start, window=wl.window, max_keys=wl.max_keys, rows=rows)
 
     threads = max(1, min(os.cpu_count() or 1, len(blocks)))
-    t0 = time.perf_counter()
+    times, queries = [], 0
     with ThreadPoolExecutor(threads) as ex:
-        res = list(ex.map(run, blocks))
-    wall = time.perf_counter() - t0
-    t_tree = sum(r[0] for r in res)
-    t_route = sum(r[1] for r in res)
-    scale = wl.nq / len(rows)
-    est_wall = wall * (t_tree + t_route * scale) / (t_tree + t_route)
-    total_q = len(blocks) * wl.nq
-    return {"value": total_q / est_wall, "unit": "queries/s", "cores": threads,
-            "kind": "oracle",
-            "sample": (f"{describe(wl)}; {len(blocks)} (b,h) blocks: each whole tree plus "
-                       f"every {max(1, min(stride, wl.nq))}-th query row ({len(rows)} of "
-                       f"{wl.nq}), time scaled to all rows; {threads} threads, one block per "
-                       f"thread; sample wall {wall:.2f} s"),
-            "sample_wall_s": wall}
+        for s in range(steps):
+            rows = np.arange((first_step + s) % R, wl.nq, R, dtype=np.int32)
+            t0 = time.perf_counter()
+            list(ex.map(run, [(bh, rows) for bh in blocks]))
+            times.append(time.perf_counter() - t0)
+            queries += len(rows) * len(blocks)
+    total = sum(times)
+    return {"value": queries / total if total > 0 else 0.0, "unit": "queries/s",
+            "cores": threads, "kind": "oracle", "step_s": times, "queries": queries,
+            "sample": (f"{describe(wl)}; {steps} step(s), each: the tree of every one of the "
+                       f"{len(blocks)} (b,h) blocks plus every {R}-th query row of it (rows "
+                       f"r = step mod {R}), {queries} queries in all, fully computed and timed "
+                       f"as run (no scaling); {threads} threads, one block per thread")}
+
+
+def oracle_single_thread(wl, inp) -> dict:
+    """BASELINE's single-threaded figure: block (b,h) = (0,0), its tree and every query row,
+    timed with std::chrono::steady_clock inside the oracle library on one thread."""
+    from oracle import oracle as orc
+    Vbits, W = _host_blocks(inp)
+    bo = None if inp["budget_override"] is None else inp["budget_override"][0, 0].numpy()
+    t, _ = orc.time_block(inp["Q"][0, 0].numpy(), inp["K"][0, 0].numpy(), Vbits[0, 0], W, bo,
+                          wl.q_start, wl.window, wl.max_keys)
+    return {"value": wl.nq / t, "unit": "queries/s", "cores": 1, "kind": "oracle",
+            "block_s": t, "us_per_query": t / wl.nq * 1e6,
+            "sample": (f"(b,h) = (0,0) of {wl.name}: its tree and all {wl.nq} queries, one "
+                       "thread, std::chrono::steady_clock inside the oracle library")}
 
 
 # ------------------------------------------------------------------ the GPU arm
 
+def fwd_algorithmic_bytes(wl, full, vb) -> int:
+    from tree_routed_sparse_b200 import metrics
+    pos = np.broadcast_to(np.arange(wl.q_start, wl.q_start + wl.nq),
+                          (full["count"].shape[0] * full["count"].shape[1], wl.nq))
+    return metrics.forward_bytes(pos, wl.n, wl.d, wl.window, full["count"].cpu().numpy(),
+                                 full["expansions"].cpu().numpy(), full["budget"].cpu().numpy(),
+                                 wl.predictor, wl.max_keys, value_bound=vb)
+
+
 def run_alhr(args, dist, rank, world):
-    from tree_routed_sparse_b200 import alhr, metrics, synth
+    from tree_routed_sparse_b200 import alhr, metrics, shard, synth
     dev = torch.device("cuda", torch.cuda.current_device())
-    wl = synth.WORKLOADS[args.workload].replace(seed=synth.WORKLOADS[args.workload].seed + rank)
+    wl = synth.WORKLOADS[args.workload]
+    wlg = shard.global_workload(wl, world)
+    lo, hi, inp = shard.shard_inputs(wlg, world, rank, dev)
+    assert hi - lo == wl.bh and inp["K"].shape[:2] == (wl.batch, wl.heads)
     vb = max(-wl.qk_lo, wl.qk_hi)
-    inp = synth.make_inputs(wl, dev)
     Q, K, V, W, bo = inp["Q"], inp["K"], inp["V"], inp["W"], inp["budget_override"]
     tree = torch.empty((wl.batch, wl.heads, alhr.tree_bytes(wl.n, wl.d, vb)), dtype=torch.uint8,
                        device=dev)
@@ -231,21 +291,15 @@ def run_alhr(args, dist, rank, world):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     kw = dict(q_start=wl.q_start, window=wl.window, max_keys=wl.max_keys,
               score_bits=wl.score_bits, value_bound=vb)
-
-    def step():
-        alhr.build_tree(K, tree, value_bound=vb)
-        alhr.forward(Q, K, V, tree, W=W, budget_override=bo, out=out, **kw)
+    path_bytes = sum(t.numel() * t.element_size() for t in (Q, K, V, W, bo, tree, out)
+                     if t is not None)
 
     # one untimed run with every output: counts for the byte model
     alhr.build_tree(K, tree, value_bound=vb)
     full = alhr.forward(Q, K, V, tree, W=W, budget_override=bo, want_count=True,
                         want_expansions=True, want_budget=True, **kw)
     torch.cuda.synchronize()
-    pos = np.broadcast_to(np.arange(wl.q_start, wl.q_start + wl.nq), (wl.bh, wl.nq))
-    fwd_bytes = metrics.forward_bytes(pos, wl.n, wl.d, wl.window, full["count"].cpu().numpy(),
-                                      full["expansions"].cpu().numpy(),
-                                      full["budget"].cpu().numpy(), wl.predictor, wl.max_keys,
-                                      value_bound=vb)
+    fwd_bytes = fwd_algorithmic_bytes(wl, full, vb)
     tree_bytes = metrics.tree_bytes(wl.bh, wl.n, wl.d, vb)
     mean_keys = float(full["count"].float().mean())
     mean_budget = float(full["budget"].float().mean())
@@ -253,12 +307,14 @@ def run_alhr(args, dist, rank, world):
 
     for _ in range(args.warmup):
         flush.fill_(1)
-        step()
+        alhr.build_tree(K, tree, value_bound=vb)
+        alhr.forward(Q, K, V, tree, W=W, budget_override=bo, out=out, **kw)
     torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream(dev)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    torch.cuda.reset_peak_memory_stats(dev)
     barrier(dist)
     torch.cuda.synchronize()
     sampler.start()
@@ -274,6 +330,7 @@ def run_alhr(args, dist, rank, world):
     wall = time.perf_counter() - wall0
     barrier(dist)
     clocks = sampler.stop()
+    peak_alloc = torch.cuda.max_memory_allocated(dev)
     t_tree = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
     t_fwd = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
     t_step = t_tree + t_fwd
@@ -307,23 +364,55 @@ def run_alhr(args, dist, rank, world):
     barrier(dist)
     t_e2e = max_over_ranks(dist, e2e_start.elapsed_time(e2e_end) / 1e3)
     e2e_value = world * queries * args.e2e_steps / t_e2e
+    del pipe, host, outs_host
+
+    # the pages' operating point (about 30 keys read per query): the same inputs, predictor
+    # rows of classes >= OP_LIVE_CLASSES zeroed; fused forward only (the tree is unchanged)
+    op = None
+    if W is not None and args.op_steps > 0:
+        W_op = W.clone()
+        W_op[OP_LIVE_CLASSES:] = 0
+        wl_op = wl.replace(live_classes=OP_LIVE_CLASSES)
+        full = alhr.forward(Q, K, V, tree, W=W_op, want_count=True, want_expansions=True,
+                            want_budget=True, **kw)
+        torch.cuda.synchronize()
+        op_bytes = fwd_algorithmic_bytes(wl_op, full, vb)
+        op_keys = float(full["count"].float().mean())
+        del full
+        for _ in range(3):
+            alhr.forward(Q, K, V, tree, W=W_op, out=out, **kw)
+        evo = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+               for _ in range(args.op_steps)]
+        barrier(dist)
+        torch.cuda.synchronize()
+        for s in range(args.op_steps):
+            flush.fill_(s & 0xFF)
+            evo[s][0].record(stream)
+            alhr.forward(Q, K, V, tree, W=W_op, out=out, **kw)
+            evo[s][1].record(stream)
+        torch.cuda.synchronize()
+        t_op = max_over_ranks(dist, sum(e[0].elapsed_time(e[1]) for e in evo) / 1e3)
+        op = {"workload": describe(wl_op), "mean_keys_per_query": op_keys,
+              "pages_keys_per_token": "30.0 / 32.0 / 30.0 at T = 1K / 4K / 16K (README TLDR)",
+              "queries_per_s": world * queries * args.op_steps / t_op,
+              "launch_ms": t_op / args.op_steps * 1e3, "algorithmic_bytes_per_launch": op_bytes}
 
     if rank != 0:
         return None
 
-    peaks = {}
-    try:
-        with open(os.path.join(HERE, "MEASURED_PEAKS.json")) as f:
-            peaks = json.load(f)
-    except OSError:
-        pass
-    peak = float(peaks.get("hbm_gbs", 6650.0))
-    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    peak = measured_hbm_peak()
+    peak_src = "measured" if peak_is_measured() else "fallback"
     fwd_launch_s = t_fwd / args.steps
     achieved = fwd_bytes / fwd_launch_s / 1e9
     rec = profiled_record(args.workload)
     traffic = rec.get("dram_bytes_per_launch") if rec else None
     tree_launches = tree_build_launches(wl.bh, wl.n)
+    if op is not None:
+        op_rec = profiled_record(f"{args.workload}+live{OP_LIVE_CLASSES}")
+        op_s = op["launch_ms"] / 1e3
+        op["algorithmic_GBps"] = op["algorithmic_bytes_per_launch"] / op_s / 1e9
+        op["frac_of_measured_hbm"] = op["algorithmic_GBps"] / peak
+        op["issue"] = issue_rate(op_rec, op_s)
     line = {
         "metric": METRIC,
         "value": value,
@@ -337,16 +426,15 @@ def run_alhr(args, dist, rank, world):
         "vs_baseline": None,
         "dtype": "int32",
         "data": "synthetic (seeded SplitMix64; random int8 predictor weights, no trained model)",
-        "config": {
-            "workload": describe(wl),
-            "queries_per_step_per_gpu": queries,
-            "step": "alhr_build_tree + alhr_forward (fused budget, window, descent, attention)",
-            "l2": "flushed by a 512 MiB write before every timed step (not timed)",
-            "parallelism": f"{world} independent replica(s), one per GPU, no collective",
-            "score_bits": 32 if alhr.score_bits(alhr.make_dims(Q, K, **kw)) == 32 else 64,
-            "mean_keys_per_query": mean_keys,
-            "mean_budget": mean_budget,
-        },
+        "config": bench_config(wl),
+        "step": "alhr_build_tree + alhr_forward (fused budget, window, descent, attention)",
+        "parallelism": (f"{world} GPU(s): a global batch of {wlg.batch} sequences x {wl.heads} "
+                        f"heads, each rank its contiguous {wl.bh} (b,h) blocks; no collective "
+                        "on the data path"),
+        "queries_per_step_per_gpu": queries,
+        "score_bits": 32 if alhr.score_bits(alhr.make_dims(Q, K, **kw)) == 32 else 64,
+        "mean_keys_per_query": mean_keys,
+        "mean_budget": mean_budget,
         "roofline": {
             "bound": "hbm",
             "kernel": "query_kernel (fused alhr_forward)",
@@ -358,17 +446,28 @@ def run_alhr(args, dist, rank, world):
             "algorithmic_bytes_per_launch": fwd_bytes,
             "launch_ms": fwd_launch_s * 1e3,
             "traffic": traffic,
+            "dram": dram_rate(traffic, fwd_launch_s, peak),
             "issue": issue_rate(rec, fwd_launch_s),
-            "note": ("algorithmic bytes count every row the path reads as if from DRAM; "
-                     "queries run in (b, h, i) order, so the rows in use at any time (about "
-                     "one head's tree, keys and values) stay in L2, repeat reads are served "
-                     "there and achieved can exceed the DRAM peak; traffic is the DRAM bytes "
-                     "ncu measured (compulsory reads and the output); issue is the binding "
-                     "resource, the kernel's warp instructions against the GPU's issue slots"),
+            "binding_resource": "instruction issue (see issue.frac); DRAM is not the limit",
+            "note": ("achieved counts every row the path reads (the algorithmic bytes of the "
+                     "metric) as if it came from DRAM; queries run in (b, h, i) order, so the "
+                     "rows in use at any time (about one head's tree, keys and values) stay in "
+                     "L2 and repeat reads are served there: achieved is a rate of row reads and "
+                     "can exceed the DRAM peak. dram is the DRAM traffic ncu measured "
+                     "(compulsory reads and the output) over the same launch time; issue is "
+                     "the binding resource, the kernel's warp instructions against the GPU's "
+                     "issue slots"),
         },
         "stages_ms": {"tree_build": t_tree / args.steps * 1e3,
                       "forward": t_fwd / args.steps * 1e3,
                       "tree_build_GBps": tree_bytes / (t_tree / args.steps) / 1e9},
+        "memory": {"peak_allocated_bytes": peak_alloc,
+                   "path_bytes": path_bytes,
+                   "l2_flush_buffer_bytes": L2_FLUSH_BYTES,
+                   "note": ("peak_allocated_bytes: torch.cuda.max_memory_allocated over the "
+                            "timed steps (the step's inputs, tree and output, plus the L2 flush "
+                            "buffer); the library itself allocates nothing")},
+        "operating_point_30_keys": op,
         "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                 "how": "HostPipeline: every step copies Q, K, V, W in from pinned host memory "
@@ -389,6 +488,24 @@ def measured_hbm_peak() -> float:
             return float(json.load(f)["hbm_gbs"])
     except (OSError, KeyError, ValueError):
         return 6650.0
+
+
+def peak_is_measured() -> bool:
+    try:
+        with open(os.path.join(HERE, "MEASURED_PEAKS.json")) as f:
+            return "hbm_gbs" in json.load(f)
+    except (OSError, ValueError):
+        return False
+
+
+def dram_rate(traffic, launch_s: float, peak: float):
+    """DRAM bytes per launch (ncu) over the live launch time, against the measured copy peak."""
+    if not traffic:
+        return None
+    gbps = traffic / launch_s / 1e9
+    return {"bytes_per_launch": traffic, "GBps": gbps, "frac": gbps / peak,
+            "source": "dram__bytes_read.sum + dram__bytes_write.sum from profiles/traffic.json "
+                      "(ncu), live launch time"}
 
 
 def tree_build_launches(bh: int, n: int) -> int:
@@ -581,57 +698,73 @@ def issue_rate(rec, launch_s: float):
             "source": "instruction count from profiles/traffic.json (ncu), live launch time"}
 
 
-def main():
-    args = parse()
+def run_reference(args):
+    """The reference arm: the oracle on the host cores, rank 0 only, K timed steps after W
+    warm-up steps, each step a fully computed unit of the same workload (oracle_steps)."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    from tree_routed_sparse_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    inp = synth.make_inputs(wl, "cpu")
+    if args.warmup:
+        oracle_steps(wl, inp, args.warmup, args.row_stride)
+    r = oracle_steps(wl, inp, args.steps, args.row_stride, first_step=args.warmup)
+    cb = {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": r["value"], "unit": "queries/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sum(r["step_s"]) / max(1, len(r["step_s"])) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64",
+        "data": "synthetic (seeded SplitMix64; random int8 predictor weights, no trained model)",
+        "config": bench_config(wl),
+        "step": ("the oracle (tree build + whole path) on every (b,h) block's tree and every "
+                 f"{max(1, min(args.row_stride, wl.nq))}-th query row, fully computed"),
+        "queries_per_step": r["queries"] // max(1, args.steps),
+        "cpu_baseline": cb,
+        "e2e": {"value": r["value"], "unit": "queries/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }))
+
+
+def cpu_baseline(args) -> dict:
+    """The GPU arm's CPU baseline (rank 0, N = 1 line): the reference arm's procedure for
+    --cpu-steps steps on all host cores, plus the single-threaded full-block figure."""
+    from tree_routed_sparse_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    inp = synth.make_inputs(wl, "cpu")
+    r = oracle_steps(wl, inp, args.cpu_steps, args.row_stride)
+    cb = {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    if not args.no_single_thread:
+        cb["single_thread"] = oracle_single_thread(wl, inp)
+    return cb
+
+
+def main(argv=None):
+    args = parse(argv)
     if args.impl == "reference":
-        # the oracle on the host cores; under torchrun only rank 0 works
-        rank = int(os.environ.get("RANK", "0"))
-        world = int(os.environ.get("WORLD_SIZE", "1"))
-        if rank != 0:
-            return
-        from tree_routed_sparse_b200 import synth
-        wl = synth.WORKLOADS[args.workload]
-        inp = synth.make_inputs(wl, "cpu")
-        all_blocks = [(b, h) for b in range(wl.batch) for h in range(wl.heads)]
-        # one step = one (b,h) block (whole tree, every stride-th query row), round robin
-        pick = lambda k: [all_blocks[j % len(all_blocks)] for j in range(k)]
-        if args.warmup:
-            oracle_sample(wl, args.ref_stride, pick(args.warmup), inp)
-        r = oracle_sample(wl, args.ref_stride, pick(args.steps), inp)
-        print(json.dumps({
-            "impl": "reference", "metric": METRIC, "value": r["value"], "unit": "queries/s",
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": wl.nq / r["value"] * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64",
-            "data": "synthetic", "config": {"workload": describe(wl),
-                                            "step": "one (b,h) block of the workload"},
-            "cpu_baseline": {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")},
-            "e2e": {"value": r["value"], "unit": "queries/s", "h2d_bytes_per_step": 0,
-                    "d2h_bytes_per_step": 0},
-        }))
+        run_reference(args)
+        return
+    if args.labels or args.tree or args.stages:
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA device")
+        from tree_routed_sparse_b200 import build
+        build.build()
+        (run_labels if args.labels else run_tree if args.tree else run_stages)(args)
         return
 
-    if args.labels:
-        if not torch.cuda.is_available():
-            raise SystemExit("bench.py needs a CUDA device")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: start this script again under torch.distributed.run
+        if not torch.cuda.is_available() or torch.cuda.device_count() < args.gpus:
+            raise SystemExit(f"--gpus {args.gpus}: only "
+                             f"{torch.cuda.device_count() if torch.cuda.is_available() else 0} "
+                             "CUDA device(s) visible")
         from tree_routed_sparse_b200 import build
-        build.build()
-        run_labels(args)
-        return
-    if args.tree:
-        if not torch.cuda.is_available():
-            raise SystemExit("bench.py needs a CUDA device")
-        from tree_routed_sparse_b200 import build
-        build.build()
-        run_tree(args)
-        return
-    if args.stages:
-        if not torch.cuda.is_available():
-            raise SystemExit("bench.py needs a CUDA device")
-        from tree_routed_sparse_b200 import build
-        build.build()
-        run_stages(args)
-        return
+        build.build()  # once, before the ranks start
+        argv = sys.argv[1:] if argv is None else list(argv)
+        rc = subprocess.run(torchrun_command(argv, args.gpus, free_port())).returncode
+        raise SystemExit(rc)
 
     dist, rank, world = dist_setup(args.gpus)
     if not torch.cuda.is_available():
@@ -642,10 +775,8 @@ def main():
     barrier(dist)
     line = run_alhr(args, dist, rank, world)
     if rank == 0:
-        if not args.no_cpu_baseline:
-            from tree_routed_sparse_b200 import synth
-            cb = oracle_sample(synth.WORKLOADS[args.workload], args.cpu_sample_stride)
-            line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(args)
         print(json.dumps(line))
     if dist is not None:
         dist.destroy_process_group()

@@ -50,10 +50,18 @@
  *
  * Errors: arguments are checked on the host before anything is launched; on any non-OK
  * status nothing has been launched and no output has been written. A launch failure returns
- * ALHR_ERR_CUDA. Data errors that only the device can see (a budget below 1, a Q or K value
- * outside [-value_bound, value_bound]) never trap: the offending value is clamped (budgets)
- * or used as is (values), and the matching ALHR_DEVERR_* bit is OR-ed into *dev_err when
- * dev_err is non-NULL. Kernels contain no unbounded loop and no spin-wait.
+ * ALHR_ERR_CUDA. Conditions that only the device can see never trap; the kernel handles them
+ * as listed and ORs the matching bit into *dev_err when dev_err is non-NULL:
+ *   ALHR_DEVERR_BUDGET_LOW   a budget below 1 was read: it is treated as 1;
+ *   ALHR_DEVERR_VALUE_RANGE  a Q or K value outside [-value_bound, value_bound]: it is used as
+ *                            is (results stay defined, but narrow tree levels and int32 scores
+ *                            may no longer be exact);
+ *   ALHR_DEVERR_INDEX        alhr_attend: an idx entry outside [0, i] is skipped (weight 0);
+ *   ALHR_DEVERR_TIMEOUT      alhr_topk_labels: a bounded wait on the tensor core ran out; the
+ *                            rows of that CTA's query tile (128 queries) are NOT written, so
+ *                            labels and scores there keep whatever the buffers held before.
+ * Kernels contain no unbounded loop; the only waits (alhr_topk_labels, on its own MMAs) are
+ * bounded.
  */
 #ifndef ALHR_H
 #define ALHR_H
@@ -191,7 +199,9 @@ ALHR_API alhr_status alhr_build_tree(const alhr_dims* dims, const int8_t* K, voi
  *   k       1 <= k <= 16
  *   labels  device int32 [batch][heads][nq][k], written
  *   scores  device int32 [batch][heads][nq][k] or NULL, written
- *   dev_err device uint32 or NULL; ALHR_DEVERR_TIMEOUT if a bounded wait ran out (not expected)
+ *   dev_err device uint32 or NULL; ALHR_DEVERR_TIMEOUT if a bounded wait on the tensor core
+ *           ran out (not expected): the 128-query tile of that CTA is then left unwritten in
+ *           labels and scores, and the caller should treat the whole call's outputs as invalid
  * ALHR_ERR_INVALID_ARG for bad sizes or pointers (Q, K 16-byte aligned).
  */
 ALHR_API alhr_status alhr_topk_labels(const alhr_dims* dims, const int8_t* Q, const int8_t* K,

@@ -50,6 +50,7 @@
 //       all buckets already.
 
 #include <algorithm>
+#include <chrono>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -343,4 +344,23 @@ void oracle_topk_labels(int n, int d, const int8_t* Q, const int8_t* K, int q_st
   }
 }
 
+// Timing harness of the CPU baseline (no arithmetic of its own): the wall time, measured with
+// std::chrono::steady_clock on the calling thread, of oracle_build_tree on one block followed by
+// oracle_forward over the listed query rows of that block (rows NULL: all nq rows). Outputs as
+// oracle_forward; nodes is scratch of [n-1][d] int32. Returns seconds, or -1.0 when a tree sum
+// leaves int32.
+double oracle_time_block(int n, int d, int q_start, int nq, int w, int max_keys,
+                         const int8_t* Q, const int8_t* K, const uint16_t* V, const int8_t* W,
+                         const int32_t* budget_override, const int32_t* rows, int n_rows,
+                         int32_t* nodes, double* out, int32_t* idx, int32_t* count,
+                         int32_t* expansions, int32_t* budget_out) {
+  const auto t0 = std::chrono::steady_clock::now();
+  if (oracle_build_tree(n, d, K, nodes) != 0) return -1.0;
+  oracle_forward(n, d, q_start, nq, w, max_keys, 0, 0, Q, K, V, nodes, W, budget_override, rows,
+                 n_rows, out, idx, count, expansions, budget_out, nullptr);
+  const auto t1 = std::chrono::steady_clock::now();
+  return std::chrono::duration<double>(t1 - t0).count();
+}
+
 }  // extern "C"
+

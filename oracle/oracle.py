@@ -60,6 +60,8 @@ def _configure(L):
     L.oracle_forward.restype = None
     L.oracle_topk_labels.argtypes = [I, I, P, P, I, I, I, P, P]
     L.oracle_topk_labels.restype = None
+    L.oracle_time_block.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, I, P, P, P, P, P, P]
+    L.oracle_time_block.restype = ctypes.c_double
     return L
 
 
@@ -188,3 +190,30 @@ def topk_labels(Q, K, q_start: int, k: int = 16):
     lib().oracle_topk_labels(K.shape[0], d, _p(Q), _p(K), q_start, nq, k, _p(labels),
                              _p(scores))
     return labels, scores
+
+
+def time_block(Q, K, V_bits, W, budget_override, q_start: int, window: int, max_keys: int,
+               rows=None) -> tuple[float, dict]:
+    """Tree build plus the whole path over the listed query rows (None = all) of one (b,h)
+    block, timed inside the oracle library with std::chrono::steady_clock on the calling thread.
+    -> (seconds, outputs as forward() without by_level)."""
+    Q = _c(Q, np.int8)
+    K = _c(K, np.int8)
+    V_bits = _c(V_bits, np.uint16)
+    W = None if W is None else _c(W, np.int8)
+    bo = None if budget_override is None else _c(budget_override, np.int32)
+    nq, d = Q.shape
+    n = K.shape[0]
+    rws = None if rows is None else _c(rows, np.int32)
+    nodes = np.empty((n - 1, d), dtype=np.int32)
+    out = np.zeros((nq, d), dtype=np.float64)
+    idx = np.full((nq, max_keys), -1, dtype=np.int32)
+    count = np.zeros(nq, dtype=np.int32)
+    exp = np.zeros((nq, 2), dtype=np.int32)
+    bud = np.zeros(nq, dtype=np.int32)
+    t = lib().oracle_time_block(n, d, q_start, nq, window, max_keys, _p(Q), _p(K), _p(V_bits),
+                                _p(W), _p(bo), _p(rws), 0 if rws is None else len(rws),
+                                _p(nodes), _p(out), _p(idx), _p(count), _p(exp), _p(bud))
+    if t < 0:
+        raise OverflowError("tree sum outside int32")
+    return float(t), dict(out=out, idx=idx, count=count, expansions=exp, budget=bud)

@@ -58,3 +58,37 @@ def test_recall_planting():
         assert int(p.max()) < 512 and int(u.min()) >= 512
         diff = inp["Q"][b][:, u].to(torch.int16) - inp["K"][b][:, p].to(torch.int16)
         assert int(diff.abs().max()) <= 2
+
+
+def test_block_inputs_are_slices_of_the_batch():
+    wl = synth.WORKLOADS["recall_b2h4_n16384_d128"].replace(n=256, nq=256, plant_pairs=8)
+    full = synth.make_inputs(wl)
+    for lo, hi in [(0, 8), (1, 6), (3, 4), (4, 8), (5, 5)]:
+        part = synth.make_block_inputs(wl, lo, hi)
+        for k in ("Q", "K", "V"):
+            flat = full[k].reshape(-1, *full[k].shape[2:])
+            assert torch.equal(part[k][0], flat[lo:hi]), (lo, hi, k)
+        assert torch.equal(part["W"], full["W"])
+
+
+def test_shards_of_a_global_batch():
+    from tree_routed_sparse_b200 import shard
+    wl = synth.WORKLOADS["prefill_b4h8_n4096"].replace(batch=1, heads=3, n=128, nq=128)
+    g = shard.global_workload(wl, 2)
+    assert g.batch == 2 and g.bh == 6
+    full = synth.make_inputs(g)
+    parts = [shard.shard_inputs(g, 2, r) for r in range(2)]
+    assert [(lo, hi) for lo, hi, _ in parts] == [(0, 3), (3, 6)]
+    for r, (lo, hi, inp) in enumerate(parts):
+        assert inp["Q"].shape == (1, 3, 128, 64)
+        assert torch.equal(inp["K"], full["K"][r:r + 1]) and torch.equal(inp["Q"], full["Q"][r:r + 1])
+    lo, hi, inp = shard.shard_inputs(g, 4, 1)  # blocks [2, 4): not whole sequences
+    assert (lo, hi) == (2, 4) and inp["K"].shape == (1, 2, 128, 64)
+    assert torch.equal(inp["K"][0], full["K"].reshape(6, 128, 64)[2:4])
+
+
+def test_live_classes_zero_the_upper_predictor_rows():
+    wl = synth.WORKLOADS["prefill_b4h8_n4096"].replace(batch=1, heads=1, n=64, nq=64,
+                                                        live_classes=20)
+    W = synth.make_inputs(wl)["W"]
+    assert int(W[20:].abs().max()) == 0 and int(W[:20].abs().max()) > 0

@@ -14,8 +14,9 @@
 // (tcgen05.ld, one TMEM lane per thread) 32 columns at a time, queues the columns that beat its
 // 16th best in shared memory, and inserts the queued ones in deferred rounds into a sorted
 // 16-entry list held in registers. Operand tiles are staged with cp.async in the no-swizzle K-major
-// core-matrix layout (8 rows x 16 bytes per 128-byte core matrix). Every wait on the MMA's mbarrier is bounded; on
-// timeout the CTA stops, sets ALHR_DEVERR_TIMEOUT and still frees its tensor memory.
+// core-matrix layout (8 rows x 16 bytes per 128-byte core matrix). Every wait on the MMA's
+// mbarrier is bounded; on timeout the CTA stops, sets ALHR_DEVERR_TIMEOUT, writes none of its
+// rows, waits (bounded) for the one MMA that can still be in flight and frees its tensor memory.
 #include <climits>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -271,12 +272,14 @@ __global__ void __launch_bounds__(kLThreads, D == 64 ? 4 : 3)
   int* const qbase = queue + tid;  // this thread's queue column
   int* qp = qbase;                 // next free entry
   int epoch = 0;                   // key base of the queued entries
+  int drain_b = -1;                // after an abort: the barrier of the MMA still in flight
+  uint32_t drain_parity = 0u;
   for (int t = 0; t < ntiles; ++t) {
     const int b = t & 1;
+    const uint32_t parity = (phases >> b) & 1u;
     // 1. MMA t done (as this thread sees it): its accumulator is ready, its key buffer free
     bool ok = false;
-    for (uint32_t w = 0; w < kWaitLimit && !ok; ++w)
-      ok = mbar_try_wait(smem_u32(mbar + b), (phases >> b) & 1u);
+    for (uint32_t w = 0; w < kWaitLimit && !ok; ++w) ok = mbar_try_wait(smem_u32(mbar + b), parity);
     phases ^= 1u << b;
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
     // 2. key tile t + 2 into the freed buffer (its own cp.async group)
@@ -297,6 +300,8 @@ __global__ void __launch_bounds__(kLThreads, D == 64 ? 4 : 3)
         *abort_flag = 1;
         if (dev_err) atomicOr(dev_err, ALHR_DEVERR_TIMEOUT);
       }
+      drain_b = b;
+      drain_parity = parity;
       break;
     }
     if (t + 1 < ntiles && tid == 0) issue_mma(t + 1);
@@ -355,6 +360,21 @@ __global__ void __launch_bounds__(kLThreads, D == 64 ? 4 : 3)
     }
   }
   asm volatile("cp.async.wait_all;\n" ::: "memory");  // nothing in flight after an abort
+  if (drain_b >= 0) {
+    // After an abort exactly one committed MMA can still be writing tensor memory: the MMA of
+    // tile t, whose wait ran out. (MMA t + 1 is issued only after the tile's barrier has agreed
+    // that no wait ran out, and the wait of every earlier tile succeeded on every thread, so
+    // their MMAs are complete.) Wait for its commit once more, bounded like every wait, before
+    // the accumulators are freed below; once the commit has been observed nothing targets them.
+    // Should even this wait run out, the tensor core has lost a committed MMA: the memory is
+    // still freed (a CTA must free what it allocated before it exits, and a leaked allocation
+    // would starve the CTAs that come after it on this SM), and ALHR_DEVERR_TIMEOUT, already
+    // set, tells the caller that no output of this launch can be trusted.
+    bool done = false;
+    for (uint32_t w = 0; w < kWaitLimit && !done; ++w)
+      done = mbar_try_wait(smem_u32(mbar + drain_b), drain_parity);
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  }
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
   if (warp == 0)

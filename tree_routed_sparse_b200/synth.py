@@ -91,14 +91,14 @@ def uniform_int8(seed: int, tid: int, shape, lo: int, hi: int, device="cpu",
     return _fill(numel, device, torch.int8, fn).view(*shape)
 
 
-def normal_bf16(seed: int, tid: int, shape, device="cpu") -> torch.Tensor:
+def normal_bf16(seed: int, tid: int, shape, device="cpu", offset: int = 0) -> torch.Tensor:
     """bf16 N(0,1) by Box-Muller in float64 (element k uses stream words 2k and 2k+1),
-    rounded to nearest even."""
+    rounded to nearest even. `offset` is the flat index of the first element."""
     numel = math.prod(shape)
     two53 = float(1 << 53)
 
     def fn(s, c):
-        x = raw_words(seed, tid, 2 * s, 2 * c, device).view(c, 2)
+        x = raw_words(seed, tid, 2 * (offset + s), 2 * c, device).view(c, 2)
         u1 = (_lsr(x[:, 0], 11).to(torch.float64) + 0.5) / two53
         u2 = _lsr(x[:, 1], 11).to(torch.float64) / two53
         z = torch.sqrt(-2.0 * torch.log(u1)) * torch.cos(2.0 * math.pi * u2)
@@ -128,6 +128,7 @@ class Workload:
     plant_pairs: int = 0          # associative-recall planting per sequence
     plant_noise: int = 2
     seed: int = 0
+    live_classes: int = 32        # predictor rows of classes >= live_classes are zero
 
     @property
     def bh(self) -> int:
@@ -175,30 +176,62 @@ def plant_positions(wl: Workload, b: int, device="cpu"):
     return p, u
 
 
+def make_block_inputs(wl: Workload, lo: int, hi: int, device="cpu") -> dict:
+    """The inputs of the flat (b,h) blocks [lo, hi) of a workload (block k = b * heads + h), with
+    the same bits as the same blocks of make_inputs(wl): every element is drawn at its flat
+    index in the whole batch, so a rank of a sharded run generates its own blocks only.
+
+    Q int8 [1, hi-lo, nq, d], K int8 [1, hi-lo, n, d], V bf16 [1, hi-lo, n, d] (reshaped to
+    [sequences, heads, ...] by the caller where the range is whole sequences), W int8 [32, 2d]
+    (or None), budget_override int32 [1, hi-lo, nq] (or None)."""
+    if not 0 <= lo <= hi <= wl.bh:
+        raise ValueError(f"blocks [{lo}, {hi}) outside [0, {wl.bh})")
+    H, n, d, nb = wl.heads, wl.n, wl.d, hi - lo
+    K = uniform_int8(wl.seed, TID_K, (1, nb, n, d), wl.qk_lo, wl.qk_hi, device,
+                     offset=lo * n * d)
+    Q = uniform_int8(wl.seed, TID_Q, (1, nb, wl.nq, d), wl.qk_lo, wl.qk_hi, device,
+                     offset=lo * wl.nq * d)
+    V = normal_bf16(wl.seed, TID_V, (1, nb, n, d), device, offset=lo * n * d)
+    if wl.plant_pairs and nb:
+        assert wl.q_start == 0 and wl.nq == n
+        P = wl.plant_pairs
+        for b in range(lo // H, (hi - 1) // H + 1):
+            p, u = plant_positions(wl, b, device)
+            h0, h1 = max(lo, b * H) - b * H, min(hi, (b + 1) * H) - b * H
+            # planting noise: one stream slice per sequence, [heads, pairs, d]
+            noise = uniform_int8(wl.seed, TID_NOISE, (h1 - h0, P, d), -wl.plant_noise,
+                                 wl.plant_noise, device, offset=(b * H + h0) * P * d)
+            k0 = b * H + h0 - lo
+            planted = K[0, k0:k0 + h1 - h0][:, p, :].to(torch.int16) + noise.to(torch.int16)
+            Qs = Q[0, k0:k0 + h1 - h0]  # a view: [heads of this range, nq, d]
+            Qs[:, u, :] = planted.clamp(wl.qk_lo, wl.qk_hi).to(torch.int8)
+    W = None
+    budget = None
+    if wl.predictor:
+        W = uniform_int8(wl.seed, TID_W, (32, 2 * d), wl.w_lo, wl.w_hi, device)
+        if wl.live_classes < 32:
+            W[wl.live_classes:] = 0
+    else:
+        pos = torch.arange(wl.q_start, wl.q_start + wl.nq, dtype=torch.int32, device=device)
+        budget = torch.clamp(pos + 1, max=wl.fixed_budget_cap).expand(1, nb, wl.nq).contiguous()
+    return dict(Q=Q, K=K, V=V, W=W, budget_override=budget)
+
+
+def as_sequences(inp: dict, heads: int) -> dict:
+    """Block inputs [1, k*heads, ...] viewed as [k, heads, ...] (whole sequences)."""
+    out = {}
+    for key, t in inp.items():
+        if t is None or key == "W":
+            out[key] = t
+        else:
+            assert t.shape[1] % heads == 0
+            out[key] = t.view(t.shape[1] // heads, heads, *t.shape[2:])
+    return out
+
+
 def make_inputs(wl: Workload, device="cpu") -> dict:
     """All inputs of a workload as torch tensors on `device`.
 
     Q int8 [B,H,nq,d], K int8 [B,H,n,d], V bf16 [B,H,n,d], W int8 [32,2d] (or None),
     budget_override int32 [B,H,nq] (or None)."""
-    B, H, n, d = wl.batch, wl.heads, wl.n, wl.d
-    K = uniform_int8(wl.seed, TID_K, (B, H, n, d), wl.qk_lo, wl.qk_hi, device)
-    Q = uniform_int8(wl.seed, TID_Q, (B, H, wl.nq, d), wl.qk_lo, wl.qk_hi, device)
-    V = normal_bf16(wl.seed, TID_V, (B, H, n, d), device)
-    if wl.plant_pairs:
-        assert wl.q_start == 0 and wl.nq == n
-        P = wl.plant_pairs
-        for b in range(B):
-            p, u = plant_positions(wl, b, device)
-            noise = uniform_int8(wl.seed, TID_NOISE, (H, P, d), -wl.plant_noise,
-                                 wl.plant_noise, device, offset=b * H * P * d)
-            planted = (K[b][:, p, :].to(torch.int16) + noise.to(torch.int16))
-            planted = planted.clamp(wl.qk_lo, wl.qk_hi).to(torch.int8)
-            Q[b][:, u, :] = planted
-    W = None
-    budget = None
-    if wl.predictor:
-        W = uniform_int8(wl.seed, TID_W, (32, 2 * d), wl.w_lo, wl.w_hi, device)
-    else:
-        pos = torch.arange(wl.q_start, wl.q_start + wl.nq, dtype=torch.int32, device=device)
-        budget = torch.clamp(pos + 1, max=wl.fixed_budget_cap).expand(B, H, wl.nq).contiguous()
-    return dict(Q=Q, K=K, V=V, W=W, budget_override=budget)
+    return as_sequences(make_block_inputs(wl, 0, wl.bh, device), wl.heads)
