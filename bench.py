@@ -267,13 +267,30 @@ def oracle_single_thread(wl, inp) -> dict:
 
 # ------------------------------------------------------------------ the GPU arm
 
-def fwd_algorithmic_bytes(wl, full, vb) -> int:
+# resident CTAs per SM of the latency shape (one query per CTA); launches of at most this many
+# queries per SM take it under the automatic launch mode, larger ones the warp-per-query shape
+LAT_CTAS_PER_SM = 4
+
+
+def takes_warp_shape(queries: int, dev) -> bool:
+    return queries > torch.cuda.get_device_properties(dev).multi_processor_count * LAT_CTAS_PER_SM
+
+
+def fwd_algorithmic_bytes(wl, full, vb, warp_shape: bool = True) -> tuple[int, int]:
+    """(algorithmic bytes, bytes of the rows the kernel reads) of one fused-forward launch. The
+    first is the byte model as the method defines it (G_i from the forest roots and the window
+    keys); the second differs only where the warp-per-query kernel at d = 64 forms G_i from the
+    blocks of [0, i+1) instead."""
     from tree_routed_sparse_b200 import metrics
     pos = np.broadcast_to(np.arange(wl.q_start, wl.q_start + wl.nq),
                           (full["count"].shape[0] * full["count"].shape[1], wl.nq))
-    return metrics.forward_bytes(pos, wl.n, wl.d, wl.window, full["count"].cpu().numpy(),
-                                 full["expansions"].cpu().numpy(), full["budget"].cpu().numpy(),
-                                 wl.predictor, wl.max_keys, value_bound=vb)
+    args = (pos, wl.n, wl.d, wl.window, full["count"].cpu().numpy(),
+            full["expansions"].cpu().numpy(), full["budget"].cpu().numpy(), wl.predictor,
+            wl.max_keys)
+    plain = metrics.forward_bytes(*args, value_bound=vb)
+    kernel = metrics.forward_bytes(*args, value_bound=vb,
+                                   g_from_blocks=warp_shape and wl.d == 64)
+    return plain, kernel
 
 
 def run_alhr(args, dist, rank, world):
@@ -299,7 +316,8 @@ def run_alhr(args, dist, rank, world):
     full = alhr.forward(Q, K, V, tree, W=W, budget_override=bo, want_count=True,
                         want_expansions=True, want_budget=True, **kw)
     torch.cuda.synchronize()
-    fwd_bytes = fwd_algorithmic_bytes(wl, full, vb)
+    warp_shape = takes_warp_shape(wl.bh * wl.nq, dev)
+    fwd_bytes, fwd_kernel_bytes = fwd_algorithmic_bytes(wl, full, vb, warp_shape)
     tree_bytes = metrics.tree_bytes(wl.bh, wl.n, wl.d, vb)
     mean_keys = float(full["count"].float().mean())
     mean_budget = float(full["budget"].float().mean())
@@ -376,7 +394,7 @@ def run_alhr(args, dist, rank, world):
         full = alhr.forward(Q, K, V, tree, W=W_op, want_count=True, want_expansions=True,
                             want_budget=True, **kw)
         torch.cuda.synchronize()
-        op_bytes = fwd_algorithmic_bytes(wl_op, full, vb)
+        op_bytes, op_kernel_bytes = fwd_algorithmic_bytes(wl_op, full, vb, warp_shape)
         op_keys = float(full["count"].float().mean())
         del full
         for _ in range(3):
@@ -395,7 +413,8 @@ def run_alhr(args, dist, rank, world):
         op = {"workload": describe(wl_op), "mean_keys_per_query": op_keys,
               "pages_keys_per_token": "30.0 / 32.0 / 30.0 at T = 1K / 4K / 16K (README TLDR)",
               "queries_per_s": world * queries * args.op_steps / t_op,
-              "launch_ms": t_op / args.op_steps * 1e3, "algorithmic_bytes_per_launch": op_bytes}
+              "launch_ms": t_op / args.op_steps * 1e3, "algorithmic_bytes_per_launch": op_bytes,
+              "kernel_row_bytes_per_launch": op_kernel_bytes}
 
     if rank != 0:
         return None
@@ -444,13 +463,16 @@ def run_alhr(args, dist, rank, world):
             "frac": achieved / peak,
             "peak_source": f"{peak_src} hbm_gbs",
             "algorithmic_bytes_per_launch": fwd_bytes,
+            "kernel_row_bytes_per_launch": fwd_kernel_bytes,
             "launch_ms": fwd_launch_s * 1e3,
             "traffic": traffic,
             "dram": dram_rate(traffic, fwd_launch_s, peak),
             "issue": issue_rate(rec, fwd_launch_s),
             "binding_resource": "instruction issue (see issue.frac); DRAM is not the limit",
-            "note": ("achieved counts every row the path reads (the algorithmic bytes of the "
-                     "metric) as if it came from DRAM; queries run in (b, h, i) order, so the "
+            "note": ("achieved counts every row the method reads (the algorithmic bytes: G_i from "
+                     "the forest roots and the window keys) as if it came from DRAM; "
+                     "kernel_row_bytes are the rows the kernel reads (at d = 64 it forms G_i from "
+                     "the blocks of [0, i+1), a few more rows); queries run in (b, h, i) order, so the "
                      "rows in use at any time (about one head's tree, keys and values) stay in "
                      "L2 and repeat reads are served there: achieved is a rate of row reads and "
                      "can exceed the DRAM peak. dram is the DRAM traffic ncu measured "
@@ -571,10 +593,7 @@ def run_stages(args):
             lambda: alhr.forward(Q, K, V, tree, W=W, budget_override=bo, out=out, **kw), reps, flush)
         full = alhr.forward(Q, K, V, tree, W=W, budget_override=bo, want_count=True,
                             want_expansions=True, want_budget=True, **kw)
-        pos = np.broadcast_to(np.arange(wl.q_start, wl.q_start + wl.nq), (wl.bh, wl.nq))
-        fb = metrics.forward_bytes(pos, wl.n, wl.d, wl.window, full["count"].cpu().numpy(),
-                                   full["expansions"].cpu().numpy(), full["budget"].cpu().numpy(),
-                                   wl.predictor, wl.max_keys, value_bound=vb)
+        fb, _ = fwd_algorithmic_bytes(wl, full, vb)
         keys = float(count.float().mean())
         del inp, tree, out, idx, count, budget, full
         torch.cuda.empty_cache()

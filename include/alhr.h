@@ -245,6 +245,24 @@ ALHR_API alhr_status alhr_tree_unpack(const alhr_dims* dims, const void* tree, i
                                       void* stream);
 
 /*
+ * alhr_tree_pack -- the inverse of alhr_tree_unpack: plain level-major int32 node rows (the
+ * nodes[b][h][r][:] layout above; node(l, j) = sum of keys [j*2^l, (j+1)*2^l)) written into the
+ * tree layout that alhr_predict_budget, alhr_route and alhr_forward read, for callers that
+ * build or keep the key tree as int32 rows themselves [README opening paragraph: every branch
+ * is indexed by the sum of the key vectors beneath it]. Reads dims->batch, heads, n, d and
+ * value_bound.
+ *   nodes   device, int32 [batch][heads][n-1][d], 16-byte aligned, read only
+ *   tree    device, 32-byte aligned, batch*heads*alhr_tree_bytes(n, d, value_bound) bytes,
+ *           fully overwritten
+ *   dev_err device uint32 or NULL; ALHR_DEVERR_VALUE_RANGE if a value of a narrow (int16)
+ *           level l lies outside [-value_bound * 2^l, value_bound * 2^l] (it cannot then be a
+ *           sum of keys within the bound; it is stored saturated to int16)
+ * alhr_tree_pack(alhr_tree_unpack(tree)) == tree for every tree alhr_build_tree wrote.
+ */
+ALHR_API alhr_status alhr_tree_pack(const alhr_dims* dims, const int32_t* nodes, void* tree,
+                                    uint32_t* dev_err, void* stream);
+
+/*
  * alhr_predict_budget -- the budget predictor [README §Inference stage, second paragraph: a
  * trainable function of the current query and the global key sum that outputs a leaf group,
  * i.e. the number of keys the query asks for; §Results and Variables: 32 classes, <= 96 keys].

@@ -168,6 +168,10 @@ def test_entry_points_reject_bad_arguments_before_launch(A):
     assert L.alhr_build_tree(d, fake, odd32, null, null) == 1
     assert L.alhr_update_tree(d, fake, odd32, 0, 1, null, null) == 1
     assert L.alhr_tree_unpack(d, odd32, fake, null) == 1
+    assert L.alhr_tree_pack(d, fake, odd32, null, null) == 1
+    assert L.alhr_tree_pack(d, odd, fake, null, null) == 1
+    assert L.alhr_tree_pack(d, null, fake, null, null) == 1
+    assert L.alhr_tree_pack(ctypes.byref(_dims(A, d=32)), fake, fake, null, null) == 2
     assert L.alhr_forward(d, fake, fake, fake, odd32, fake, null, fake, null, null, null, null,
                           null, null) == 1
     assert L.alhr_route(d, fake, fake, odd32, fake, fake, fake, null, null, null) == 1

@@ -15,10 +15,10 @@ def test_hand_counted_query_without_predictor():
 
 
 def test_hand_counted_query_with_predictor():
-    # causal sum: [0,8) is one block, the root row (8); the roots of [0,6) differ from it
-    # (i+1 = 8 and i-w+1 = 6 differ at bit 3), so both are read + W once (64*2)
+    # the causal sum is formed from the roots of [0,6) and the window keys, which the query
+    # reads anyway (same 64 bytes as without the predictor) + W once (64*2)
     assert metrics.forward_bytes([7], 8, 2, 2, [5], [[1, 3, 1]], [5], predictor=True) == \
-        64 + 8 + 128
+        64 + 128
 
 
 def test_narrow_rows_at_d128():
@@ -38,15 +38,32 @@ def test_no_descent_reads_no_roots():
         2 + 2 * 2 + 2 * 4 + 8
 
 
-def test_shared_blocks_counted_once():
+def test_predictor_reads_every_root_and_window_key():
+    # i = 20, w = 2, budget 1: no descent and one selected key, but the causal sum G_i still
+    # needs every root of [0, 19) (19 = 10011b: levels 4, 1, 0) and both window keys
+    d = 2
+    got = metrics.forward_bytes([20], 32, d, 2, [1], [[0, 0, 0]], [1], predictor=True)
+    roots = 4 * d + 4 * d + d
+    assert got == d + roots + 2 * d + 1 * 2 * d + 4 * d + 64 * d
+    # without the predictor the same query reads neither the roots nor the unselected key
+    assert metrics.forward_bytes([20], 32, d, 2, [1], [[0, 0, 0]], [1], predictor=False) == \
+        d + d + 2 * d + 4 * d
+
+
+def test_g_from_blocks_counts_the_blocks_of_the_prefix():
     # i = 20, w = 2: i+1 = 21 = 10101b, i-w+1 = 19 = 10011b differ first at bit 2, so the
     # level-4 block [0,16) is read once for both; G needs bits 2 and 0 of 21 (a level-2 row, a
-    # key), the descent also bits 1 and 0 of 19 (a level-1 row and a key)
+    # key), the descent also bits 1 and 0 of 19 (a level-1 row and a key); only the selected
+    # window keys are read
     d = 2
-    got = metrics.forward_bytes([20], 32, d, 2, [3], [[0, 0, 0]], [3], predictor=True)
+    got = metrics.forward_bytes([20], 32, d, 2, [3], [[0, 0, 0]], [3], predictor=True,
+                                g_from_blocks=True)
     g_rows = 4 * d + 4 * d + d          # [0,16), [16,20), [20,21)
     roots_rest = 4 * d + d              # [16,18), [18,19)
     assert got == d + g_rows + roots_rest + 2 * d + 3 * 2 * d + 4 * d + 64 * d
+    # the survey's count of the same query: the roots of [0,19) and both window keys
+    plain = metrics.forward_bytes([20], 32, d, 2, [3], [[0, 0, 0]], [3], predictor=True)
+    assert plain == d + (4 * d + 4 * d + d) + 2 * d + 3 * 2 * d + 4 * d + 64 * d
 
 
 @pytest.mark.parametrize("n,d,vb", [(16384, 64, 16), (16384, 128, 16), (262144, 128, 16),

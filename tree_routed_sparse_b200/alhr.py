@@ -29,7 +29,7 @@ EXPORTS = ["alhr_tree_rows", "alhr_tree_narrow_levels", "alhr_tree_bytes",
            "alhr_tree_level_offset", "alhr_score_bits", "alhr_status_string", "alhr_build_info",
            "alhr_build_tree", "alhr_update_tree", "alhr_tree_unpack", "alhr_predict_budget",
            "alhr_route", "alhr_attend", "alhr_forward", "alhr_set_launch_mode",
-           "alhr_get_launch_mode", "alhr_topk_labels"]
+           "alhr_get_launch_mode", "alhr_topk_labels", "alhr_tree_pack"]
 
 
 class AlhrError(RuntimeError):
@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
         L.alhr_build_tree.argtypes = [DP, P, P, P, P]
         L.alhr_update_tree.argtypes = [DP, P, P, I32, I32, P, P]
         L.alhr_tree_unpack.argtypes = [DP, P, P, P]
+        L.alhr_tree_pack.argtypes = [DP, P, P, P, P]
         L.alhr_predict_budget.argtypes = [DP, P, P, P, P, P, P, P]
         L.alhr_route.argtypes = [DP, P, P, P, P, P, P, P, P, P]
         L.alhr_attend.argtypes = [DP, P, P, P, P, P, P, P, P]
@@ -76,7 +77,7 @@ def lib() -> ctypes.CDLL:
         L.alhr_topk_labels.argtypes = [DP, P, P, I32, P, P, P, P]
         L.alhr_set_launch_mode.argtypes = [I32]
         L.alhr_get_launch_mode.argtypes, L.alhr_get_launch_mode.restype = [], I32
-        for f in ("alhr_build_tree", "alhr_update_tree", "alhr_tree_unpack",
+        for f in ("alhr_build_tree", "alhr_update_tree", "alhr_tree_unpack", "alhr_tree_pack",
                   "alhr_predict_budget", "alhr_route", "alhr_attend", "alhr_forward",
                   "alhr_set_launch_mode", "alhr_topk_labels"):
             getattr(L, f).restype = I32
@@ -184,6 +185,22 @@ def tree_unpack(tree: torch.Tensor, n: int, d: int, value_bound: int = 16) -> to
     _check(lib().alhr_tree_unpack(ctypes.byref(dims), _ptr(tree), _ptr(nodes),
                                   _stream(tree.device)), "alhr_tree_unpack")
     return nodes
+
+
+def tree_pack(nodes: torch.Tensor, value_bound: int = 16, tree: torch.Tensor | None = None,
+              dev_err: torch.Tensor | None = None) -> torch.Tensor:
+    """Plain level-major int32 rows [B,H,n-1,d] into the tree layout (alhr_tree_pack)."""
+    B, H, rows, d = nodes.shape
+    n = rows + 1
+    _want(nodes, torch.int32, (B, H, rows, d), "nodes")
+    tb = tree_bytes(n, d, value_bound)
+    if tree is None:
+        tree = torch.empty((B, H, tb), dtype=torch.uint8, device=nodes.device)
+    _want(tree, torch.uint8, (B, H, tb), "tree")
+    dims = Dims(B, H, n, d, 0, 0, 16, 96, 0, value_bound)
+    _check(lib().alhr_tree_pack(ctypes.byref(dims), _ptr(nodes), _ptr(tree), _ptr(dev_err),
+                                _stream(nodes.device)), "alhr_tree_pack")
+    return tree
 
 
 def predict_budget(Q, K, tree, W, q_start=0, window=16, max_keys=96, score_bits=0,

@@ -194,6 +194,18 @@ alhr_status alhr_tree_unpack(const alhr_dims* dims, const void* tree, int32_t* n
                                             static_cast<cudaStream_t>(stream)));
 }
 
+alhr_status alhr_tree_pack(const alhr_dims* dims, const int32_t* nodes, void* tree,
+                           uint32_t* dev_err, void* stream) {
+  const alhr_status s = check_common(dims);
+  if (s != ALHR_OK) return s;
+  if (!tree || !nodes || !aligned32(tree) || !aligned16(nodes)) return ALHR_ERR_INVALID_ARG;
+  const long long bh = (long long)dims->batch * dims->heads;
+  const alhr::TreeLayout tl = alhr::make_tree_layout(dims->n, dims->d, dims->value_bound);
+  return from_cuda(alhr::launch_tree_pack(nodes, tl, bh, value_bound_of(dims),
+                                          static_cast<char*>(tree), dev_err,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 alhr_status alhr_predict_budget(const alhr_dims* dims, const int8_t* Q, const int8_t* K,
                                 const void* tree, const int8_t* W, int32_t* budget,
                                 uint32_t* dev_err, void* stream) {

@@ -21,6 +21,7 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kMaxKeys = 96;        // 32 budget classes x 3 keys
 constexpr int kMaxFrontier = 96;    // r <= max_keys - 1 nodes survive a step
 constexpr int kMaxCand = 192;       // a step offers at most 2 r candidates
+constexpr int kMaxWindow = 32;      // the largest neighbour window the kernels accept
 constexpr int kFrontSlots = kMaxFrontier / 32;
 constexpr int kWarps = 8;           // queries in flight per CTA
 
@@ -32,9 +33,6 @@ struct Lay {
 };
 
 // Node descriptor: (start << 5) | level; the node covers keys [start, start + 2^level).
-// Bits 29 and 30 are free (start < 2^20) and carry flags in the phase-one row list.
-constexpr int kFlagRoot = 1 << 29;  // the row is a root of the descent forest
-constexpr int kFlagG = 1 << 30;     // the row is a block of the causal sum G_i
 __device__ __forceinline__ int desc_level(int desc) { return desc & 31; }
 __device__ __forceinline__ int desc_start(int desc) { return (desc >> 5) & 0xFFFFF; }
 __device__ __forceinline__ int make_desc(int start, int level) { return (start << 5) | level; }
@@ -440,9 +438,12 @@ struct WarpBuf {
   S xleft[kMaxFrontier];     // score of that left child
   int selk[kMaxKeys];        // the selected keys and their softmax weights
   float selp[kMaxKeys];
-  int plist[32];             // phase-one row list (causal-sum blocks and roots)
-  int winsc[32];             // scores of the window keys
+  int plist[32];             // the roots of the descent forest, largest first
+  int winsc[kMaxWindow + 4]; // scores of the window keys (+ a spare slot for idle row groups;
+                             // padded so that the buffer stays a multiple of 16 bytes)
 };
+static_assert(sizeof(WarpBuf<int>) % 16 == 0 && sizeof(WarpBuf<long long>) % 16 == 0,
+              "per-warp buffers keep 16-byte alignment");
 
 // ------------------------------------------------------------------ top-r selection
 

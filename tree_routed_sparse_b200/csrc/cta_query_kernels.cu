@@ -1,0 +1,579 @@
+// cta_query_kernels.cu -- CTA-per-query kernels of the ALHR inference path (sm_100a): the
+// latency shape, for launches too small to fill the GPU with one warp per query (decode).
+//
+// Same computation as the warp-per-query kernels of query_kernels.cu (README of ALHR, section
+// "Inference stage": causal key sum and budget predictor, own key and neighbour window, descent
+// of the past-only forest, exact attention), with one query per CTA of kCtaWarps warps. A query
+// at decode time is a chain of about log2 n dependent descent steps, so its latency is what
+// counts: the row work of every phase is spread over the CTA's kCtaWarps * RPI row groups (the
+// roots and window keys of the causal sum, a step's left-child rows, the value rows), so that a
+// step's rows take one round trip to memory and are scored in parallel, while warp 0 alone runs
+// the short serial parts on the shared buffers (classifying the frontier, writing the children,
+// the top-r selection). Two CTA barriers per descent step order the two.
+#include <cstddef>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "query_common.cuh"
+
+namespace alhr {
+
+constexpr int kCtaWarps = 4;
+
+// Shared state of one query: the warp-per-query buffer (used here by the whole CTA) plus the
+// cross-warp partial sums and the counts warp 0 hands to the others.
+template <typename S, int D>
+struct CtaBuf {
+  WarpBuf<S> B;
+  long long logit[32];                    // class logits of the predictor
+  alignas(16) int gpart[kCtaWarps][D];    // per-warp partial sums of G_i (lane-slot order:
+                                          // sub * 16 + j), read and written as int4
+  alignas(16) float opart[kCtaWarps][D];  // per-warp partial sums of the output row (float4)
+  int ctl[8];                             // counts of a descent step (wide, narrow, key, leaf, nf)
+  float inv;                              // 1 / softmax denominator
+};
+// the 16-byte accesses above need 16-byte offsets
+using CtaBufI64 = CtaBuf<int, 64>;
+using CtaBufL128 = CtaBuf<long long, 128>;
+static_assert(offsetof(CtaBufI64, gpart) % 16 == 0 && offsetof(CtaBufI64, opart) % 16 == 0,
+              "CtaBuf alignment");
+static_assert(offsetof(CtaBufL128, gpart) % 16 == 0 && offsetof(CtaBufL128, opart) % 16 == 0,
+              "CtaBuf alignment");
+
+template <typename S, int D, int MODE>
+struct CtaSmem {
+  static_assert(QuerySmem<S, D, MODE>::w_bytes % 16 == 0, "CtaBuf placement");
+  static constexpr size_t bytes = QuerySmem<S, D, MODE>::w_bytes + sizeof(CtaBuf<S, D>);
+};
+
+// One pass over CTA-wide positions [base, end) of the expanded-node lists: row group gg takes
+// positions base + gg + u * NG (u < US), loads them all, then scores them. KIND 0: int32 tree
+// rows, 1: int16 tree rows, 2: key rows. A warp without positions in the pass skips it.
+template <int KIND, int US, typename S, int D>
+__device__ __forceinline__ void cta_child_pass(WarpBuf<S>& B, const char* Th, const int8_t* Kh,
+                                               const RowQ& q, int base, int end, int warp,
+                                               int gg, int sub) {
+  constexpr int RPI = Lay<D>::RPI;
+  constexpr int TPR = Lay<D>::TPR;
+  constexpr int NG = kCtaWarps * RPI;
+  if (base + warp * RPI >= end) return;  // warp-uniform
+  constexpr int WORDS = KIND == 0 ? 16 : (KIND == 1 ? 8 : 4);
+  int x[US][WORDS];
+#pragma unroll
+  for (int u = 0; u < US; ++u) {
+    const int xi = base + u * NG + gg;
+    if (xi < end) {
+      if constexpr (KIND == 0) ld_tree<D>(Th + B.xrow[xi], sub, x[u]);
+      else if constexpr (KIND == 1) ld_tree16<D>(Th + B.xrow[xi], sub, x[u]);
+      else ld_key<D>(Kh + B.xrow[xi], sub, x[u]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < WORDS; ++j) x[u][j] = 0;
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int u = 0; u < US; ++u) {
+    const int xi = base + u * NG + gg;
+    S left;
+    if constexpr (KIND == 0) left = group_sum<S, TPR>(dot_tree<S>(q, x[u]));
+    else if constexpr (KIND == 1) left = S(group_sum<int, TPR>(dot_tree16(q, x[u])));
+    else left = S(group_sum<int, TPR>(dot_key(q, x[u])));
+    if (xi < end && sub == 0) B.xleft[xi] = left;
+  }
+}
+
+// The value rows of keys [k0, k1) of the staged selection, weighted, summed over the warp's
+// value groups; the warp's partial output row goes to part[0 .. D).
+template <int D, int UV>
+__device__ __forceinline__ void gather_values_part(const int* selk, const float* selp, int k0,
+                                                   int k1, const uint16_t* Vh, int lane,
+                                                   float* part) {
+  constexpr int VPR = D / 8;
+  constexpr int KPP = 32 / VPR;
+  const int kg = lane / VPR;
+  const int vs = lane % VPR;
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  for (int base = k0; base < k1; base += UV * KPP) {
+    uint4 raw[UV];
+    float p[UV];
+#pragma unroll
+    for (int u = 0; u < UV; ++u) {
+      const int k = base + u * KPP + kg;
+      if (k < k1) {
+        raw[u] = __ldg(reinterpret_cast<const uint4*>(Vh + (long long)selk[k] * D) + vs);
+        p[u] = selp[k];
+      } else {
+        raw[u] = make_uint4(0u, 0u, 0u, 0u);
+        p[u] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UV; ++u) {
+      const unsigned w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc[2 * j] = fmaf(p[u], __uint_as_float(w[j] << 16), acc[2 * j]);
+        acc[2 * j + 1] = fmaf(p[u], __uint_as_float(w[j] & 0xffff0000u), acc[2 * j + 1]);
+      }
+    }
+  }
+#pragma unroll
+  for (int off = VPR; off < 32; off *= 2)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] += __shfl_xor_sync(kFull, acc[j], off);
+  if (lane < VPR) {
+    float4* o = reinterpret_cast<float4*>(part + 8 * vs);
+    o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+}
+
+// VAR compiles in the descent variants (ranking by means, leaf buckets), as in query_kernel.
+template <typename S, int D, int MODE, bool VAR>
+__global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const QueryArgs a) {
+  constexpr int TPR = Lay<D>::TPR;
+  constexpr int RPI = Lay<D>::RPI;
+  constexpr int NG = kCtaWarps * RPI;  // row groups of the CTA
+  constexpr bool kUsesW = (MODE == kForwardPredict || MODE == kPredictOnly);
+  constexpr bool kDescend = (MODE != kPredictOnly);
+  constexpr bool kAttend = (MODE == kForwardPredict || MODE == kForwardOverride);
+  constexpr bool kNarrow = (D == 128);
+  // rows per group and pass: int32 tree rows, int16 tree rows, key rows (a step expands at most
+  // kMaxFrontier - 1 nodes: one pass of each kind covers NG * U of them)
+  constexpr int UW = D == 128 ? 3 : 3;
+  constexpr int UN = 6;
+  constexpr int UK = D == 128 ? 6 : 3;
+
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  int* sWg = reinterpret_cast<int*>(smem_raw);
+  int* sWq = sWg + 32 * WLayout<D>::g_stride;
+  CtaBuf<S, D>& C = *reinterpret_cast<CtaBuf<S, D>*>(smem_raw + QuerySmem<S, D, MODE>::w_bytes);
+  WarpBuf<S>& B = C.B;
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int grp = lane / TPR;
+  const int sub = lane % TPR;
+  const int gg = warp * RPI + grp;  // this lane's row group in the CTA
+  if constexpr (kUsesW) stage_weights<D>(a.W, sWg, sWq);
+  const int n = a.n;
+  const int w = a.window;
+  const long long tree_block = a.tl.block_bytes;
+  const int narrow = kNarrow ? a.tl.narrow : 0;
+  const int bucket = VAR ? a.bucket : 0;
+  const int norm_l = VAR ? a.norm_l : 0;
+
+  for (long long qi = blockIdx.x; qi < a.num_queries; qi += gridDim.x) {
+    __syncthreads();  // the weights are staged; the previous query is done with the buffers
+    const long long bh = qi / a.nq;
+    const int i = a.q_start + int(qi - bh * a.nq);
+    const int8_t* Kh = a.K + bh * (long long)n * D;
+    const char* Th = a.tree + bh * tree_block;
+
+    RowQ q;
+    load_rowq<D>(a.Q + qi * D, sub, q);
+    if (warp == 0) {
+      bool bad = false;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) bad |= (q.qn[j] > a.value_bound) | (q.qn[j] < -a.value_bound);
+      if (__any_sync(kFull, bad) && lane == 0) flag(a.dev_err, ALHR_DEVERR_VALUE_RANGE);
+    }
+
+    const int nwin = min(w, i + 1);
+    const int M = i - w + 1;
+    const unsigned Mu = M > 0 ? unsigned(M) : 0u;
+    const int nR = __popc(Mu);
+
+    int budget = 0, b_eff = 0, nsel_win = 0, r = 0;
+    auto settle = [&](int bud) {
+      if (bud < 1) {
+        if (threadIdx.x == 0) flag(a.dev_err, ALHR_DEVERR_BUDGET_LOW);
+        bud = 1;
+      }
+      budget = bud;
+      b_eff = min(min(bud, i + 1), a.max_keys);
+      nsel_win = min(b_eff, nwin);
+      r = b_eff - nsel_win;
+    };
+    if constexpr (!kUsesW) settle(__ldg(a.budget_in + qi));
+
+    if (warp == 0 && ((Mu >> lane) & 1u))
+      B.plist[__popc(Mu >> lane) - 1] = make_desc(int((Mu >> lane) << lane) - (1 << lane), lane);
+    __syncthreads();
+
+    // ---- 1. causal sum G_i = (roots of [0, i-w]) + (window keys), scored in the same pass
+    if constexpr (kUsesW) {
+      constexpr int U1 = (kMaxLevels + kMaxWindow + NG - 1) / NG;
+      const int nI = nR + nwin;
+      int G[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) G[j] = 0;
+      S rsc[U1];
+      {
+        int x[U1][16];
+#pragma unroll
+        for (int u = 0; u < U1; ++u) {
+          const int k = u * NG + gg;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) x[u][j] = 0;
+          if (k < nI)
+            ld_node32<D, kNarrow>(Th, Kh, n, narrow,
+                                  k < nR ? B.plist[k] : make_desc(i - (k - nR), 0), sub, x[u]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < U1; ++u) {
+          rsc[u] = S(0);
+          if (u * NG < nI) {  // CTA-uniform
+#pragma unroll
+            for (int j = 0; j < 16; ++j) G[j] += x[u][j];
+            rsc[u] = group_sum<S, TPR>(dot_tree<S>(q, x[u]));
+          }
+        }
+      }
+#pragma unroll
+      for (int off = TPR; off < 32; off *= 2)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) G[j] += __shfl_xor_sync(kFull, G[j], off);
+      if (grp == 0) {
+        int4* gp = reinterpret_cast<int4*>(&C.gpart[warp][sub * 16]);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) gp[v] = make_int4(G[4 * v], G[4 * v + 1], G[4 * v + 2], G[4 * v + 3]);
+      }
+#pragma unroll
+      for (int u = 0; u < U1; ++u) {
+        const int k = u * NG + gg;
+        if (k < nI && sub == 0) {
+          if (k < nR) B.cand.put(k, B.plist[k], rsc[u]);
+          else B.winsc[k - nR] = int(rsc[u]);
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) G[j] = 0;
+#pragma unroll
+      for (int ww = 0; ww < kCtaWarps; ++ww) {
+        const int4* gp = reinterpret_cast<const int4*>(&C.gpart[ww][sub * 16]);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int4 t = gp[v];
+          G[4 * v] += t.x;
+          G[4 * v + 1] += t.y;
+          G[4 * v + 2] += t.z;
+          G[4 * v + 3] += t.w;
+        }
+      }
+      // ---- 2. budget predictor: the CTA's row groups take the 32 classes
+#pragma unroll
+      for (int kk = 0; kk < (32 + NG - 1) / NG; ++kk) {
+        const int c = gg + NG * kk;
+        if (c < 32) {  // row-group-uniform
+          const long long lg = group_sum<long long, TPR>(class_logit_part<D>(sWg, sWq, c, sub, q, G));
+          if (sub == 0) C.logit[c] = lg;
+        }
+      }
+      __syncthreads();
+      // largest logit, then lowest class (every warp finds the same)
+      long long key = C.logit[lane] * 32 + (31 - lane);
+      key = warp_max<long long>(key);
+      settle(3 * (31 - int(key & 31) + 1));
+    }
+
+    if constexpr (MODE == kPredictOnly) {
+      if (threadIdx.x == 0) a.budget_out[qi] = budget;
+      continue;
+    }
+
+    // ---- 3. descent of the past-only forest
+    int nf = 0, exp_hi = 0, exp_l1 = 0, exp_wide = 0;  // counters: warp 0's copies
+    const int keep = r >> bucket;
+    if (kDescend && keep > 0) {
+      if constexpr (!kUsesW) {
+        constexpr int UR = (kMaxLevels + NG - 1) / NG;
+        int x[UR][16];
+#pragma unroll
+        for (int u = 0; u < UR; ++u) {
+          const int k = u * NG + gg;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) x[u][j] = 0;
+          if (k < nR) ld_node32<D, kNarrow>(Th, Kh, n, narrow, B.plist[k], sub, x[u]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < UR; ++u) {
+          const int k = u * NG + gg;
+          const S sc = group_sum<S, TPR>(dot_tree<S>(q, x[u]));
+          if (k < nR && sub == 0) B.cand.put(k, B.plist[k], sc);
+        }
+        __syncthreads();
+      }
+      nf = nR;
+
+      for (int step = 0; step < 32; ++step) {
+        if (warp == 0) {
+          // classify the frontier (as query_kernel): keys stay; expanded nodes go to the x
+          // lists [wide | narrow | key] with the byte offset of their left child's row
+          int fd[kFrontSlots];
+          S fs[kFrontSlots];
+          int cat[kFrontSlots];
+          unsigned bl_[kFrontSlots], bw_[kFrontSlots], bn_[kFrontSlots], bk_[kFrontSlots];
+          int nl = 0, nw = 0, nn = 0, nk = 0;
+#pragma unroll
+          for (int s = 0; s < kFrontSlots; ++s) {
+            cat[s] = 0;
+            bl_[s] = bw_[s] = bn_[s] = bk_[s] = 0u;
+            fd[s] = 0;
+            fs[s] = S(0);
+            if (32 * s < nf) {
+              const int e = lane + 32 * s;
+              if (e < nf) {
+                const Cand<S> cd = B.cand.get(e);
+                fd[s] = cd.desc;
+                fs[s] = cd.score;
+                const int lv = desc_level(fd[s]);
+                cat[s] = lv <= bucket ? 1 : (lv == 1 ? 4 : ((!kNarrow || lv - 1 > narrow) ? 2 : 3));
+              }
+              bl_[s] = __ballot_sync(kFull, cat[s] == 1);
+              bw_[s] = __ballot_sync(kFull, cat[s] == 2);
+              if constexpr (kNarrow) bn_[s] = __ballot_sync(kFull, cat[s] == 3);
+              bk_[s] = __ballot_sync(kFull, cat[s] == 4);
+              nl += __popc(bl_[s]);
+              nw += __popc(bw_[s]);
+              nn += __popc(bn_[s]);
+              nk += __popc(bk_[s]);
+            }
+          }
+          const int nx = nw + nn + nk;
+          if (nx == 0) {
+            if constexpr (VAR) {
+              if (nf > keep) {
+                select_top_r<S, true>(B, nf, keep, lane, norm_l);
+                nf = keep;
+              }
+            }
+          } else {
+            exp_hi += nw + nn;
+            exp_l1 += nk;
+            exp_wide += nw;
+            __syncwarp();
+            const unsigned below = lanemask_lt(lane);
+            int ow = 0, on = nw, ok = nw + nn, ol = 0;
+#pragma unroll
+            for (int s = 0; s < kFrontSlots; ++s) {
+              if (cat[s] >= 2) {
+                const int pos = cat[s] == 2 ? ow + __popc(bw_[s] & below)
+                                            : (cat[s] == 3 ? on + __popc(bn_[s] & below)
+                                                           : ok + __popc(bk_[s] & below));
+                const int cl = desc_level(fd[s]) - 1;
+                const int st = desc_start(fd[s]);
+                B.xnode.put(pos, fd[s], fs[s]);
+                B.xrow[pos] = cat[s] == 4 ? st * D : tree_row_offset<D>(n, narrow, cl, st >> cl);
+              } else if (cat[s] == 1) {
+                B.cand.put(ol + __popc(bl_[s] & below), fd[s], fs[s]);
+              }
+              ow += __popc(bw_[s]);
+              on += __popc(bn_[s]);
+              ok += __popc(bk_[s]);
+              ol += __popc(bl_[s]);
+            }
+          }
+          if (lane == 0) {
+            C.ctl[0] = nw;
+            C.ctl[1] = nn;
+            C.ctl[2] = nk;
+            C.ctl[3] = nl;
+            C.ctl[4] = nf;
+          }
+        }
+        __syncthreads();
+        const int nw = C.ctl[0], nhi = nw + C.ctl[1], nx = nhi + C.ctl[2];
+        if (nx == 0) break;  // CTA-uniform
+        // left children over the CTA's row groups: int32 rows, int16 rows, key rows
+        for (int base = 0; base < nw; base += NG * UW)
+          cta_child_pass<0, UW, S, D>(B, Th, Kh, q, base, nw, warp, gg, sub);
+        if constexpr (kNarrow)
+          for (int base = nw; base < nhi; base += NG * UN)
+            cta_child_pass<1, UN, S, D>(B, Th, Kh, q, base, nhi, warp, gg, sub);
+        for (int base = nhi; base < nx; base += NG * UK)
+          cta_child_pass<2, UK, S, D>(B, Th, Kh, q, base, nx, warp, gg, sub);
+        __syncthreads();
+        if (warp == 0) {
+          const int nl = C.ctl[3];
+          for (int x0 = lane; x0 < nx; x0 += 32)
+            put_children<S>(B, nl, x0, B.xnode.get(x0), B.xleft[x0]);
+          const int Cn = nl + 2 * nx;
+          if (Cn > keep) {
+            select_top_r<S, VAR>(B, Cn, keep, lane, norm_l);
+            nf = keep;
+          } else {
+            nf = Cn;
+            __syncwarp();
+          }
+        }
+      }
+      nf = C.ctl[4];
+      if constexpr (VAR) {
+        if (bucket > 0) {
+          __syncthreads();  // every warp has read ctl before warp 0 rewrites it
+          if (warp == 0) {
+            nf = expand_buckets<S, D>(B, nf, Kh, q, lane);
+            if (lane == 0) C.ctl[4] = nf;
+          }
+          __syncthreads();
+          nf = C.ctl[4];
+        }
+      }
+    }
+
+    // ---- window key scores (with the predictor they were taken in phase 1)
+    if constexpr (kAttend && !kUsesW) {
+      constexpr int UWIN = (kMaxWindow + NG - 1) / NG;
+#pragma unroll
+      for (int u = 0; u < UWIN; ++u) {
+        const int x = u * NG + gg;
+        if (u * NG < nsel_win) {  // CTA-uniform
+          int xp[4] = {0, 0, 0, 0};
+          if (x < nsel_win) ld_key<D>(Kh + (long long)(i - x) * D, sub, xp);
+          const int s = group_sum<int, TPR>(dot_key(q, xp));
+          if (x < nsel_win && sub == 0) B.winsc[x] = s;
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- outputs of the route (warp 0)
+    const int count = nsel_win + nf;
+    if (warp == 0) {
+      if (lane == 0) {
+        if (a.count_out) a.count_out[qi] = count;
+        if (a.exp_out) {
+          a.exp_out[3 * qi] = exp_hi;
+          a.exp_out[3 * qi + 1] = exp_l1;
+          a.exp_out[3 * qi + 2] = exp_wide;
+        }
+        if (a.budget_out) a.budget_out[qi] = budget;
+      }
+      if (a.idx_out)
+        write_selection<S>(B, nf, nsel_win, i, a.idx_out + qi * a.max_keys, a.max_keys, lane);
+    }
+
+    // ---- 4. exact attention over window + routed keys
+    if constexpr (kAttend) {
+      if (warp == 0) {
+        const float scale = a.scale;
+        const float sw = lane < nsel_win ? float(B.winsc[lane]) * scale : -INFINITY;
+        float sr[kFrontSlots];
+        int kr[kFrontSlots];
+#pragma unroll
+        for (int s = 0; s < kFrontSlots; ++s) {
+          const int e = lane + 32 * s;
+          Cand<S> cd{0, S(0)};
+          if (e < nf) cd = B.cand.get(e);
+          sr[s] = e < nf ? float(cd.score) * scale : -INFINITY;
+          kr[s] = desc_start(cd.desc);
+        }
+        float m = sw;
+#pragma unroll
+        for (int s = 0; s < kFrontSlots; ++s) m = fmaxf(m, sr[s]);
+        m = warp_maxf(m);
+        const float pw = lane < nsel_win ? __expf(sw - m) : 0.f;
+        float pr[kFrontSlots];
+        float psum = pw;
+#pragma unroll
+        for (int s = 0; s < kFrontSlots; ++s) {
+          pr[s] = (lane + 32 * s) < nf ? __expf(sr[s] - m) : 0.f;
+          psum += pr[s];
+        }
+        const float den = warp_sumf(psum);
+        if (lane < nsel_win) {
+          B.selk[lane] = i - lane;
+          B.selp[lane] = pw;
+        }
+#pragma unroll
+        for (int s = 0; s < kFrontSlots; ++s) {
+          const int e = lane + 32 * s;
+          if (e < nf) {
+            B.selk[nsel_win + e] = kr[s];
+            B.selp[nsel_win + e] = pr[s];
+          }
+        }
+        if (lane == 0) C.inv = 1.f / den;
+      }
+      __syncthreads();
+      const int per = (count + kCtaWarps - 1) / kCtaWarps;
+      const int k0 = min(count, warp * per);
+      gather_values_part<D, 2>(B.selk, B.selp, k0, min(count, k0 + per),
+                               a.V + bh * (long long)n * D, lane, C.opart[warp]);
+      __syncthreads();
+      const float inv = C.inv;
+      for (int t = threadIdx.x; t < D; t += kCtaWarps * 32) {
+        float o = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < kCtaWarps; ++ww) o += C.opart[ww][t];
+        a.out[qi * D + t] = o * inv;
+      }
+    }
+  }
+}
+
+namespace {
+
+template <typename S, int D, int MODE, bool VAR>
+cudaError_t launch_cta_mode(const QueryArgs& a, cudaStream_t st) {
+  constexpr size_t smem = CtaSmem<S, D, MODE>::bytes;
+  auto kern = cta_query_kernel<S, D, MODE, VAR>;
+  static thread_local int cached_dev = -1;
+  static thread_local int per_sm = 0, sms = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != cached_dev) {
+    if (smem > 48 * 1024) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      if (e != cudaSuccess) return e;
+    }
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int b = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, kCtaWarps * 32, smem);
+    per_sm = b > 0 ? b : 1;
+    cached_dev = dev;
+  }
+  const long long cap = (long long)sms * per_sm;
+  const int blocks = int(a.num_queries < cap ? a.num_queries : cap);
+  if (blocks <= 0) return cudaSuccess;
+  kern<<<blocks, kCtaWarps * 32, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename S, int D, int MODE>
+cudaError_t launch_cta_variant(const QueryArgs& a, cudaStream_t st) {
+  if (MODE != kPredictOnly && (a.norm_l != 0 || a.bucket != 0))
+    return launch_cta_mode<S, D, MODE, MODE != kPredictOnly>(a, st);
+  return launch_cta_mode<S, D, MODE, false>(a, st);
+}
+
+template <int MODE>
+cudaError_t dispatch_cta(const QueryArgs& a, int d, int score_bits, cudaStream_t st) {
+  if (d == 64)
+    return score_bits == 32 ? launch_cta_variant<int, 64, MODE>(a, st)
+                            : launch_cta_variant<long long, 64, MODE>(a, st);
+  return score_bits == 32 ? launch_cta_variant<int, 128, MODE>(a, st)
+                          : launch_cta_variant<long long, 128, MODE>(a, st);
+}
+
+}  // namespace
+
+cudaError_t launch_query_cta(const QueryArgs& a, int d, int score_bits, int mode,
+                             cudaStream_t st) {
+  switch (mode) {
+    case kForwardPredict: return dispatch_cta<kForwardPredict>(a, d, score_bits, st);
+    case kForwardOverride: return dispatch_cta<kForwardOverride>(a, d, score_bits, st);
+    case kRouteOnly: return dispatch_cta<kRouteOnly>(a, d, score_bits, st);
+    default: return dispatch_cta<kPredictOnly>(a, d, score_bits, st);
+  }
+}
+
+}  // namespace alhr

@@ -21,6 +21,9 @@ cudaError_t launch_update_tree(const int8_t* K, char* tree, const TreeLayout& tl
 // The tree as plain int32 rows, level-major (see tree_build.cu).
 cudaError_t launch_tree_unpack(const char* tree, const TreeLayout& tl, long long bh,
                                int32_t* nodes, cudaStream_t st);
+// Plain int32 rows into the tree layout (see tree_build.cu).
+cudaError_t launch_tree_pack(const int32_t* nodes, const TreeLayout& tl, long long bh, int vb,
+                             char* tree, uint32_t* dev_err, cudaStream_t st);
 
 // Warp-per-query kernels (see query_kernels.cu).
 cudaError_t launch_forward(const QueryArgs& a, int d, int score_bits, bool predict,
@@ -28,6 +31,10 @@ cudaError_t launch_forward(const QueryArgs& a, int d, int score_bits, bool predi
 cudaError_t launch_route(const QueryArgs& a, int d, int score_bits, cudaStream_t st);
 cudaError_t launch_predict(const QueryArgs& a, int d, int score_bits, cudaStream_t st);
 cudaError_t launch_attend(const QueryArgs& a, int d, cudaStream_t st);
+// The latency shape: one query per CTA (see cta_query_kernels.cu); mode is a Mode of
+// query_common.cuh.
+cudaError_t launch_query_cta(const QueryArgs& a, int d, int score_bits, int mode,
+                             cudaStream_t st);
 
 // Phase-2 labels: top-k keys of every query's causal q . K row (see label_kernels.cu).
 cudaError_t launch_topk_labels(const int8_t* Q, const int8_t* K, int32_t* labels,

@@ -6,63 +6,31 @@
 // over the selected keys.
 //
 // Per query (one warp, rows scored in row groups, see alhr_device.cuh):
-//   1. causal sum: G_i = sum of keys [0, i] is the sum of the tree rows of the binary
-//      decomposition of [0, i+1). Its largest blocks are also the largest roots of the descent
-//      forest of [0, i-w] (both decompositions share every block above the highest bit where
-//      i+1 and i-w+1 differ), so their scores are taken in the same pass;
+//   1. causal sum: G_i = sum of keys [0, i] = (sum of the roots of the past-only forest, the
+//      aligned power-of-two blocks of [0, i-w]) + (sum of the window keys (i-w, i]). Both kinds
+//      of rows are read in one pass and scored there too: the roots for the descent, the window
+//      keys for the attention, so G_i costs no extra row;
 //   2. budget: logits over 32 classes from W in shared memory (int64, ties -> lower class), or
-//      the given budget;
-//   3. the remaining roots, then the descent: each step reads only the LEFT child of every
-//      expanded node (the right child's score is parent - left, exact in integers) and keeps the
-//      best r by an exact integer bisection (select_top_r);
-//   4. attention: the selected window keys are scored, routed keys keep the scores of the
-//      descent (their key rows are not read again), and the value rows are gathered.
+//      the given budget (the roots and window keys are then read only where they are used);
+//   3. the descent: each step reads only the LEFT child of every expanded node (the right
+//      child's score is parent - left, exact in integers) and keeps the best r by an exact
+//      integer bisection (select_top_r);
+//   4. attention: routed keys keep the scores of the descent (their key rows are not read
+//      again), the window keys theirs from phase 1, and the value rows are gathered.
 // Descent variants (runtime, both off by default): ranking by means (the selection scales each
 // candidate's sum by 2^(L - level)), and leaf buckets (nodes of level <= b are not expanded, the
 // beam keeps r >> b of them, and their keys are listed and scored after the descent).
 #include <atomic>
 #include <cuda_runtime.h>
 
-#include "alhr_device.cuh"
 #include "internal.h"
+#include "query_common.cuh"
 
 namespace alhr {
 
-enum Mode : int { kForwardPredict = 0, kForwardOverride = 1, kRouteOnly = 2, kPredictOnly = 3 };
-
-// Writes the two children of expanded node x (the node p; its left child's score `left`).
-template <typename S>
-__device__ __forceinline__ void put_children(WarpBuf<S>& B, int nl, int x, Cand<S> p, S left) {
-  const int cl = desc_level(p.desc) - 1;
-  const int st = desc_start(p.desc);
-  const S ps = p.score;
-  B.cand.put(nl + 2 * x, make_desc(st, cl), left);
-  B.cand.put(nl + 2 * x + 1, make_desc(st + (1 << cl), cl), ps - left);
-}
-
-// Dynamic shared memory of a query kernel: the predictor weights (the G half widened to
-// int32, then the q half as packed int8 words; within a class row the 4-dim words are stored
-// grouped by their position in a lane's 16 dims, and rows are padded, so that the row groups,
-// which read different classes at once, hit different banks) followed by one WarpBuf per
-// warp.
-template <int D>
-struct WLayout {
-  static constexpr int g_stride = D + 16;     // ints per class row of the G half
-  static constexpr int q_stride = D / 4 + 4;  // words per class row of the q half
-};
-template <typename S, int D, int MODE>
-struct QuerySmem {
-  static constexpr bool kUsesW = (MODE == kForwardPredict || MODE == kPredictOnly);
-  static constexpr size_t w_bytes =
-      kUsesW ? size_t(32 * WLayout<D>::g_stride + 32 * WLayout<D>::q_stride) * 4 : 0;
-  static constexpr size_t bytes_for(int warps) { return w_bytes + warps * sizeof(WarpBuf<S>); }
-};
-
-// Warps (queries in flight) per CTA: the latency shape runs 4, one per SM sub-partition, so that
-// a small launch spreads over twice as many SMs and no two of its queries share an issue slot.
-constexpr int kLatWarps = 4;
-template <bool LAT>
-constexpr int warps_per_cta() { return LAT ? kLatWarps : kWarps; }
+// Bit 29 of a node descriptor is free (start < 2^20): it marks, in the list of causal-sum
+// blocks, a block that is also a root of the descent forest.
+constexpr int kFlagRoot = 1 << 29;
 
 // Register budget: int32 scores keep three CTAs (24 warps) per SM with two tree rows in flight
 // per row group; int64 scores need more registers, so two CTAs (and one int32 row in flight).
@@ -102,49 +70,6 @@ __device__ __forceinline__ void tree_child_pass(WarpBuf<S>& B, const char* Th, c
   }
 }
 
-// Leaf buckets (descent variant): the kept nodes, all of level <= bucket, become the list of
-// their keys, each scored q . k, in place of the frontier; returns the number of keys. At most
-// r >> bucket nodes (< 64) and r keys (< 96). Out of line: only the bucket variant reaches it.
-template <typename S, int D>
-__device__ __noinline__ int expand_buckets(WarpBuf<S>& B, int nf, const int8_t* Kh, const RowQ q,
-                                           int lane) {
-  constexpr int TPR = Lay<D>::TPR;
-  constexpr int RPI = Lay<D>::RPI;
-  const int grp = lane / TPR, sub = lane % TPR;
-  int total = 0;
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    const int e = lane + 32 * s;
-    int sz = 0, st = 0;
-    if (e < nf) {
-      const int ds = B.cand.desc(e);
-      sz = 1 << desc_level(ds);
-      st = desc_start(ds);
-    }
-    int incl = sz;  // inclusive scan of the bucket sizes over the lanes
-#pragma unroll
-    for (int off = 1; off < 32; off *= 2) {
-      const int y = __shfl_up_sync(kFull, incl, off);
-      if (lane >= off) incl += y;
-    }
-    const int pos = total + incl - sz;
-    for (int t = 0; t < sz; ++t) B.xrow[pos + t] = st + t;
-    total += __shfl_sync(kFull, incl, 31);
-  }
-  __syncwarp();
-  for (int base = 0; base < total; base += RPI) {
-    const int k = base + grp;
-    int xp[4] = {0, 0, 0, 0};
-    if (k < total) ld_key<D>(Kh + (long long)B.xrow[k] * D, sub, xp);
-    const int sc = group_sum<int, TPR>(dot_key(q, xp));
-    if (k < total && sub == 0) {
-      B.cand.put(k, make_desc(B.xrow[k], 0), S(sc));
-    }
-  }
-  __syncwarp();
-  return total;
-}
-
 // One pass over expanded nodes whose left child is an int16 tree row (positions [base, end) of
 // the x lists, all narrow): US rows per group, every load issued before any is scored.
 template <int US, typename S, int D>
@@ -174,70 +99,34 @@ __device__ __forceinline__ void narrow_child_pass(WarpBuf<S>& B, const char* Th,
   }
 }
 
-// The selection in ascending order, -1 padded: the routed keys (all below the window) sorted by
-// rank counting, then the window keys. Out of line: only the route outputs ask for it.
-template <typename S>
-__device__ __noinline__ void write_selection(const WarpBuf<S>& B, int nf, int nsel_win, int i,
-                                             int32_t* io, int max_keys, int lane) {
-#pragma unroll
-  for (int s = 0; s < kFrontSlots; ++s) {
-    const int e = lane + 32 * s;
-    if (e < nf) {
-      const int st = desc_start(B.cand.desc(e));
-      int rank = 0;
-      for (int f = 0; f < nf; ++f) rank += desc_start(B.cand.desc(f)) < st ? 1 : 0;
-      io[rank] = st;
-    }
-  }
-  if (lane < nsel_win) io[nf + nsel_win - 1 - lane] = i - lane;
-  for (int pp = nf + nsel_win + lane; pp < max_keys; pp += 32) io[pp] = -1;
-}
-
-// Any node of the forest (a key at level 0, an int16 or int32 tree row above) as this lane's 16
-// per-dimension integers; used by the latency mode's batched passes over causal-sum rows and roots.
-template <int D, bool kNarrow>
-__device__ __forceinline__ void ld_node32(const char* Th, const int8_t* Kh, int n, int narrow,
-                                          int pd, int sub, int (&x)[16]) {
-  const int lvl = desc_level(pd);
-  const int st = desc_start(pd);
-  if (lvl == 0) {
-    int xp[4];
-    ld_key<D>(Kh + (long long)st * D, sub, xp);
-#pragma unroll
-    for (int v = 0; v < 4; ++v)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) x[4 * v + e] = sx8(xp[v], e);
-  } else if (kNarrow && lvl <= narrow) {
-    ld_tree16_as32<D>(Th + tree_row_offset<D>(n, narrow, lvl, st >> lvl), sub, x);
-  } else {
-    ld_tree<D>(Th + tree_row_offset<D>(n, narrow, lvl, st >> lvl), sub, x);
-  }
-}
-
-// LAT selects the latency mode, for launches with too few queries to fill the GPU (decode): every
-// warp keeps many more rows in flight per pass (registers are no constraint at one CTA per SM),
-// so a descent step takes one or two round trips to memory instead of up to ten.
-// VAR compiles in the descent variants (ranking by means, leaf buckets; chosen at run time from
-// the arguments); without it the method's descent carries none of their code.
-template <typename S, int D, int MODE, bool LAT, bool VAR>
-__global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_blocks_per_sm<S>())
+// The warp-per-query kernel (the throughput shape: several CTAs of eight warps per SM, for
+// launches that fill the GPU; smaller launches take the CTA-per-query kernel of
+// cta_query_kernels.cu). VAR compiles in the descent variants (ranking by means, leaf buckets;
+// chosen at run time from the arguments); without it the method's descent carries none of their
+// code.
+template <typename S, int D, int MODE, bool VAR>
+__global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>())
     query_kernel(const QueryArgs a) {
-  constexpr int NW = warps_per_cta<LAT>();
+  constexpr int NW = kWarps;
   constexpr int TPR = Lay<D>::TPR;
   constexpr int RPI = Lay<D>::RPI;
-  // tree rows per group per pass (at d = 128: int16 rows; int32 rows take UW)
-  constexpr int U = LAT ? (D == 128 ? 12 : 4) : tree_rows_in_flight<S, D>();
-  constexpr int UK = LAT ? 8 : 1;  // key rows per group per pass
-  constexpr int UW = LAT ? 4 : 1;  // d = 128: int32 tree rows per group per pass
-  constexpr int UV = LAT ? 8 : 2;  // value-row passes in flight
+  // tree rows per group per pass (at d = 128: int16 rows; int32 rows go one per pass)
+  constexpr int U = tree_rows_in_flight<S, D>();
+  constexpr int UV = 2;  // value-row passes in flight
   constexpr bool kUsesW = (MODE == kForwardPredict || MODE == kPredictOnly);
   constexpr bool kDescend = (MODE != kPredictOnly);
   constexpr bool kAttend = (MODE == kForwardPredict || MODE == kForwardOverride);
   constexpr bool kNarrow = (D == 128);  // int16 tree levels exist (see tree_layout.h)
+  // How G_i is formed with the predictor. At d = 128: from the forest roots of [0, i-w] and the
+  // window keys, which the query reads anyway (no extra row). At d = 64: from the blocks of the
+  // binary decomposition of [0, i+1), whose largest blocks are also the largest roots (read
+  // once for both) -- about 2.6 more rows per query, but measured 3 % faster there than summing
+  // the window keys into G_i, which costs 16 more instructions per key row and spills
+  // registers in this register-bound kernel.
+  constexpr bool kGBlocks = kUsesW && D == 64;
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
   constexpr int GS = WLayout<D>::g_stride;
-  constexpr int QS = WLayout<D>::q_stride;
   int* sWg = reinterpret_cast<int*>(smem_raw);
   int* sWq = sWg + 32 * GS;
   WarpBuf<S>* wbuf = reinterpret_cast<WarpBuf<S>*>(smem_raw + QuerySmem<S, D, MODE>::w_bytes);
@@ -247,16 +136,7 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
   const int grp = lane / TPR;
   const int sub = lane % TPR;
   if constexpr (kUsesW) {
-    // word m (dims 4m .. 4m+3) of a class row goes to slot w_slot<D>(m), so that the lanes of
-    // a row group read consecutive slots
-    for (int k = threadIdx.x; k < 32 * D / 4; k += blockDim.x) {
-      const int c = k / (D / 4), m = k - c * (D / 4);
-      sWq[c * QS + w_slot<D>(m)] = __ldg(reinterpret_cast<const int*>(a.W + c * 2 * D) + m);
-    }
-    for (int k = threadIdx.x; k < 32 * D; k += blockDim.x) {
-      const int c = k / D, t = k - c * D;
-      sWg[c * GS + 4 * w_slot<D>(t >> 2) + (t & 3)] = a.W[c * 2 * D + D + t];
-    }
+    stage_weights<D>(a.W, sWg, sWq);
     __syncthreads();
   }
   WarpBuf<S>& B = wbuf[warp];
@@ -290,12 +170,13 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
     const int nwin = min(w, i + 1);  // keys of the window
     const int M = i - w + 1;         // keys before the window: [0, M)
     const unsigned Mu = M > 0 ? unsigned(M) : 0u;
+    const int nR = __popc(Mu);       // roots of the descent forest: the blocks of [0, M)
+    // kGBlocks: the blocks of [0, i+1) above the highest bit where i+1 and i-w+1 differ are also
+    // the largest roots; the rest of the roots (below that bit) are read only for the descent
     const unsigned A = unsigned(i + 1);
-    // highest bit where i+1 and i-w+1 differ; the blocks above it are shared by the causal-sum
-    // decomposition and the descent forest
-    const int p = kUsesW ? (M > 0 ? 31 - __clz(A ^ Mu) : 31) : 31;
+    const int p = kGBlocks ? (M > 0 ? 31 - __clz(A ^ Mu) : 31) : 31;
     const unsigned low_mask = p >= 31 ? 0xffffffffu : ((2u << p) - 1u);
-    const int n_common = __popc(Mu & ~low_mask);
+    const int n_common = kGBlocks ? __popc(Mu & ~low_mask) : 0;
 
     int budget = 0, b_eff = 0, nsel_win = 0, r = 0;
     auto settle = [&](int bud) {
@@ -310,118 +191,120 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
     };
     if constexpr (!kUsesW) settle(__ldg(a.budget_in + qi));
 
-    // ---- 1. causal sum G_i over the blocks of [0, i+1) (and the shared roots' scores)
+    // ---- 1. causal sum G_i and budget
     if constexpr (kUsesW) {
       int G[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) G[j] = 0;
-      const int nA = __popc(A);
-      __syncwarp();
-      if ((A >> lane) & 1u) {
-        const int b = lane;
-        const int rank = __popc(A >> b) - 1;
-        const int start = int((A >> b) << b) - (1 << b);
-        B.plist[rank] = make_desc(start, b) | kFlagG | ((M > 0 && b > p) ? kFlagRoot : 0);
-      }
-      __syncwarp();
-      if constexpr (LAT) {
-        // All causal-sum rows in one or two round trips: UG rows per group per pass, at most
-        // NP passes (i + 1 < 2^20 has at most 20 blocks). The shared roots' scores are kept in
-        // registers and stored after the cross-group sum of G_i: with the (divergent) stores
-        // inside the pass, that sum came out wrong on sm_100a.
-        constexpr int UG = 4;
-        constexpr int NP = (kMaxLevels + UG * RPI - 1) / (UG * RPI);
-        S rsc[NP][UG];
-#pragma unroll
-        for (int ps = 0; ps < NP; ++ps) {
-          const int base = ps * UG * RPI;
-          int x[UG][16];
-#pragma unroll
-          for (int u = 0; u < UG; ++u) {
-            const int k = base + u * RPI + grp;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) x[u][j] = 0;
-            if (k < nA) ld_node32<D, kNarrow>(Th, Kh, n, narrow, B.plist[k], sub, x[u]);
-          }
-#pragma unroll
-          for (int u = 0; u < UG; ++u) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) G[j] += x[u][j];
-            rsc[ps][u] = base < nA ? group_sum<S, TPR>(dot_tree<S>(q, x[u])) : S(0);
-          }
+      if constexpr (kGBlocks) {
+        // the blocks of [0, i+1), largest first; the shared roots' scores go to the front of
+        // the candidate list
+        const int nA = __popc(A);
+        __syncwarp();
+        if ((A >> lane) & 1u) {
+          const int b = lane;
+          const int rank = __popc(A >> b) - 1;
+          const int start = int((A >> b) << b) - (1 << b);
+          B.plist[rank] = make_desc(start, b) | ((M > 0 && b > p) ? kFlagRoot : 0);
         }
         __syncwarp();
+        for (int base = 0; base < nA; base += RPI) {
+          const int k = base + grp;
+          const bool active = k < nA;
+          const int pd = active ? B.plist[k] : 0;
+          const int lvl = desc_level(pd);
+          const int st = desc_start(pd);
+          S sc = 0;
+          if (active) {
+            if (lvl > 0) {
+              int x[16];
+              const char* row = Th + tree_row_offset<D>(n, narrow, lvl, st >> lvl);
+              if (kNarrow && lvl <= narrow) ld_tree16_as32<D>(row, sub, x);
+              else ld_tree<D>(row, sub, x);
 #pragma unroll
-        for (int off = TPR; off < 32; off *= 2)
+              for (int j = 0; j < 16; ++j) G[j] += x[j];
+              sc = dot_tree<S>(q, x);
+            } else {
+              int xp[4];
+              ld_key<D>(Kh + (long long)st * D, sub, xp);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) G[j] += __shfl_xor_sync(kFull, G[j], off);
+              for (int v = 0; v < 4; ++v)
 #pragma unroll
-        for (int ps = 0; ps < NP; ++ps)
-#pragma unroll
-          for (int u = 0; u < UG; ++u) {
-            const int k = ps * UG * RPI + u * RPI + grp;
-            if (k < nA && sub == 0) {
-              const int pd = B.plist[k];
-              if (pd & kFlagRoot) {
-                B.cand.put(k, pd & ~(kFlagRoot | kFlagG), rsc[ps][u]);
-              }
+                for (int e = 0; e < 4; ++e) G[4 * v + e] += sx8(xp[v], e);
+              sc = S(dot_key(q, xp));
             }
           }
-      } else
-      for (int base = 0; base < nA; base += RPI) {
-        const int k = base + grp;
-        const bool active = k < nA;
-        const int pd = active ? B.plist[k] : 0;
-        const int lvl = desc_level(pd);
-        const int st = desc_start(pd);
-        S sc = 0;
-        if (active) {
-          if (lvl > 0) {
-            int x[16];
-            const char* row = Th + tree_row_offset<D>(n, narrow, lvl, st >> lvl);
-            if (kNarrow && lvl <= narrow) ld_tree16_as32<D>(row, sub, x);
-            else ld_tree<D>(row, sub, x);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) G[j] += x[j];
-            sc = dot_tree<S>(q, x);
-          } else {
-            int xp[4];
-            ld_key<D>(Kh + (long long)st * D, sub, xp);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) G[4 * v + e] += sx8(xp[v], e);
-            sc = S(dot_key(q, xp));
+          sc = group_sum<S, TPR>(sc);
+          if (active && sub == 0 && (pd & kFlagRoot)) {
+            B.cand.put(k, pd & ~kFlagRoot, sc);  // the shared roots are the first ones
           }
         }
-        sc = group_sum<S, TPR>(sc);
-        if (active && sub == 0 && (pd & kFlagRoot)) {
-          B.cand.put(k, pd & ~(kFlagRoot | kFlagG), sc);  // common roots are the first ones
+      } else {
+        // the forest roots, largest first
+        __syncwarp();
+        if ((Mu >> lane) & 1u) {
+          const int b = lane;
+          B.plist[__popc(Mu >> b) - 1] = make_desc(int((Mu >> b) << b) - (1 << b), b);
+        }
+        __syncwarp();
+        // roots: one row per group per pass. Every lane of a row group stores the score (the
+        // same value; rows past the end into a spare slot), so the pass has no divergent store
+        // before the cross-group sum of G_i below.
+        for (int base = 0; base < nR; base += RPI) {
+          const int k = base + grp;
+          const bool active = k < nR;
+          const int pd = active ? B.plist[k] : 0;
+          const int lvl = desc_level(pd);
+          const int st = desc_start(pd);
+          S sc = 0;
+          if (active) {
+            if (lvl > 0) {
+              int x[16];
+              const char* row = Th + tree_row_offset<D>(n, narrow, lvl, st >> lvl);
+              if (kNarrow && lvl <= narrow) ld_tree16_as32<D>(row, sub, x);
+              else ld_tree<D>(row, sub, x);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) G[j] += x[j];
+              sc = dot_tree<S>(q, x);
+            } else {
+              int xp[4];
+              ld_key<D>(Kh + (long long)st * D, sub, xp);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) G[4 * v + e] = __dp4a(xp[v], 1 << (8 * e), G[4 * v + e]);
+              sc = S(dot_key(q, xp));
+            }
+          }
+          sc = group_sum<S, TPR>(sc);
+          B.cand.put(active ? k : kMaxCand - 1, pd, sc);
+        }
+        // window keys i, i-1, ..., one per group per pass: scores for the attention, values
+        // into G_i (dp4a with a one-hot byte picks one sign-extended dimension)
+        for (int base = 0; base < nwin; base += RPI) {
+          const int x = base + grp;
+          int xp[4] = {0, 0, 0, 0};
+          if (x < nwin) ld_key<D>(Kh + (long long)(i - x) * D, sub, xp);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) G[4 * v + e] = __dp4a(xp[v], 1 << (8 * e), G[4 * v + e]);
+          const int sw = group_sum<int, TPR>(dot_key(q, xp));
+          B.winsc[x < nwin ? x : kMaxWindow] = sw;
         }
       }
-      if constexpr (!LAT) {
+      __syncwarp();
 #pragma unroll
-        for (int off = TPR; off < 32; off *= 2)
+      for (int off = TPR; off < 32; off *= 2)
 #pragma unroll
-          for (int j = 0; j < 16; ++j) G[j] += __shfl_xor_sync(kFull, G[j], off);
-      }
+        for (int j = 0; j < 16; ++j) G[j] += __shfl_xor_sync(kFull, G[j], off);
 
       // ---- 2. budget predictor: group grp scores classes grp, grp+RPI, ...
       long long best = ScoreLimits<long long>::lowest;
 #pragma unroll
       for (int k = 0; k < 32 / RPI; ++k) {
         const int c = grp + RPI * k;
-        int sq = 0;
-        long long sg = 0;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int m = w_lane_slot<D>(sub, v);  // slot of the lane's word v
-          sq = __dp4a(sWq[c * QS + m], q.qp[v], sq);
-          const int4 wg = *reinterpret_cast<const int4*>(sWg + c * GS + 4 * m);
-          sg += (long long)wg.x * G[4 * v] + (long long)wg.y * G[4 * v + 1] +
-                (long long)wg.z * G[4 * v + 2] + (long long)wg.w * G[4 * v + 3];
-        }
-        const long long logit = group_sum<long long, TPR>(sg + sq);
+        const long long logit = group_sum<long long, TPR>(class_logit_part<D>(sWg, sWq, c, sub, q, G));
         // largest logit, then lowest class: pack (logit, 31 - class)
         const long long key = logit * 32 + (31 - c);
         best = key > best ? key : best;
@@ -443,65 +326,44 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
     int nf = 0, exp_hi = 0, exp_l1 = 0, exp_wide = 0;
     const int keep = r >> bucket;  // beam width in buckets (keys when bucket = 0)
     if (kDescend && keep > 0) {    // r > 0 implies i >= w, i.e. M > 0
-      // roots not yet scored: the blocks of [0, M) below the shared ones
-      const unsigned rest = Mu & low_mask;
-      const int nB = __popc(rest);
-      __syncwarp();
-      if ((rest >> lane) & 1u) {
-        const int b = lane;
-        B.plist[__popc(rest >> b) - 1] = make_desc(int((Mu >> b) << b) - (1 << b), b);
-      }
-      __syncwarp();
-      if constexpr (LAT) {
-        constexpr int UR = 4;
-        for (int base = 0; base < nB; base += UR * RPI) {
-          int x[UR][16];
-#pragma unroll
-          for (int u = 0; u < UR; ++u) {
-            const int k = base + u * RPI + grp;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) x[u][j] = 0;
-            if (k < nB) ld_node32<D, kNarrow>(Th, Kh, n, narrow, B.plist[k], sub, x[u]);
-          }
-          __syncwarp();  // reconverge after the per-group branches, before the group sums
-#pragma unroll
-          for (int u = 0; u < UR; ++u) {
-            const int k = base + u * RPI + grp;
-            const S sc = group_sum<S, TPR>(dot_tree<S>(q, x[u]));
-            if (k < nB && sub == 0) {
-              B.cand.put(n_common + k, B.plist[k], sc);
+      // roots not scored yet: all of them without the predictor, those below the shared
+      // blocks with kGBlocks
+      if constexpr (!kUsesW || kGBlocks) {
+        const unsigned rest = Mu & low_mask;
+        const int nB = __popc(rest);
+        __syncwarp();
+        if ((rest >> lane) & 1u) {
+          const int b = lane;
+          B.plist[__popc(rest >> b) - 1] = make_desc(int((Mu >> b) << b) - (1 << b), b);
+        }
+        __syncwarp();
+        for (int base = 0; base < nB; base += RPI) {
+          const int k = base + grp;
+          const bool active = k < nB;
+          const int pd = active ? B.plist[k] : 0;
+          const int lvl = desc_level(pd);
+          const int st = desc_start(pd);
+          S sc = 0;
+          if (active) {
+            if (lvl == 0) {
+              int xp[4];
+              ld_key<D>(Kh + (long long)st * D, sub, xp);
+              sc = S(dot_key(q, xp));
+            } else if (!kNarrow || lvl > narrow) {
+              int x[16];
+              ld_tree<D>(Th + tree_row_offset<D>(n, narrow, lvl, st >> lvl), sub, x);
+              sc = dot_tree<S>(q, x);
+            } else {
+              int w[8];
+              ld_tree16<D>(Th + tree_row_offset<D>(n, narrow, lvl, st >> lvl), sub, w);
+              sc = S(dot_tree16(q, w));
             }
           }
-        }
-      } else
-      for (int base = 0; base < nB; base += RPI) {
-        const int k = base + grp;
-        const bool active = k < nB;
-        const int pd = active ? B.plist[k] : 0;
-        const int lvl = desc_level(pd);
-        const int st = desc_start(pd);
-        S sc = 0;
-        if (active) {
-          if (lvl == 0) {
-            int xp[4];
-            ld_key<D>(Kh + (long long)st * D, sub, xp);
-            sc = S(dot_key(q, xp));
-          } else if (!kNarrow || lvl > narrow) {
-            int x[16];
-            ld_tree<D>(Th + tree_row_offset<D>(n, narrow, lvl, st >> lvl), sub, x);
-            sc = dot_tree<S>(q, x);
-          } else {
-            int w[8];
-            ld_tree16<D>(Th + tree_row_offset<D>(n, narrow, lvl, st >> lvl), sub, w);
-            sc = S(dot_tree16(q, w));
-          }
-        }
-        sc = group_sum<S, TPR>(sc);
-        if (active && sub == 0) {
-          B.cand.put(n_common + k, pd, sc);
+          sc = group_sum<S, TPR>(sc);
+          if (active && sub == 0) B.cand.put(n_common + k, pd, sc);
         }
       }
-      nf = __popc(Mu);
+      nf = nR;
 
       for (int step = 0; step < 32; ++step) {
         __syncwarp();
@@ -584,31 +446,21 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
         if constexpr (kNarrow) {
           // int32 and int16 rows in passes of their own, so that every pass issues all of its
           // loads before it scores any (one memory round trip per pass)
-          for (int base = 0; base < nw; base += UW * RPI)
-            tree_child_pass<UW, S, D>(B, Th, q, base, nw, grp, sub);
+          for (int base = 0; base < nw; base += RPI)
+            tree_child_pass<1, S, D>(B, Th, q, base, nw, grp, sub);
           for (int base = nw; base < nhi; base += U * RPI)
             narrow_child_pass<U, S, D>(B, Th, q, base, nhi, grp, sub);
         } else {
           for (int base = 0; base < nhi; base += U * RPI)
             tree_child_pass<U, S, D>(B, Th, q, base, nhi, grp, sub);
         }
-        // left children that are keys: UK rows per group in flight
-        for (int base = nhi; base < nx; base += UK * RPI) {
-          int xp[UK][4];
-#pragma unroll
-          for (int u = 0; u < UK; ++u) {
-            const int xi = base + u * RPI + grp;
-#pragma unroll
-            for (int v = 0; v < 4; ++v) xp[u][v] = 0;
-            if (xi < nx) ld_key<D>(Kh + B.xrow[xi], sub, xp[u]);
-          }
-          if constexpr (LAT) __syncwarp();
-#pragma unroll
-          for (int u = 0; u < UK; ++u) {
-            const int xi = base + u * RPI + grp;
-            const int left = group_sum<int, TPR>(dot_key(q, xp[u]));
-            if (xi < nx && sub == 0) B.xleft[xi] = S(left);
-          }
+        // left children that are keys: one per group per pass
+        for (int base = nhi; base < nx; base += RPI) {
+          const int xi = base + grp;
+          int xp[4] = {0, 0, 0, 0};
+          if (xi < nx) ld_key<D>(Kh + B.xrow[xi], sub, xp);
+          const int left = group_sum<int, TPR>(dot_key(q, xp));
+          if (xi < nx && sub == 0) B.xleft[xi] = S(left);
         }
         __syncwarp();
         // both children of every expanded node, one node per lane
@@ -626,24 +478,15 @@ __global__ void __launch_bounds__(warps_per_cta<LAT>() * 32, LAT ? 1 : min_block
         if (bucket > 0) nf = expand_buckets<S, D>(B, nf, Kh, q, lane);
     }
 
-    // ---- window key scores (attention only needs the selected ones)
-    if constexpr (kAttend) {
-      for (int base = 0; base < nsel_win; base += UK * RPI) {
-        int xp[UK][4];
-#pragma unroll
-        for (int u = 0; u < UK; ++u) {
-          const int x = base + u * RPI + grp;
-#pragma unroll
-          for (int v = 0; v < 4; ++v) xp[u][v] = 0;
-          if (x < nsel_win) ld_key<D>(Kh + (long long)(i - x) * D, sub, xp[u]);
-        }
-        if constexpr (LAT) __syncwarp();
-#pragma unroll
-        for (int u = 0; u < UK; ++u) {
-          const int x = base + u * RPI + grp;
-          const int s = group_sum<int, TPR>(dot_key(q, xp[u]));
-          if (x < nsel_win && sub == 0) B.winsc[x] = s;
-        }
+    // ---- window key scores (attention only needs the selected ones; with the predictor at
+    //      d = 128 they were taken in phase 1)
+    if constexpr (kAttend && !(kUsesW && !kGBlocks)) {
+      for (int base = 0; base < nsel_win; base += RPI) {
+        const int x = base + grp;
+        int xp[4] = {0, 0, 0, 0};
+        if (x < nsel_win) ld_key<D>(Kh + (long long)(i - x) * D, sub, xp);
+        const int s = group_sum<int, TPR>(dot_key(q, xp));
+        if (x < nsel_win && sub == 0) B.winsc[x] = s;
       }
     }
     __syncwarp();
@@ -789,6 +632,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(const QueryArgs a) 
 namespace {
 
 constexpr int kOccSlots = 66;
+constexpr int kLatCtasPerSm = 4;  // resident CTAs of the latency shape per SM
 
 // Grid size of a persistent launch: the resident CTAs of every SM, capped by the work. The
 // per-device occupancy (and the opt-in to more than 48 KB of dynamic shared memory) is
@@ -821,14 +665,14 @@ int blocks_for(KernelT kernel, int slot, size_t smem, long long queries, cudaErr
   return int(need < cap ? need : cap);
 }
 
-template <typename S, int D, int MODE, bool LAT, bool VAR>
+template <typename S, int D, int MODE, bool VAR>
 cudaError_t launch_query_mode(const QueryArgs& a, cudaStream_t st) {
-  constexpr int slot = (((MODE * 2 + (D == 128 ? 1 : 0)) * 2 + (sizeof(S) == 8 ? 1 : 0)) * 2 +
-                        (LAT ? 1 : 0)) * 2 + (VAR ? 1 : 0);
+  constexpr int slot = ((MODE * 2 + (D == 128 ? 1 : 0)) * 2 + (sizeof(S) == 8 ? 1 : 0)) * 2 +
+                       (VAR ? 1 : 0);
   static_assert(slot < 64, "occupancy cache slot");
-  constexpr int nw = warps_per_cta<LAT>();
+  constexpr int nw = kWarps;
   constexpr size_t smem = QuerySmem<S, D, MODE>::bytes_for(nw);
-  auto kern = query_kernel<S, D, MODE, LAT, VAR>;
+  auto kern = query_kernel<S, D, MODE, VAR>;
   cudaError_t err;
   const int blocks = blocks_for(kern, slot, smem, a.num_queries, &err, nw);
   if (err != cudaSuccess) return err;
@@ -839,8 +683,8 @@ cudaError_t launch_query_mode(const QueryArgs& a, cudaStream_t st) {
 
 std::atomic<int> g_launch_mode{0};
 
-// Auto: a launch of at most 8 queries per SM (one warp each) cannot fill the GPU, so it takes
-// the latency shape; measured on B200 the throughput shape wins from about 2048 queries up.
+// Auto: a launch whose queries all fit the GPU as one CTA each (the latency shape, four CTAs per
+// SM) takes that shape; larger launches take one warp per query.
 template <typename S, int D, int MODE>
 cudaError_t launch_query(const QueryArgs& a, cudaStream_t st) {
   const int mode = g_launch_mode.load(std::memory_order_relaxed);
@@ -853,14 +697,13 @@ cudaError_t launch_query(const QueryArgs& a, cudaStream_t st) {
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
       cached_dev = dev;
     }
-    lat = a.num_queries <= (long long)sms * kWarps;
+    lat = a.num_queries <= (long long)sms * kLatCtasPerSm;
   }
+  if (lat) return launch_query_cta(a, D, sizeof(S) == 4 ? 32 : 64, MODE, st);
   // the predictor alone never descends: it needs no variant instantiation
   if (MODE != kPredictOnly && (a.norm_l != 0 || a.bucket != 0))
-    return lat ? launch_query_mode<S, D, MODE, true, MODE != kPredictOnly>(a, st)
-               : launch_query_mode<S, D, MODE, false, MODE != kPredictOnly>(a, st);
-  return lat ? launch_query_mode<S, D, MODE, true, false>(a, st)
-             : launch_query_mode<S, D, MODE, false, false>(a, st);
+    return launch_query_mode<S, D, MODE, MODE != kPredictOnly>(a, st);
+  return launch_query_mode<S, D, MODE, false>(a, st);
 }
 
 template <int MODE>

@@ -446,6 +446,60 @@ cudaError_t launch_update_tree(const int8_t* K, char* tree, const TreeLayout& tl
   return cudaGetLastError();
 }
 
+// The inverse of tree_unpack_kernel: plain level-major int32 rows [bh][n-1][d] into the tree
+// layout (int16 rows for the narrow levels). A value of a narrow level outside
+// [-vb * 2^l, vb * 2^l] cannot be the sum of 2^l keys within the value bound: it is saturated to
+// int16 and flags ALHR_DEVERR_VALUE_RANGE.
+template <int D>
+__global__ void __launch_bounds__(256)
+    tree_pack_kernel(const int4* __restrict__ nodes, const TreeLayout tl, long long bh, int vb,
+                     char* __restrict__ tree, uint32_t* dev_err) {
+  constexpr int Q4 = D / 4;
+  const int n = tl.n;
+  const long long per_block = (long long)(n - 1) * Q4;
+  const long long total = bh * per_block;
+  bool bad = false;
+  for (long long k = blockIdx.x * (long long)blockDim.x + threadIdx.x; k < total;
+       k += (long long)gridDim.x * blockDim.x) {
+    const long long b = k / per_block;
+    const long long rem = k - b * per_block;
+    const int r = int(rem / Q4), c = int(rem - (long long)r * Q4);
+    int l = 1;
+    while (l < tl.L && r >= n - (n >> l)) ++l;  // level l holds rows [n - (n>>(l-1)), n - (n>>l))
+    const int j = r - (n - (n >> (l - 1)));
+    char* row = tree + b * tl.block_bytes + tl.level_off[l] + (long long)j * tl.row_bytes(l);
+    const int4 v = __ldg(nodes + k);
+    if (l <= tl.narrow) {
+      const int lim = vb << l;  // <= 32767 on a narrow level
+      const int e[4] = {v.x, v.y, v.z, v.w};
+      unsigned h[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        bad |= e[t] > lim || e[t] < -lim;
+        h[t] = unsigned(min(max(e[t], -32768), 32767)) & 0xffffu;
+      }
+      reinterpret_cast<uint2*>(row)[c] = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+    } else {
+      reinterpret_cast<int4*>(row)[c] = v;
+    }
+  }
+  if (bad && dev_err) atomicOr(dev_err, ALHR_DEVERR_VALUE_RANGE);
+}
+
+cudaError_t launch_tree_pack(const int32_t* nodes, const TreeLayout& tl, long long bh, int vb,
+                             char* tree, uint32_t* dev_err, cudaStream_t st) {
+  const long long total = bh * (long long)(tl.n - 1) * (tl.d / 4);
+  long long blocks = (total + 255) / 256;
+  if (blocks > 148LL * 64) blocks = 148LL * 64;
+  if (blocks < 1) return cudaSuccess;
+  const int4* src = reinterpret_cast<const int4*>(nodes);
+  if (tl.d == 64)
+    tree_pack_kernel<64><<<unsigned(blocks), 256, 0, st>>>(src, tl, bh, vb, tree, dev_err);
+  else
+    tree_pack_kernel<128><<<unsigned(blocks), 256, 0, st>>>(src, tl, bh, vb, tree, dev_err);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_tree_unpack(const char* tree, const TreeLayout& tl, long long bh,
                                int32_t* nodes, cudaStream_t st) {
   const long long total = bh * (long long)(tl.n - 1) * (tl.d / 4);

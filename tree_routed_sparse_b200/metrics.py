@@ -1,13 +1,17 @@
 """Algorithmic byte model of the ALHR inference path (what the algorithm must touch).
 
 Row sizes: a key row d bytes, a tree row of a narrow level (at d = 128, value_bound * 2^l <=
-32767, stored as int16) 2d bytes, any other tree row 4d bytes. Per query at position i of the fused forward
-(window w, M = i - w + 1 keys before the window):
+32767, stored as int16) 2d bytes, any other tree row 4d bytes. Per query at position i of the
+fused forward (window w, M = i - w + 1 keys before the window):
   q row                         d
-  causal sum G_i (predictor)    the tree rows of the binary decomposition of [0, i+1)
-  remaining descent roots       the blocks of [0, M) not shared with that decomposition (all of
-                                them without the predictor), only when the descent runs (r > 0)
-  selected window keys          nsel_win * d
+  forest roots                  the blocks of [0, M), one row each: always with the predictor
+                                (they and the window keys give the causal sum G_i), else only
+                                when the descent runs (r > 0)
+  window keys                   all min(w, i+1) of them with the predictor (G_i), else only the
+                                nsel_win selected ones: d each
+(g_from_blocks: the warp-per-query kernel at d = 64 forms G_i from the blocks of the binary
+decomposition of [0, i+1) instead; it then reads those rows, the roots below the blocks they
+share only when the descent runs, and only the nsel_win selected window keys.)
   descent                       one left-child row per expanded node (the right child's score
                                 is parent - left): exp_wide * 4d + (exp_hi - exp_wide) * 2d +
                                 exp_l1 * d
@@ -62,13 +66,14 @@ def _highest_bit(x: np.ndarray) -> np.ndarray:
 
 def forward_bytes(positions, n: int, d: int, window: int, count, expansions, budget,
                   predictor: bool, max_keys: int = 96, value_bound: int = 16,
-                  bucket_log: int = 0) -> int:
+                  bucket_log: int = 0, g_from_blocks: bool = False) -> int:
     """Algorithmic bytes of one alhr_forward launch over the given queries.
 
     positions: query positions i (any shape); count, budget: same shape; expansions: [..., 3]
     (level >= 2 expanded, level 1 expanded, expanded with an int32 child row). With leaf
     buckets (bucket_log > 0) the descent runs only when r >> bucket_log > 0, and the keys of the
-    kept buckets are read once more to be scored."""
+    kept buckets are read once more to be scored. g_from_blocks: the rows the d = 64
+    warp-per-query kernel reads for G_i (see the module docstring)."""
     narrow = narrow_levels(n, d, value_bound)
     i = np.asarray(positions, dtype=np.int64).ravel()
     count = np.asarray(count, dtype=np.int64).ravel()
@@ -78,21 +83,24 @@ def forward_bytes(positions, n: int, d: int, window: int, count, expansions, bud
     b_eff = np.minimum(np.minimum(np.maximum(budget, 1), i + 1), max_keys)
     nsel_win = np.minimum(b_eff, nwin)
     r = b_eff - nsel_win
-    A = i + 1
     M = np.maximum(i - window + 1, 0)
-    if predictor:
+    descends = (r >> bucket_log) > 0
+    if predictor and g_from_blocks:
+        A = i + 1
         p = np.where(M > 0, _highest_bit(A ^ M), 62)
         low = (np.int64(2) << np.minimum(p, 61)) - 1
-        g_rows = _rows_bytes(A, d, narrow)
-        rest = M & low
+        g_rows = _rows_bytes(A, d, narrow) + np.where(descends, _rows_bytes(M & low, d, narrow), 0)
+        win_keys = nsel_win * d
+    elif predictor:
+        g_rows = _rows_bytes(M, d, narrow)
+        win_keys = nwin * d
     else:
-        g_rows = np.zeros_like(i)
-        rest = M
-    root_rows = np.where((r >> bucket_log) > 0, _rows_bytes(rest, d, narrow), 0)
+        g_rows = np.where(descends, _rows_bytes(M, d, narrow), 0)
+        win_keys = nsel_win * d
     descent = exp[:, 2] * 4 * d + (exp[:, 0] - exp[:, 2]) * 2 * d + exp[:, 1] * d
     if bucket_log > 0:
         descent = descent + (count - nsel_win) * d
-    per_q = d + g_rows + root_rows + nsel_win * d + descent + count * 2 * d + 4 * d
+    per_q = d + g_rows + win_keys + descent + count * 2 * d + 4 * d
     return int(per_q.sum()) + (64 * d if predictor else 0)
 
 
