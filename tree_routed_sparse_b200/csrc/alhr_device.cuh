@@ -538,28 +538,14 @@ __device__ __forceinline__ void top_r_threshold(const T (&sc)[NS], const int (&d
   }
 }
 
-// Keeps, among the C candidates (r < C <= 32*NS), the r with the largest score, ties to the
-// lower start, and packs them into the front of the buffer. With 64-bit scores the threshold
-// search runs on 32-bit copies whenever every candidate's score fits in 32 bits (one vote per
-// call; the same set either way).
-template <typename S, int NS, bool NORM>
-__device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int lane,
-                                                int norm_l) {
+// Which of the lane's NS candidates (score, descriptor; kLow marks an empty slot) are among the
+// r with the largest score, ties to the lower start (r < the number of candidates). With 64-bit
+// scores the threshold search runs on 32-bit copies whenever every candidate's score fits in 32
+// bits (one vote per call; the same set either way).
+template <typename S, int NS>
+__device__ __forceinline__ void top_r_keep(const S (&sc)[NS], const int (&ds)[NS], int r,
+                                           bool (&keep)[NS]) {
   constexpr S kLow = ScoreLimits<S>::lowest;
-  S sc[NS];
-  int ds[NS];
-#pragma unroll
-  for (int s = 0; s < NS; ++s) {
-    const int e = lane + 32 * s;
-    const bool ok = e < C;
-    Cand<S> cd{0, kLow};
-    if (ok) cd = B.cand.get(e);
-    sc[s] = cd.score;
-    ds[s] = cd.desc;
-    // ranking by means: q . sum / 2^level, scaled by 2^L to stay an exact integer
-    if (NORM && norm_l && ok) sc[s] = sc[s] * (S(1) << (norm_l - desc_level(ds[s])));
-  }
-  bool keep[NS];
   bool narrow = false;
   if constexpr (sizeof(S) == 8) {
     bool fits = true;
@@ -587,6 +573,31 @@ __device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int
     for (int s = 0; s < NS; ++s)
       keep[s] = sc[s] != kLow && (sc[s] > thr || (sc[s] == thr && desc_start(ds[s]) <= cut));
   }
+}
+
+// Keeps, among the C candidates (r < C <= 32*NS), the r with the largest score, ties to the
+// lower start, and packs them into the front of the buffer. With 64-bit scores the threshold
+// search runs on 32-bit copies whenever every candidate's score fits in 32 bits (one vote per
+// call; the same set either way).
+template <typename S, int NS, bool NORM>
+__device__ __forceinline__ void select_top_r_ns(WarpBuf<S>& B, int C, int r, int lane,
+                                                int norm_l) {
+  constexpr S kLow = ScoreLimits<S>::lowest;
+  S sc[NS];
+  int ds[NS];
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    const int e = lane + 32 * s;
+    const bool ok = e < C;
+    Cand<S> cd{0, kLow};
+    if (ok) cd = B.cand.get(e);
+    sc[s] = cd.score;
+    ds[s] = cd.desc;
+    // ranking by means: q . sum / 2^level, scaled by 2^L to stay an exact integer
+    if (NORM && norm_l && ok) sc[s] = sc[s] * (S(1) << (norm_l - desc_level(ds[s])));
+  }
+  bool keep[NS];
+  top_r_keep<S, NS>(sc, ds, r, keep);
   __syncwarp();
   int base = 0;
 #pragma unroll

@@ -46,13 +46,42 @@ struct CtaSmem {
   static constexpr size_t bytes = QuerySmem<S, D, MODE>::w_bytes + sizeof(CtaBuf<S, D>);
 };
 
+// L2 prefetch of the rows the next step may read: the left children of both children of the
+// expanded node at position xi (level lv, start st), i.e. two rows of level lv - 2 (keys when
+// lv = 2). Issued by every lane for its part of the row, as a load of that row would be.
+template <int D>
+__device__ __forceinline__ void prefetch_grandchildren(const char* Th, const int8_t* Kh, int n,
+                                                       int narrow, int bucket, int desc, int sub) {
+  const int lv = desc_level(desc);
+  if (lv - 1 <= bucket || lv < 2) return;  // the children are not expanded
+  const int gl = lv - 2;
+  const int st = desc_start(desc);
+#pragma unroll
+  for (int side = 0; side < 2; ++side) {
+    const int s2 = st + side * (1 << (lv - 1));
+    const char* p;
+    int bytes;
+    if (gl == 0) {
+      p = reinterpret_cast<const char*>(Kh) + (long long)s2 * D;
+      bytes = D;
+    } else {
+      p = Th + tree_row_offset<D>(n, narrow, gl, s2 >> gl);
+      bytes = (D == 128 && gl <= narrow) ? 2 * D : 4 * D;
+    }
+    // the row group's TPR lanes cover the row in 32-byte pieces (a 128-byte line each: a row
+    // is at most 4 lines)
+    for (int off = 128 * sub; off < bytes; off += 128 * Lay<D>::TPR)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(p + off));
+  }
+}
+
 // One pass over CTA-wide positions [base, end) of the expanded-node lists: row group gg takes
 // positions base + gg + u * NG (u < US), loads them all, then scores them. KIND 0: int32 tree
 // rows, 1: int16 tree rows, 2: key rows. A warp without positions in the pass skips it.
 template <int KIND, int US, typename S, int D>
 __device__ __forceinline__ void cta_child_pass(WarpBuf<S>& B, const char* Th, const int8_t* Kh,
                                                const RowQ& q, int base, int end, int warp,
-                                               int gg, int sub) {
+                                               int gg, int sub, int n, int narrow, int bucket) {
   constexpr int RPI = Lay<D>::RPI;
   constexpr int TPR = Lay<D>::TPR;
   constexpr int NG = kCtaWarps * RPI;
@@ -66,6 +95,7 @@ __device__ __forceinline__ void cta_child_pass(WarpBuf<S>& B, const char* Th, co
       if constexpr (KIND == 0) ld_tree<D>(Th + B.xrow[xi], sub, x[u]);
       else if constexpr (KIND == 1) ld_tree16<D>(Th + B.xrow[xi], sub, x[u]);
       else ld_key<D>(Kh + B.xrow[xi], sub, x[u]);
+      prefetch_grandchildren<D>(Th, Kh, n, narrow, bucket, B.xnode.desc(xi), sub);
     } else {
 #pragma unroll
       for (int j = 0; j < WORDS; ++j) x[u][j] = 0;
@@ -131,6 +161,106 @@ __device__ __forceinline__ void gather_values_part(const int* selk, const float*
   }
 }
 
+// Counts of the classified lists of a step: keys (and buckets) in cand[0, nl); nodes to expand in
+// the x lists, [0, nw) with int32 left-child rows, [nw, nw + nn) with int16 ones, then nk with
+// keys as left children.
+struct StepLists {
+  int nl, nw, nn, nk;
+};
+
+// Warp 0's serial part of a descent step, in one pass over registers: the step's candidates
+// (the frontier's keys cand[0, nl) and both children of every expanded node, the right child
+// scored as parent - left), the best `limit` of them when there are more (exact top r, ties to
+// the lower start; rank by means with NORM), and the kept ones written straight into the next
+// step's classified lists. Returns the new counts.
+template <typename S, int D, int NS, bool NORM>
+__device__ __forceinline__ StepLists step_select_classify(WarpBuf<S>& B, int nl, int nx, int limit,
+                                                          int lane, int norm_l, int bucket, int n,
+                                                          int narrow) {
+  constexpr S kLow = ScoreLimits<S>::lowest;
+  constexpr bool kNarrow = (D == 128);
+  const int C = nl + 2 * nx;
+  S sc[NS];   // scores (stored back as they are)
+  S rk[NS];   // ranking values (scores, or scaled to means)
+  int ds[NS];
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    const int e = lane + 32 * s;
+    sc[s] = kLow;
+    ds[s] = 0;
+    if (e < nl) {
+      const Cand<S> cd = B.cand.get(e);
+      sc[s] = cd.score;
+      ds[s] = cd.desc;
+    } else if (e < C) {
+      const int c = e - nl;
+      const Cand<S> p = B.xnode.get(c >> 1);
+      const S left = B.xleft[c >> 1];
+      const int cl = desc_level(p.desc) - 1;
+      const int st = desc_start(p.desc);
+      ds[s] = make_desc((c & 1) ? st + (1 << cl) : st, cl);
+      sc[s] = (c & 1) ? p.score - left : left;
+    }
+    rk[s] = (NORM && norm_l && e < C) ? sc[s] * (S(1) << (norm_l - desc_level(ds[s]))) : sc[s];
+  }
+  bool keep[NS];
+  if (C > limit) {
+    top_r_keep<S, NS>(rk, ds, limit, keep);
+  } else {
+#pragma unroll
+    for (int s = 0; s < NS; ++s) keep[s] = lane + 32 * s < C;
+  }
+  __syncwarp();  // every read of cand / xnode / xleft above is done before the lists are rewritten
+  // classify the kept: 1 key or bucket (stays), 2 int32 left-child row, 3 int16 one, 4 key child
+  int cat[NS];
+  unsigned b1[NS], b2[NS], b3[NS], b4[NS];
+  StepLists o{0, 0, 0, 0};
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    const int lv = desc_level(ds[s]);
+    cat[s] = !keep[s] ? 0 : (lv <= bucket ? 1 : (lv == 1 ? 4 : ((!kNarrow || lv - 1 > narrow) ? 2 : 3)));
+    b1[s] = __ballot_sync(kFull, cat[s] == 1);
+    b2[s] = __ballot_sync(kFull, cat[s] == 2);
+    b3[s] = kNarrow ? __ballot_sync(kFull, cat[s] == 3) : 0u;
+    b4[s] = __ballot_sync(kFull, cat[s] == 4);
+    o.nl += __popc(b1[s]);
+    o.nw += __popc(b2[s]);
+    o.nn += __popc(b3[s]);
+    o.nk += __popc(b4[s]);
+  }
+  const unsigned below = lanemask_lt(lane);
+  int p1 = 0, p2 = 0, p3 = o.nw, p4 = o.nw + o.nn;
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    if (cat[s] == 1) {
+      B.cand.put(p1 + __popc(b1[s] & below), ds[s], sc[s]);
+    } else if (cat[s] >= 2) {
+      const int pos = cat[s] == 2 ? p2 + __popc(b2[s] & below)
+                                  : (cat[s] == 3 ? p3 + __popc(b3[s] & below)
+                                                 : p4 + __popc(b4[s] & below));
+      const int cl = desc_level(ds[s]) - 1;
+      const int st = desc_start(ds[s]);
+      B.xnode.put(pos, ds[s], sc[s]);
+      B.xrow[pos] = cat[s] == 4 ? st * D : tree_row_offset<D>(n, narrow, cl, st >> cl);
+    }
+    p1 += __popc(b1[s]);
+    p2 += __popc(b2[s]);
+    p3 += __popc(b3[s]);
+    p4 += __popc(b4[s]);
+  }
+  __syncwarp();
+  return o;
+}
+
+template <typename S, int D, bool NORM>
+__device__ __forceinline__ StepLists step_select_classify_any(WarpBuf<S>& B, int nl, int nx,
+                                                              int limit, int lane, int norm_l,
+                                                              int bucket, int n, int narrow) {
+  if (nl + 2 * nx <= 96)
+    return step_select_classify<S, D, 3, NORM>(B, nl, nx, limit, lane, norm_l, bucket, n, narrow);
+  return step_select_classify<S, D, 6, NORM>(B, nl, nx, limit, lane, norm_l, bucket, n, narrow);
+}
+
 // VAR compiles in the descent variants (ranking by means, leaf buckets), as in query_kernel.
 template <typename S, int D, int MODE, bool VAR>
 __global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const QueryArgs a) {
@@ -159,6 +289,17 @@ __global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const Quer
   const int sub = lane % TPR;
   const int gg = warp * RPI + grp;  // this lane's row group in the CTA
   if constexpr (kUsesW) stage_weights<D>(a.W, sWg, sWq);
+  // The serial parts run on one warp, chosen to put the serial warps of the CTAs sharing an SM
+  // on different SM sub-partitions (schedulers). A heuristic: if the SM hands a CTA four
+  // consecutive warp slots, one per sub-partition, the CTA whose first slot is 4k takes its warp
+  // k mod 4. Any choice gives the same results; this one only spreads the serial chains.
+  if (threadIdx.x == 0) {
+    unsigned wid;
+    asm volatile("mov.u32 %0, %%warpid;" : "=r"(wid));
+    C.ctl[5] = int((wid >> 2) & (kCtaWarps - 1));
+  }
+  __syncthreads();
+  const int sw = C.ctl[5];
   const int n = a.n;
   const int w = a.window;
   const long long tree_block = a.tl.block_bytes;
@@ -175,7 +316,7 @@ __global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const Quer
 
     RowQ q;
     load_rowq<D>(a.Q + qi * D, sub, q);
-    if (warp == 0) {
+    if (warp == sw) {
       bool bad = false;
 #pragma unroll
       for (int j = 0; j < 16; ++j) bad |= (q.qn[j] > a.value_bound) | (q.qn[j] < -a.value_bound);
@@ -200,7 +341,7 @@ __global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const Quer
     };
     if constexpr (!kUsesW) settle(__ldg(a.budget_in + qi));
 
-    if (warp == 0 && ((Mu >> lane) & 1u))
+    if (warp == sw && ((Mu >> lane) & 1u))
       B.plist[__popc(Mu >> lane) - 1] = make_desc(int((Mu >> lane) << lane) - (1 << lane), lane);
     __syncthreads();
 
@@ -310,115 +451,62 @@ __global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const Quer
         }
         __syncthreads();
       }
-      nf = nR;
-
-      for (int step = 0; step < 32; ++step) {
-        if (warp == 0) {
-          // classify the frontier (as query_kernel): keys stay; expanded nodes go to the x
-          // lists [wide | narrow | key] with the byte offset of their left child's row
-          int fd[kFrontSlots];
-          S fs[kFrontSlots];
-          int cat[kFrontSlots];
-          unsigned bl_[kFrontSlots], bw_[kFrontSlots], bn_[kFrontSlots], bk_[kFrontSlots];
-          int nl = 0, nw = 0, nn = 0, nk = 0;
-#pragma unroll
-          for (int s = 0; s < kFrontSlots; ++s) {
-            cat[s] = 0;
-            bl_[s] = bw_[s] = bn_[s] = bk_[s] = 0u;
-            fd[s] = 0;
-            fs[s] = S(0);
-            if (32 * s < nf) {
-              const int e = lane + 32 * s;
-              if (e < nf) {
-                const Cand<S> cd = B.cand.get(e);
-                fd[s] = cd.desc;
-                fs[s] = cd.score;
-                const int lv = desc_level(fd[s]);
-                cat[s] = lv <= bucket ? 1 : (lv == 1 ? 4 : ((!kNarrow || lv - 1 > narrow) ? 2 : 3));
-              }
-              bl_[s] = __ballot_sync(kFull, cat[s] == 1);
-              bw_[s] = __ballot_sync(kFull, cat[s] == 2);
-              if constexpr (kNarrow) bn_[s] = __ballot_sync(kFull, cat[s] == 3);
-              bk_[s] = __ballot_sync(kFull, cat[s] == 4);
-              nl += __popc(bl_[s]);
-              nw += __popc(bw_[s]);
-              nn += __popc(bn_[s]);
-              nk += __popc(bk_[s]);
-            }
-          }
-          const int nx = nw + nn + nk;
-          if (nx == 0) {
-            if constexpr (VAR) {
-              if (nf > keep) {
-                select_top_r<S, true>(B, nf, keep, lane, norm_l);
-                nf = keep;
-              }
-            }
-          } else {
-            exp_hi += nw + nn;
-            exp_l1 += nk;
-            exp_wide += nw;
-            __syncwarp();
-            const unsigned below = lanemask_lt(lane);
-            int ow = 0, on = nw, ok = nw + nn, ol = 0;
-#pragma unroll
-            for (int s = 0; s < kFrontSlots; ++s) {
-              if (cat[s] >= 2) {
-                const int pos = cat[s] == 2 ? ow + __popc(bw_[s] & below)
-                                            : (cat[s] == 3 ? on + __popc(bn_[s] & below)
-                                                           : ok + __popc(bk_[s] & below));
-                const int cl = desc_level(fd[s]) - 1;
-                const int st = desc_start(fd[s]);
-                B.xnode.put(pos, fd[s], fs[s]);
-                B.xrow[pos] = cat[s] == 4 ? st * D : tree_row_offset<D>(n, narrow, cl, st >> cl);
-              } else if (cat[s] == 1) {
-                B.cand.put(ol + __popc(bl_[s] & below), fd[s], fs[s]);
-              }
-              ow += __popc(bw_[s]);
-              on += __popc(bn_[s]);
-              ok += __popc(bk_[s]);
-              ol += __popc(bl_[s]);
-            }
-          }
-          if (lane == 0) {
-            C.ctl[0] = nw;
-            C.ctl[1] = nn;
-            C.ctl[2] = nk;
-            C.ctl[3] = nl;
-            C.ctl[4] = nf;
-          }
+      // warp 0 classifies the roots (no pruning before the first expansion; with leaf
+      // buckets, roots that are all buckets are pruned to the beam)
+      if (warp == sw) {
+        StepLists o = step_select_classify_any<S, D, VAR>(B, nR, 0, 1 << 30, lane, norm_l, bucket,
+                                                          n, narrow);
+        if constexpr (VAR) {
+          if (o.nw + o.nn + o.nk == 0 && o.nl > keep)
+            o = step_select_classify_any<S, D, true>(B, o.nl, 0, keep, lane, norm_l, bucket, n,
+                                                     narrow);
         }
-        __syncthreads();
-        const int nw = C.ctl[0], nhi = nw + C.ctl[1], nx = nhi + C.ctl[2];
-        if (nx == 0) break;  // CTA-uniform
-        // left children over the CTA's row groups: int32 rows, int16 rows, key rows
-        for (int base = 0; base < nw; base += NG * UW)
-          cta_child_pass<0, UW, S, D>(B, Th, Kh, q, base, nw, warp, gg, sub);
-        if constexpr (kNarrow)
-          for (int base = nw; base < nhi; base += NG * UN)
-            cta_child_pass<1, UN, S, D>(B, Th, Kh, q, base, nhi, warp, gg, sub);
-        for (int base = nhi; base < nx; base += NG * UK)
-          cta_child_pass<2, UK, S, D>(B, Th, Kh, q, base, nx, warp, gg, sub);
-        __syncthreads();
-        if (warp == 0) {
-          const int nl = C.ctl[3];
-          for (int x0 = lane; x0 < nx; x0 += 32)
-            put_children<S>(B, nl, x0, B.xnode.get(x0), B.xleft[x0]);
-          const int Cn = nl + 2 * nx;
-          if (Cn > keep) {
-            select_top_r<S, VAR>(B, Cn, keep, lane, norm_l);
-            nf = keep;
-          } else {
-            nf = Cn;
-            __syncwarp();
-          }
+        exp_hi += o.nw + o.nn;
+        exp_l1 += o.nk;
+        exp_wide += o.nw;
+        if (lane == 0) {
+          C.ctl[0] = o.nw;
+          C.ctl[1] = o.nn;
+          C.ctl[2] = o.nk;
+          C.ctl[3] = o.nl;
         }
       }
-      nf = C.ctl[4];
+      __syncthreads();
+      for (int step = 0; step < 32; ++step) {
+        const int nw = C.ctl[0], nhi = nw + C.ctl[1], nx = nhi + C.ctl[2], nl = C.ctl[3];
+        if (nx == 0) {  // CTA-uniform: every frontier node is a key (or a bucket)
+          nf = nl;
+          break;
+        }
+        // left children over the CTA's row groups: int32 rows, int16 rows, key rows (and an L2
+        // prefetch of the rows the next step may need)
+        for (int base = 0; base < nw; base += NG * UW)
+          cta_child_pass<0, UW, S, D>(B, Th, Kh, q, base, nw, warp, gg, sub, n, narrow, bucket);
+        if constexpr (kNarrow)
+          for (int base = nw; base < nhi; base += NG * UN)
+            cta_child_pass<1, UN, S, D>(B, Th, Kh, q, base, nhi, warp, gg, sub, n, narrow, bucket);
+        for (int base = nhi; base < nx; base += NG * UK)
+          cta_child_pass<2, UK, S, D>(B, Th, Kh, q, base, nx, warp, gg, sub, n, narrow, bucket);
+        __syncthreads();
+        if (warp == sw) {
+          const StepLists o = step_select_classify_any<S, D, VAR>(B, nl, nx, keep, lane, norm_l,
+                                                                  bucket, n, narrow);
+          exp_hi += o.nw + o.nn;
+          exp_l1 += o.nk;
+          exp_wide += o.nw;
+          if (lane == 0) {
+            C.ctl[0] = o.nw;
+            C.ctl[1] = o.nn;
+            C.ctl[2] = o.nk;
+            C.ctl[3] = o.nl;
+          }
+        }
+        __syncthreads();
+      }
       if constexpr (VAR) {
         if (bucket > 0) {
           __syncthreads();  // every warp has read ctl before warp 0 rewrites it
-          if (warp == 0) {
+          if (warp == sw) {
             nf = expand_buckets<S, D>(B, nf, Kh, q, lane);
             if (lane == 0) C.ctl[4] = nf;
           }
@@ -446,7 +534,7 @@ __global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const Quer
 
     // ---- outputs of the route (warp 0)
     const int count = nsel_win + nf;
-    if (warp == 0) {
+    if (warp == sw) {
       if (lane == 0) {
         if (a.count_out) a.count_out[qi] = count;
         if (a.exp_out) {
@@ -462,7 +550,7 @@ __global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const Quer
 
     // ---- 4. exact attention over window + routed keys
     if constexpr (kAttend) {
-      if (warp == 0) {
+      if (warp == sw) {
         const float scale = a.scale;
         const float sw = lane < nsel_win ? float(B.winsc[lane]) * scale : -INFINITY;
         float sr[kFrontSlots];

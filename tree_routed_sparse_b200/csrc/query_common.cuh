@@ -38,20 +38,47 @@ struct QuerySmem {
 };
 
 // Predictor weights into shared memory, in the layout of WLayout (all threads of the CTA take
-// part; the caller synchronises before reading them).
+// part; the caller synchronises before reading them). W is read as 16-byte pieces, every piece
+// of a thread loaded before any is stored (one round trip to memory instead of one per word:
+// this runs at the start of every CTA, so at decode it sits on the critical path).
 template <int D>
 __device__ __forceinline__ void stage_weights(const int8_t* W, int* sWg, int* sWq) {
   constexpr int GS = WLayout<D>::g_stride;
   constexpr int QS = WLayout<D>::q_stride;
-  // word m (dims 4m .. 4m+3) of a class row goes to slot w_slot<D>(m), so that the lanes of a
-  // row group read consecutive slots
-  for (int k = threadIdx.x; k < 32 * D / 4; k += blockDim.x) {
-    const int c = k / (D / 4), m = k - c * (D / 4);
-    sWq[c * QS + w_slot<D>(m)] = __ldg(reinterpret_cast<const int*>(W + c * 2 * D) + m);
-  }
-  for (int k = threadIdx.x; k < 32 * D; k += blockDim.x) {
-    const int c = k / D, t = k - c * D;
-    sWg[c * GS + 4 * w_slot<D>(t >> 2) + (t & 3)] = W[c * 2 * D + D + t];
+  constexpr int kPieces = 32 * 2 * D / 16;  // 16-byte pieces of W [32][2d]
+  constexpr int kPerThread = 8;             // pieces per thread per round (blockDim >= 128)
+  const int4* W4 = reinterpret_cast<const int4*>(W);
+  for (int base = 0; base < kPieces; base += kPerThread * blockDim.x) {
+    int4 v[kPerThread];
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+      const int k = base + u * blockDim.x + threadIdx.x;
+      if (k < kPieces) v[u] = __ldg(W4 + k);
+    }
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+      const int k = base + u * blockDim.x + threadIdx.x;
+      if (k < kPieces) {
+        const int c = k / (2 * D / 16);               // class row
+        const int m0 = (k - c * (2 * D / 16)) * 4;    // first 4-byte word of the piece in the row
+        const int wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int m = m0 + j;  // words 0 .. D/4-1: the q half; D/4 .. D/2-1: the G half
+          if (m < D / 4) {
+            // word m (dims 4m .. 4m+3) goes to slot w_slot<D>(m), so that the lanes of a row
+            // group read consecutive slots
+            sWq[c * QS + w_slot<D>(m)] = wv[j];
+          } else {
+            // the G half, widened to int32: dims t = 4(m - D/4) .. +3
+            const int t = 4 * (m - D / 4);
+            int* g = sWg + c * GS + 4 * w_slot<D>(t >> 2);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) g[e] = sx8(wv[j], e);
+          }
+        }
+      }
+    }
   }
 }
 
