@@ -72,7 +72,14 @@ def parse(argv=None):
                     help="instead of the bench line: time the tree build (alhr_build_tree) on "
                          "the workload's keys (1 GPU)")
     ap.add_argument("--batch", type=int, default=0,
-                    help="with --tree: replace the workload's batch (sequences)")
+                    help="with --tree, --labels or --forward-only: replace the workload's batch "
+                         "(sequences)")
+    ap.add_argument("--n", type=int, default=0,
+                    help="with --forward-only: replace the workload's sequence length (decode "
+                         "workloads keep their one query at position n-1)")
+    ap.add_argument("--forward-only", action="store_true",
+                    help="instead of the bench line: time the fused forward (tree prebuilt, L2 "
+                         "flushed before each launch) on the workload, e.g. one decode launch")
     ap.add_argument("--cpu-steps", type=int, default=4,
                     help="CPU baseline: oracle steps on all host cores (each as a reference step)")
     ap.add_argument("--row-stride", type=int, default=16,
@@ -653,12 +660,57 @@ def run_tree(args):
                       "gpu": torch.cuda.get_device_name(dev)}))
 
 
+def override_workload(wl, args):
+    """The workload with --batch / --n applied (a decode workload keeps its query at n-1)."""
+    if args.batch:
+        wl = wl.replace(batch=args.batch)
+    if args.n:
+        if wl.nq == 1 and wl.q_start == wl.n - 1:
+            wl = wl.replace(n=args.n, q_start=args.n - 1)
+        else:
+            wl = wl.replace(n=args.n, nq=args.n, q_start=0)
+    return wl
+
+
+def run_forward_only(args):
+    """The fused forward alone (tree prebuilt), L2 flushed before every launch: one JSON line with
+    the median launch time, queries per second and the algorithmic bytes' rate."""
+    from tree_routed_sparse_b200 import alhr, synth
+    dev = torch.device("cuda", 0)
+    alhr.set_launch_mode(args.launch_mode)
+    wl = override_workload(synth.WORKLOADS[args.workload], args)
+    vb = max(-wl.qk_lo, wl.qk_hi)
+    inp = synth.make_inputs(wl, dev)
+    kw = dict(q_start=wl.q_start, window=wl.window, max_keys=wl.max_keys,
+              score_bits=wl.score_bits, value_bound=vb)
+    tree = alhr.build_tree(inp["K"], value_bound=vb)
+    out = torch.empty((wl.batch, wl.heads, wl.nq, wl.d), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    run = lambda: alhr.forward(inp["Q"], inp["K"], inp["V"], tree, W=inp["W"],
+                               budget_override=inp["budget_override"], out=out, **kw)
+    for _ in range(args.warmup):
+        run()
+    t = _event_time(run, max(args.steps, 3), flush)
+    full = alhr.forward(inp["Q"], inp["K"], inp["V"], tree, W=inp["W"],
+                        budget_override=inp["budget_override"], want_count=True,
+                        want_expansions=True, want_budget=True, **kw)
+    torch.cuda.synchronize()
+    fb, kb = fwd_algorithmic_bytes(wl, full, vb, takes_warp_shape(wl.bh * wl.nq, dev)
+                                   if args.launch_mode == "auto" else args.launch_mode == "throughput")
+    q = wl.bh * wl.nq
+    print(json.dumps({"report": "forward", "workload": describe(wl), "launch_mode": args.launch_mode,
+                      "queries": q, "us": t * 1e6, "queries_per_s": q / t,
+                      "mean_keys_per_query": float(full["count"].float().mean()),
+                      "algorithmic_bytes": fb, "kernel_row_bytes": kb,
+                      "algorithmic_GBps": fb / t / 1e9, "gpu": torch.cuda.get_device_name(dev)}))
+
+
 def run_labels(args):
     """The phase-2 label kernel on the workload's Q and K: one JSON line with its time, the
     causal scores it ranks per second and the int8 tensor operations it issues."""
     from tree_routed_sparse_b200 import alhr, synth
     dev = torch.device("cuda", 0)
-    wl = synth.WORKLOADS[args.workload]
+    wl = override_workload(synth.WORKLOADS[args.workload], args)
     inp = synth.make_inputs(wl, dev)
     Q, K = inp["Q"], inp["K"]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -765,12 +817,13 @@ def main(argv=None):
     if args.impl == "reference":
         run_reference(args)
         return
-    if args.labels or args.tree or args.stages:
+    if args.labels or args.tree or args.stages or args.forward_only:
         if not torch.cuda.is_available():
             raise SystemExit("bench.py needs a CUDA device")
         from tree_routed_sparse_b200 import build
         build.build()
-        (run_labels if args.labels else run_tree if args.tree else run_stages)(args)
+        (run_labels if args.labels else run_tree if args.tree else
+         run_forward_only if args.forward_only else run_stages)(args)
         return
 
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:

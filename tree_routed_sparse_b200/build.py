@@ -45,7 +45,7 @@ def _hash() -> str:
     return h.hexdigest()
 
 
-HEADERS = ["alhr_device.cuh", "internal.h", "tree_layout.h"]
+HEADERS = ["alhr_device.cuh", "internal.h", "tree_layout.h", "query_common.cuh"]
 
 
 def code_only(text: str) -> str:
