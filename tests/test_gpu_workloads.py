@@ -129,3 +129,32 @@ def test_largest_sequence_decode_and_update(alhr):
     K2[:, :, n - 1] = -K2[:, :, n - 1]
     alhr.update_tree(K2, tree, n - 1, n)
     assert torch.equal(tree, alhr.build_tree(K2))
+
+
+@pytest.mark.parametrize("d,bits", [(128, 64), (64, 32)])
+def test_mid_size_decode_launch(alhr, d, bits):
+    """768 decode queries: more than the four-warp CTA shape holds at once on a B200 (4 per SM),
+    so the latency shape runs two warps per query; auto and forced latency mode both take it.
+    Sampled blocks against the oracle (bit-exact index sets, budgets, counts, expansions)."""
+    from tree_routed_sparse_b200 import synth
+    n = 4096
+    wl = synth.WORKLOADS["decode_s64h8_n262144_d128"].replace(batch=96, n=n, d=d, q_start=n - 1,
+                                                              score_bits=bits, seed=5)
+    inp = synth.make_inputs(wl, "cuda")
+    tree = alhr.build_tree(inp["K"])
+    kw = dict(q_start=wl.q_start, window=wl.window, max_keys=wl.max_keys, score_bits=bits)
+    cpu = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
+    rng = np.random.default_rng(3)
+    blocks = [(0, 0), (95, 7)] + [tuple(x) for x in zip(rng.integers(0, 96, 10),
+                                                        rng.integers(0, 8, 10))]
+    refs = {bh: oracle_slice(cpu, wl, bh[0], bh[1]) for bh in blocks}
+    for shape in ("auto", "latency"):
+        alhr.set_launch_mode(shape)
+        try:
+            res = alhr.forward(inp["Q"], inp["K"], inp["V"], tree, W=inp["W"], want_idx=True,
+                               want_count=True, want_expansions=True, want_budget=True, **kw)
+            torch.cuda.synchronize()
+        finally:
+            alhr.set_launch_mode("auto")
+        for (b, h), ref in refs.items():
+            compare_rows(res, ref, b, h, np.arange(1), TOL, f"768 queries {shape} d={d} {(b, h)}")

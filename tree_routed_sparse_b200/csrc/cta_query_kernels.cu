@@ -18,32 +18,36 @@
 
 namespace alhr {
 
+// Warps per query: four for launches whose queries all fit the GPU at once as CTAs of four
+// warps (at most four per SM), two for launches up to about twice that size (so that those
+// too are resident at once, at half the row parallelism per query).
 constexpr int kCtaWarps = 4;
+constexpr int kCtaWarpsWide = 2;
 
 // Shared state of one query: the warp-per-query buffer (used here by the whole CTA) plus the
 // cross-warp partial sums and the counts warp 0 hands to the others.
-template <typename S, int D>
+template <typename S, int D, int NWC>
 struct CtaBuf {
   WarpBuf<S> B;
-  long long logit[32];                    // class logits of the predictor
-  alignas(16) int gpart[kCtaWarps][D];    // per-warp partial sums of G_i (lane-slot order:
-                                          // sub * 16 + j), read and written as int4
-  alignas(16) float opart[kCtaWarps][D];  // per-warp partial sums of the output row (float4)
+  long long logit[32];              // class logits of the predictor
+  alignas(16) int gpart[NWC][D];    // per-warp partial sums of G_i (lane-slot order:
+                                    // sub * 16 + j), read and written as int4
+  alignas(16) float opart[NWC][D];  // per-warp partial sums of the output row (float4)
   int ctl[8];                             // counts of a descent step (wide, narrow, key, leaf, nf)
   float inv;                              // 1 / softmax denominator
 };
 // the 16-byte accesses above need 16-byte offsets
-using CtaBufI64 = CtaBuf<int, 64>;
-using CtaBufL128 = CtaBuf<long long, 128>;
+using CtaBufI64 = CtaBuf<int, 64, kCtaWarps>;
+using CtaBufL128 = CtaBuf<long long, 128, kCtaWarpsWide>;
 static_assert(offsetof(CtaBufI64, gpart) % 16 == 0 && offsetof(CtaBufI64, opart) % 16 == 0,
               "CtaBuf alignment");
 static_assert(offsetof(CtaBufL128, gpart) % 16 == 0 && offsetof(CtaBufL128, opart) % 16 == 0,
               "CtaBuf alignment");
 
-template <typename S, int D, int MODE>
+template <typename S, int D, int MODE, int NWC>
 struct CtaSmem {
   static_assert(QuerySmem<S, D, MODE>::w_bytes % 16 == 0, "CtaBuf placement");
-  static constexpr size_t bytes = QuerySmem<S, D, MODE>::w_bytes + sizeof(CtaBuf<S, D>);
+  static constexpr size_t bytes = QuerySmem<S, D, MODE>::w_bytes + sizeof(CtaBuf<S, D, NWC>);
 };
 
 // L2 prefetch of the rows the next step may read: the left children of both children of the
@@ -78,13 +82,13 @@ __device__ __forceinline__ void prefetch_grandchildren(const char* Th, const int
 // One pass over CTA-wide positions [base, end) of the expanded-node lists: row group gg takes
 // positions base + gg + u * NG (u < US), loads them all, then scores them. KIND 0: int32 tree
 // rows, 1: int16 tree rows, 2: key rows. A warp without positions in the pass skips it.
-template <int KIND, int US, typename S, int D>
+template <int KIND, int US, typename S, int D, int NWC>
 __device__ __forceinline__ void cta_child_pass(WarpBuf<S>& B, const char* Th, const int8_t* Kh,
                                                const RowQ& q, int base, int end, int warp,
                                                int gg, int sub, int n, int narrow, int bucket) {
   constexpr int RPI = Lay<D>::RPI;
   constexpr int TPR = Lay<D>::TPR;
-  constexpr int NG = kCtaWarps * RPI;
+  constexpr int NG = NWC * RPI;
   if (base + warp * RPI >= end) return;  // warp-uniform
   constexpr int WORDS = KIND == 0 ? 16 : (KIND == 1 ? 8 : 4);
   int x[US][WORDS];
@@ -262,11 +266,11 @@ __device__ __forceinline__ StepLists step_select_classify_any(WarpBuf<S>& B, int
 }
 
 // VAR compiles in the descent variants (ranking by means, leaf buckets), as in query_kernel.
-template <typename S, int D, int MODE, bool VAR>
-__global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const QueryArgs a) {
+template <typename S, int D, int MODE, bool VAR, int NWC>
+__global__ void __launch_bounds__(NWC * 32, 16 / NWC) cta_query_kernel(const QueryArgs a) {
   constexpr int TPR = Lay<D>::TPR;
   constexpr int RPI = Lay<D>::RPI;
-  constexpr int NG = kCtaWarps * RPI;  // row groups of the CTA
+  constexpr int NG = NWC * RPI;  // row groups of the CTA
   constexpr bool kUsesW = (MODE == kForwardPredict || MODE == kPredictOnly);
   constexpr bool kDescend = (MODE != kPredictOnly);
   constexpr bool kAttend = (MODE == kForwardPredict || MODE == kForwardOverride);
@@ -280,7 +284,8 @@ __global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const Quer
   extern __shared__ __align__(16) unsigned char smem_raw[];
   int* sWg = reinterpret_cast<int*>(smem_raw);
   int* sWq = sWg + 32 * WLayout<D>::g_stride;
-  CtaBuf<S, D>& C = *reinterpret_cast<CtaBuf<S, D>*>(smem_raw + QuerySmem<S, D, MODE>::w_bytes);
+  CtaBuf<S, D, NWC>& C =
+      *reinterpret_cast<CtaBuf<S, D, NWC>*>(smem_raw + QuerySmem<S, D, MODE>::w_bytes);
   WarpBuf<S>& B = C.B;
 
   const int lane = threadIdx.x & 31;
@@ -296,7 +301,7 @@ __global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const Quer
   if (threadIdx.x == 0) {
     unsigned wid;
     asm volatile("mov.u32 %0, %%warpid;" : "=r"(wid));
-    C.ctl[5] = int((wid >> 2) & (kCtaWarps - 1));
+    C.ctl[5] = int((wid / 4) % NWC);
   }
   __syncthreads();
   const int sw = C.ctl[5];
@@ -353,26 +358,37 @@ __global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const Quer
 #pragma unroll
       for (int j = 0; j < 16; ++j) G[j] = 0;
       S rsc[U1];
-      {
-        int x[U1][16];
+      // rounds of up to 4 rows per group in flight (one round with four warps per query)
+      constexpr int UG = U1 < 4 ? U1 : 4;
 #pragma unroll
-        for (int u = 0; u < U1; ++u) {
-          const int k = u * NG + gg;
+      for (int u0 = 0; u0 < U1; u0 += UG) {
+        if (u0 * NG < nI) {  // CTA-uniform
+          int x[UG][16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) x[u][j] = 0;
-          if (k < nI)
-            ld_node32<D, kNarrow>(Th, Kh, n, narrow,
-                                  k < nR ? B.plist[k] : make_desc(i - (k - nR), 0), sub, x[u]);
-        }
-        __syncwarp();
+          for (int uu = 0; uu < UG; ++uu) {
+            const int k = (u0 + uu) * NG + gg;
 #pragma unroll
-        for (int u = 0; u < U1; ++u) {
-          rsc[u] = S(0);
-          if (u * NG < nI) {  // CTA-uniform
-#pragma unroll
-            for (int j = 0; j < 16; ++j) G[j] += x[u][j];
-            rsc[u] = group_sum<S, TPR>(dot_tree<S>(q, x[u]));
+            for (int j = 0; j < 16; ++j) x[uu][j] = 0;
+            if (u0 + uu < U1 && k < nI)
+              ld_node32<D, kNarrow>(Th, Kh, n, narrow,
+                                    k < nR ? B.plist[k] : make_desc(i - (k - nR), 0), sub, x[uu]);
           }
+          __syncwarp();
+#pragma unroll
+          for (int uu = 0; uu < UG; ++uu) {
+            if (u0 + uu < U1) {
+              rsc[u0 + uu] = S(0);
+              if ((u0 + uu) * NG < nI) {  // CTA-uniform
+#pragma unroll
+                for (int j = 0; j < 16; ++j) G[j] += x[uu][j];
+                rsc[u0 + uu] = group_sum<S, TPR>(dot_tree<S>(q, x[uu]));
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int uu = 0; uu < UG; ++uu)
+            if (u0 + uu < U1) rsc[u0 + uu] = S(0);
         }
       }
 #pragma unroll
@@ -396,7 +412,7 @@ __global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const Quer
 #pragma unroll
       for (int j = 0; j < 16; ++j) G[j] = 0;
 #pragma unroll
-      for (int ww = 0; ww < kCtaWarps; ++ww) {
+      for (int ww = 0; ww < NWC; ++ww) {
         const int4* gp = reinterpret_cast<const int4*>(&C.gpart[ww][sub * 16]);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
@@ -481,12 +497,12 @@ __global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const Quer
         // left children over the CTA's row groups: int32 rows, int16 rows, key rows (and an L2
         // prefetch of the rows the next step may need)
         for (int base = 0; base < nw; base += NG * UW)
-          cta_child_pass<0, UW, S, D>(B, Th, Kh, q, base, nw, warp, gg, sub, n, narrow, bucket);
+          cta_child_pass<0, UW, S, D, NWC>(B, Th, Kh, q, base, nw, warp, gg, sub, n, narrow, bucket);
         if constexpr (kNarrow)
           for (int base = nw; base < nhi; base += NG * UN)
-            cta_child_pass<1, UN, S, D>(B, Th, Kh, q, base, nhi, warp, gg, sub, n, narrow, bucket);
+            cta_child_pass<1, UN, S, D, NWC>(B, Th, Kh, q, base, nhi, warp, gg, sub, n, narrow, bucket);
         for (int base = nhi; base < nx; base += NG * UK)
-          cta_child_pass<2, UK, S, D>(B, Th, Kh, q, base, nx, warp, gg, sub, n, narrow, bucket);
+          cta_child_pass<2, UK, S, D, NWC>(B, Th, Kh, q, base, nx, warp, gg, sub, n, narrow, bucket);
         __syncthreads();
         if (warp == sw) {
           const StepLists o = step_select_classify_any<S, D, VAR>(B, nl, nx, keep, lane, norm_l,
@@ -591,16 +607,16 @@ __global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const Quer
         if (lane == 0) C.inv = 1.f / den;
       }
       __syncthreads();
-      const int per = (count + kCtaWarps - 1) / kCtaWarps;
+      const int per = (count + NWC - 1) / NWC;
       const int k0 = min(count, warp * per);
       gather_values_part<D, 2>(B.selk, B.selp, k0, min(count, k0 + per),
                                a.V + bh * (long long)n * D, lane, C.opart[warp]);
       __syncthreads();
       const float inv = C.inv;
-      for (int t = threadIdx.x; t < D; t += kCtaWarps * 32) {
+      for (int t = threadIdx.x; t < D; t += NWC * 32) {
         float o = 0.f;
 #pragma unroll
-        for (int ww = 0; ww < kCtaWarps; ++ww) o += C.opart[ww][t];
+        for (int ww = 0; ww < NWC; ++ww) o += C.opart[ww][t];
         a.out[qi * D + t] = o * inv;
       }
     }
@@ -609,10 +625,11 @@ __global__ void __launch_bounds__(kCtaWarps * 32, 4) cta_query_kernel(const Quer
 
 namespace {
 
-template <typename S, int D, int MODE, bool VAR>
-cudaError_t launch_cta_mode(const QueryArgs& a, cudaStream_t st) {
-  constexpr size_t smem = CtaSmem<S, D, MODE>::bytes;
-  auto kern = cta_query_kernel<S, D, MODE, VAR>;
+// Resident CTAs per SM of one instantiation (cached per device) and, with `launch`, the launch.
+template <typename S, int D, int MODE, bool VAR, int NWC>
+cudaError_t cta_mode(const QueryArgs& a, cudaStream_t st, bool launch, long long* per_sm_out) {
+  constexpr size_t smem = CtaSmem<S, D, MODE, NWC>::bytes;
+  auto kern = cta_query_kernel<S, D, MODE, VAR, NWC>;
   static thread_local int cached_dev = -1;
   static thread_local int per_sm = 0, sms = 0;
   int dev = 0;
@@ -625,42 +642,68 @@ cudaError_t launch_cta_mode(const QueryArgs& a, cudaStream_t st) {
     }
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int b = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, kCtaWarps * 32, smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, NWC * 32, smem);
     per_sm = b > 0 ? b : 1;
     cached_dev = dev;
   }
   const long long cap = (long long)sms * per_sm;
+  if (per_sm_out) *per_sm_out = cap;
+  if (!launch) return cudaSuccess;
   const int blocks = int(a.num_queries < cap ? a.num_queries : cap);
   if (blocks <= 0) return cudaSuccess;
-  kern<<<blocks, kCtaWarps * 32, smem, st>>>(a);
+  kern<<<blocks, NWC * 32, smem, st>>>(a);
   return cudaGetLastError();
 }
 
+// Four warps per query while every query fits at once that way; else two while they fit; else,
+// when `forced` is false, nothing is launched (*launched = false: the caller takes the
+// throughput shape); when forced, four warps per query in several waves.
 template <typename S, int D, int MODE>
-cudaError_t launch_cta_variant(const QueryArgs& a, cudaStream_t st) {
-  if (MODE != kPredictOnly && (a.norm_l != 0 || a.bucket != 0))
-    return launch_cta_mode<S, D, MODE, MODE != kPredictOnly>(a, st);
-  return launch_cta_mode<S, D, MODE, false>(a, st);
+cudaError_t cta_dispatch(const QueryArgs& a, cudaStream_t st, bool forced, bool* launched) {
+  const bool var = MODE != kPredictOnly && (a.norm_l != 0 || a.bucket != 0);
+  long long cap4 = 0;
+  cudaError_t e = var ? cta_mode<S, D, MODE, true, kCtaWarps>(a, st, false, &cap4)
+                      : cta_mode<S, D, MODE, false, kCtaWarps>(a, st, false, &cap4);
+  if (e != cudaSuccess) return e;
+  *launched = true;
+  if (a.num_queries <= cap4 || var) {
+    if (a.num_queries > cap4 && !forced) {
+      *launched = false;
+      return cudaSuccess;
+    }
+    return var ? cta_mode<S, D, MODE, true, kCtaWarps>(a, st, true, nullptr)
+               : cta_mode<S, D, MODE, false, kCtaWarps>(a, st, true, nullptr);
+  }
+  long long cap2 = 0;
+  e = cta_mode<S, D, MODE, false, kCtaWarpsWide>(a, st, false, &cap2);
+  if (e != cudaSuccess) return e;
+  if (a.num_queries <= cap2) return cta_mode<S, D, MODE, false, kCtaWarpsWide>(a, st, true, nullptr);
+  if (!forced) {
+    *launched = false;
+    return cudaSuccess;
+  }
+  return cta_mode<S, D, MODE, false, kCtaWarps>(a, st, true, nullptr);
 }
 
 template <int MODE>
-cudaError_t dispatch_cta(const QueryArgs& a, int d, int score_bits, cudaStream_t st) {
+cudaError_t dispatch_cta(const QueryArgs& a, int d, int score_bits, cudaStream_t st, bool forced,
+                         bool* launched) {
   if (d == 64)
-    return score_bits == 32 ? launch_cta_variant<int, 64, MODE>(a, st)
-                            : launch_cta_variant<long long, 64, MODE>(a, st);
-  return score_bits == 32 ? launch_cta_variant<int, 128, MODE>(a, st)
-                          : launch_cta_variant<long long, 128, MODE>(a, st);
+    return score_bits == 32 ? cta_dispatch<int, 64, MODE>(a, st, forced, launched)
+                            : cta_dispatch<long long, 64, MODE>(a, st, forced, launched);
+  return score_bits == 32 ? cta_dispatch<int, 128, MODE>(a, st, forced, launched)
+                          : cta_dispatch<long long, 128, MODE>(a, st, forced, launched);
 }
 
 }  // namespace
 
-cudaError_t launch_query_cta(const QueryArgs& a, int d, int score_bits, int mode,
-                             cudaStream_t st) {
+cudaError_t launch_query_cta(const QueryArgs& a, int d, int score_bits, int mode, bool forced,
+                             bool* launched, cudaStream_t st) {
   switch (mode) {
-    case kForwardPredict: return dispatch_cta<kForwardPredict>(a, d, score_bits, st);
-    case kForwardOverride: return dispatch_cta<kForwardOverride>(a, d, score_bits, st);
-    case kRouteOnly: return dispatch_cta<kRouteOnly>(a, d, score_bits, st);
-    default: return dispatch_cta<kPredictOnly>(a, d, score_bits, st);
+    case kForwardPredict: return dispatch_cta<kForwardPredict>(a, d, score_bits, st, forced, launched);
+    case kForwardOverride: return dispatch_cta<kForwardOverride>(a, d, score_bits, st, forced, launched);
+    case kRouteOnly: return dispatch_cta<kRouteOnly>(a, d, score_bits, st, forced, launched);
+    default: return dispatch_cta<kPredictOnly>(a, d, score_bits, st, forced, launched);
   }
 }
 

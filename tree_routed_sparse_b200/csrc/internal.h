@@ -32,9 +32,10 @@ cudaError_t launch_route(const QueryArgs& a, int d, int score_bits, cudaStream_t
 cudaError_t launch_predict(const QueryArgs& a, int d, int score_bits, cudaStream_t st);
 cudaError_t launch_attend(const QueryArgs& a, int d, cudaStream_t st);
 // The latency shape: one query per CTA (see cta_query_kernels.cu); mode is a Mode of
-// query_common.cuh.
-cudaError_t launch_query_cta(const QueryArgs& a, int d, int score_bits, int mode,
-                             cudaStream_t st);
+// query_common.cuh. Unless `forced`, it launches only when every query is resident at once
+// (*launched tells whether it launched; if not, the caller takes the throughput shape).
+cudaError_t launch_query_cta(const QueryArgs& a, int d, int score_bits, int mode, bool forced,
+                             bool* launched, cudaStream_t st);
 
 // Phase-2 labels: top-k keys of every query's causal q . K row (see label_kernels.cu).
 cudaError_t launch_topk_labels(const int8_t* Q, const int8_t* K, int32_t* labels,

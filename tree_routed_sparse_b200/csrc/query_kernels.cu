@@ -632,7 +632,6 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(const QueryArgs a) 
 namespace {
 
 constexpr int kOccSlots = 66;
-constexpr int kLatCtasPerSm = 4;  // resident CTAs of the latency shape per SM
 
 // Grid size of a persistent launch: the resident CTAs of every SM, capped by the work. The
 // per-device occupancy (and the opt-in to more than 48 KB of dynamic shared memory) is
@@ -683,23 +682,18 @@ cudaError_t launch_query_mode(const QueryArgs& a, cudaStream_t st) {
 
 std::atomic<int> g_launch_mode{0};
 
-// Auto: a launch whose queries all fit the GPU as one CTA each (the latency shape, four CTAs per
-// SM) takes that shape; larger launches take one warp per query.
+// Auto: a launch whose queries are all resident at once as one CTA each (latency shape: four
+// warps per query up to four CTAs per SM, two warps per query beyond that) takes that shape;
+// larger launches take one warp per query. The latency mode forces the CTA shape.
 template <typename S, int D, int MODE>
 cudaError_t launch_query(const QueryArgs& a, cudaStream_t st) {
   const int mode = g_launch_mode.load(std::memory_order_relaxed);
-  bool lat = mode == 2;
-  if (mode == 0) {
-    static thread_local int cached_dev = -1, sms = 148;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev != cached_dev) {
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-      cached_dev = dev;
-    }
-    lat = a.num_queries <= (long long)sms * kLatCtasPerSm;
+  if (mode != 1) {
+    bool launched = false;
+    const cudaError_t e =
+        launch_query_cta(a, D, sizeof(S) == 4 ? 32 : 64, MODE, mode == 2, &launched, st);
+    if (e != cudaSuccess || launched) return e;
   }
-  if (lat) return launch_query_cta(a, D, sizeof(S) == 4 ? 32 : 64, MODE, st);
   // the predictor alone never descends: it needs no variant instantiation
   if (MODE != kPredictOnly && (a.norm_l != 0 || a.bucket != 0))
     return launch_query_mode<S, D, MODE, MODE != kPredictOnly>(a, st);
