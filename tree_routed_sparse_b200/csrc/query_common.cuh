@@ -185,4 +185,104 @@ __device__ __forceinline__ void ld_node32(const char* Th, const int8_t* Kh, int 
   }
 }
 
+// Counts of the classified lists of a step: keys (and buckets) in cand[0, nl); nodes to expand in
+// the x lists, [0, nw) with int32 left-child rows, [nw, nw + nn) with int16 ones, then nk with
+// keys as left children.
+struct StepLists {
+  int nl, nw, nn, nk;
+};
+
+// Warp 0's serial part of a descent step, in one pass over registers: the step's candidates
+// (the frontier's keys cand[0, nl) and both children of every expanded node, the right child
+// scored as parent - left), the best `limit` of them when there are more (exact top r, ties to
+// the lower start; rank by means with NORM), and the kept ones written straight into the next
+// step's classified lists. Returns the new counts.
+template <typename S, int D, int NS, bool NORM>
+__device__ __forceinline__ StepLists step_select_classify(WarpBuf<S>& B, int nl, int nx, int limit,
+                                                          int lane, int norm_l, int bucket, int n,
+                                                          int narrow) {
+  constexpr S kLow = ScoreLimits<S>::lowest;
+  constexpr bool kNarrow = (D == 128);
+  const int C = nl + 2 * nx;
+  S sc[NS];   // scores (stored back as they are)
+  S rk[NS];   // ranking values (scores, or scaled to means)
+  int ds[NS];
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    const int e = lane + 32 * s;
+    sc[s] = kLow;
+    ds[s] = 0;
+    if (e < nl) {
+      const Cand<S> cd = B.cand.get(e);
+      sc[s] = cd.score;
+      ds[s] = cd.desc;
+    } else if (e < C) {
+      const int c = e - nl;
+      const Cand<S> p = B.xnode.get(c >> 1);
+      const S left = B.xleft[c >> 1];
+      const int cl = desc_level(p.desc) - 1;
+      const int st = desc_start(p.desc);
+      ds[s] = make_desc((c & 1) ? st + (1 << cl) : st, cl);
+      sc[s] = (c & 1) ? p.score - left : left;
+    }
+    rk[s] = (NORM && norm_l && e < C) ? sc[s] * (S(1) << (norm_l - desc_level(ds[s]))) : sc[s];
+  }
+  bool keep[NS];
+  if (C > limit) {
+    top_r_keep<S, NS>(rk, ds, limit, keep);
+  } else {
+#pragma unroll
+    for (int s = 0; s < NS; ++s) keep[s] = lane + 32 * s < C;
+  }
+  __syncwarp();  // every read of cand / xnode / xleft above is done before the lists are rewritten
+  // classify the kept: 1 key or bucket (stays), 2 int32 left-child row, 3 int16 one, 4 key child
+  int cat[NS];
+  unsigned b1[NS], b2[NS], b3[NS], b4[NS];
+  StepLists o{0, 0, 0, 0};
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    const int lv = desc_level(ds[s]);
+    cat[s] = !keep[s] ? 0 : (lv <= bucket ? 1 : (lv == 1 ? 4 : ((!kNarrow || lv - 1 > narrow) ? 2 : 3)));
+    b1[s] = __ballot_sync(kFull, cat[s] == 1);
+    b2[s] = __ballot_sync(kFull, cat[s] == 2);
+    b3[s] = kNarrow ? __ballot_sync(kFull, cat[s] == 3) : 0u;
+    b4[s] = __ballot_sync(kFull, cat[s] == 4);
+    o.nl += __popc(b1[s]);
+    o.nw += __popc(b2[s]);
+    o.nn += __popc(b3[s]);
+    o.nk += __popc(b4[s]);
+  }
+  const unsigned below = lanemask_lt(lane);
+  int p1 = 0, p2 = 0, p3 = o.nw, p4 = o.nw + o.nn;
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    if (cat[s] == 1) {
+      B.cand.put(p1 + __popc(b1[s] & below), ds[s], sc[s]);
+    } else if (cat[s] >= 2) {
+      const int pos = cat[s] == 2 ? p2 + __popc(b2[s] & below)
+                                  : (cat[s] == 3 ? p3 + __popc(b3[s] & below)
+                                                 : p4 + __popc(b4[s] & below));
+      const int cl = desc_level(ds[s]) - 1;
+      const int st = desc_start(ds[s]);
+      B.xnode.put(pos, ds[s], sc[s]);
+      B.xrow[pos] = cat[s] == 4 ? st * D : tree_row_offset<D>(n, narrow, cl, st >> cl);
+    }
+    p1 += __popc(b1[s]);
+    p2 += __popc(b2[s]);
+    p3 += __popc(b3[s]);
+    p4 += __popc(b4[s]);
+  }
+  __syncwarp();
+  return o;
+}
+
+template <typename S, int D, bool NORM>
+__device__ __forceinline__ StepLists step_select_classify_any(WarpBuf<S>& B, int nl, int nx,
+                                                              int limit, int lane, int norm_l,
+                                                              int bucket, int n, int narrow) {
+  if (nl + 2 * nx <= 96)
+    return step_select_classify<S, D, 3, NORM>(B, nl, nx, limit, lane, norm_l, bucket, n, narrow);
+  return step_select_classify<S, D, 6, NORM>(B, nl, nx, limit, lane, norm_l, bucket, n, narrow);
+}
+
 }  // namespace alhr
