@@ -158,3 +158,36 @@ def test_mid_size_decode_launch(alhr, d, bits):
             alhr.set_launch_mode("auto")
         for (b, h), ref in refs.items():
             compare_rows(res, ref, b, h, np.arange(1), TOL, f"768 queries {shape} d={d} {(b, h)}")
+
+
+@pytest.mark.parametrize("d,bits", [(128, 64), (64, 0)])
+def test_mid_size_route_predict_override(alhr, d, bits):
+    """The other entry points at 768 queries (the two-warp CTA shape): alhr_predict_budget,
+    alhr_route (with expansions) and alhr_forward with a budget override, against the oracle
+    on sampled blocks."""
+    from tree_routed_sparse_b200 import synth
+    n = 2048
+    wl = synth.WORKLOADS["decode_s64h8_n262144_d128"].replace(batch=96, n=n, d=d, q_start=n - 1,
+                                                              score_bits=bits, seed=9)
+    inp = synth.make_inputs(wl, "cuda")
+    tree = alhr.build_tree(inp["K"])
+    kw = dict(q_start=wl.q_start, window=wl.window, max_keys=wl.max_keys, score_bits=bits)
+    budget = alhr.predict_budget(inp["Q"], inp["K"], tree, inp["W"], **kw)
+    r = alhr.route(inp["Q"], inp["K"], tree, budget, **kw)
+    # an override budget of 3..96 keys, different from the predicted one
+    bo = ((torch.arange(wl.bh, device="cuda", dtype=torch.int32) * 7) % 96 + 1).view(
+        wl.batch, wl.heads, 1).contiguous()
+    f = alhr.forward(inp["Q"], inp["K"], inp["V"], tree, budget_override=bo, want_idx=True,
+                     want_count=True, want_expansions=True, **kw)
+    torch.cuda.synchronize()
+    cpu = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
+    rng = np.random.default_rng(4)
+    for b, h in [(0, 0), (95, 7)] + [tuple(x) for x in zip(rng.integers(0, 96, 8),
+                                                           rng.integers(0, 8, 8))]:
+        ref = oracle_slice(cpu, wl, b, h)
+        assert int(budget[b, h, 0]) == int(ref["budget"][0]), (b, h)
+        compare_rows({"idx": r["idx"], "count": r["count"], "expansions": r["expansions"]},
+                     ref, b, h, np.arange(1), TOL, f"route 768 d={d} {(b, h)}")
+        cpu_bo = dict(cpu, W=None, budget_override=bo.cpu())
+        ref_o = oracle_slice(cpu_bo, wl.replace(predictor=False), b, h)
+        compare_rows(f, ref_o, b, h, np.arange(1), TOL, f"override 768 d={d} {(b, h)}")
