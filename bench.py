@@ -274,9 +274,10 @@ def oracle_single_thread(wl, inp) -> dict:
 
 # ------------------------------------------------------------------ the GPU arm
 
-# resident CTAs per SM of the latency shape (one query per CTA); launches of at most this many
-# queries per SM take it under the automatic launch mode, larger ones the warp-per-query shape
-LAT_CTAS_PER_SM = 4
+# The latency shape (one query per CTA) takes launches whose queries are all resident at once:
+# four warps per query up to 4 CTAs per SM, two warps per query up to 8 per SM (7 where shared
+# memory runs out first); larger launches take the warp-per-query shape.
+LAT_CTAS_PER_SM = 8
 
 
 def takes_warp_shape(queries: int, dev) -> bool:

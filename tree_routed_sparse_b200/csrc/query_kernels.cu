@@ -235,9 +235,10 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>())
             }
           }
           sc = group_sum<S, TPR>(sc);
-          if (active && sub == 0 && (pd & kFlagRoot)) {
-            B.cand.put(k, pd & ~kFlagRoot, sc);  // the shared roots are the first ones
-          }
+          // the shared roots are the first ones; every lane stores (the same value per row
+          // group; rows that are no roots into a spare slot), so no divergent store precedes the
+          // cross-group sum of G_i below
+          B.cand.put((active && (pd & kFlagRoot)) ? k : kMaxCand - 1, pd & ~kFlagRoot, sc);
         }
       } else {
         // the forest roots, largest first
