@@ -80,3 +80,64 @@ def test_two_gloo_ranks_match_single_process():
         r = oracle_slice(inp, wl, b, h)
         assert np.array_equal(idx, r["idx"]) and np.array_equal(count, r["count"])
         assert np.array_equal(out, r["out"])
+
+
+def _bench_shard_worker(rank, world, port, q):
+    """As bench.py's GPU arm shards its global batch, on the host: rank k draws its blocks with
+    shard.shard_inputs, runs the oracle on them, and the gathered blocks must be the global
+    batch's blocks in order."""
+    import sys
+    sys.path[:0] = [ROOT, os.path.join(ROOT, "tests")]
+    import datetime
+    import torch.distributed as dist
+    import bench
+    from parity_util import oracle_slice
+    from tree_routed_sparse_b200 import shard as sh, synth
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    per_gpu = synth.WORKLOADS["prefill_b4h8_n4096"].replace(batch=1, heads=3, n=128, nq=128)
+    g = sh.global_workload(per_gpu, world)
+    lo, hi, inp = sh.shard_inputs(g, world, rank)
+    mine = {}
+    for b in range(inp["K"].shape[0]):
+        for h in range(inp["K"].shape[1]):
+            flat = lo + b * inp["K"].shape[1] + h
+            r = oracle_slice(inp, g, b, h)
+            mine[flat] = (inp["K"][b, h].numpy().copy(), r["idx"], r["out"])
+    gathered = [None] * world
+    dist.all_gather_object(gathered, mine)
+    t = bench.max_over_ranks(dist, 1.0 + 0.25 * rank)
+    if rank == 0:
+        merged = {}
+        for part in gathered:
+            merged.update(part)
+        q.put((merged, t))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_shard_a_global_batch():
+    import sys
+    sys.path[:0] = [os.path.join(ROOT, "tests")]
+    from parity_util import oracle_slice
+    from tree_routed_sparse_b200 import shard as sh, synth
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bench_shard_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    merged, t = q.get(timeout=240)
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    assert t == 1.25
+    per_gpu = synth.WORKLOADS["prefill_b4h8_n4096"].replace(batch=1, heads=3, n=128, nq=128)
+    g = sh.global_workload(per_gpu, 2)
+    full = synth.make_inputs(g, "cpu")
+    assert sorted(merged) == list(range(g.bh))
+    for flat, (K, idx, out) in merged.items():
+        b, h = divmod(flat, g.heads)
+        assert np.array_equal(K, full["K"][b, h].numpy())
+        ref = oracle_slice(full, g, b, h)
+        assert np.array_equal(idx, ref["idx"]) and np.array_equal(out, ref["out"])
