@@ -509,7 +509,7 @@ __global__ void __launch_bounds__(NWC * 32, 16 / NWC) cta_query_kernel(const Que
       __syncthreads();
       const int per = (count + NWC - 1) / NWC;
       const int k0 = min(count, warp * per);
-      gather_values_part<D, 2>(B.selk, B.selp, k0, min(count, k0 + per),
+      gather_values_part<D, 8>(B.selk, B.selp, k0, min(count, k0 + per),
                                a.V + bh * (long long)n * D, lane, C.opart[warp]);
       __syncthreads();
       const float inv = C.inv;
