@@ -191,3 +191,27 @@ def test_mid_size_route_predict_override(alhr, d, bits):
         cpu_bo = dict(cpu, W=None, budget_override=bo.cpu())
         ref_o = oracle_slice(cpu_bo, wl.replace(predictor=False), b, h)
         compare_rows(f, ref_o, b, h, np.arange(1), TOL, f"override 768 d={d} {(b, h)}")
+
+
+@pytest.mark.parametrize("d,window,max_keys", [(128, 32, 50), (64, 1, 7), (64, 32, 96)])
+def test_mid_size_edges_ties(alhr, d, window, max_keys):
+    """The two-warp CTA shape (768 decode-style queries) with the edge settings of the small
+    parity tests: window 1 or 32, a small key cap, and values in [-1, 1] so that equal scores
+    are everywhere (ties to the lower start decide the sets). Sampled blocks against the oracle."""
+    from tree_routed_sparse_b200 import synth
+    n = 1024
+    wl = synth.WORKLOADS["decode_s64h8_n262144_d128"].replace(
+        batch=96, n=n, d=d, q_start=n - 1, window=window, max_keys=max_keys, qk_lo=-1, qk_hi=1,
+        score_bits=0, seed=11)
+    inp = synth.make_inputs(wl, "cuda")
+    tree = alhr.build_tree(inp["K"], value_bound=1)
+    res = alhr.forward(inp["Q"], inp["K"], inp["V"], tree, W=inp["W"], q_start=wl.q_start,
+                       window=window, max_keys=max_keys, value_bound=1, want_idx=True,
+                       want_count=True, want_expansions=True, want_budget=True)
+    torch.cuda.synchronize()
+    cpu = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
+    rng = np.random.default_rng(6)
+    for b, h in [(0, 0), (95, 7)] + [tuple(x) for x in zip(rng.integers(0, 96, 8),
+                                                           rng.integers(0, 8, 8))]:
+        ref = oracle_slice(cpu, wl, b, h)
+        compare_rows(res, ref, b, h, np.arange(1), TOL, f"768 ties d={d} w={window} {(b, h)}")
