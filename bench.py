@@ -304,7 +304,7 @@ def oracle_steps(wl, inp, steps: int, row_stride: int, first_step: int = 0) -> d
 
 
 def oracle_single_thread(wl, inp) -> dict:
-    """BASELINE's single-threaded figure: block (b,h) = (0,0), its tree and every query row,
+    """The single-threaded oracle figure: block (b,h) = (0,0), its tree and every query row,
     timed with std::chrono::steady_clock inside the oracle library on one thread."""
     from oracle import oracle as orc
     Vbits, W = _host_blocks(inp)
