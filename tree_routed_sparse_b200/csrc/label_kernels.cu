@@ -276,10 +276,10 @@ __global__ void __launch_bounds__(kLThreads, D == 64 ? 4 : 3)
   uint32_t drain_parity = 0u;
   for (int t = 0; t < ntiles; ++t) {
     const int b = t & 1;
-    const uint32_t parity = (phases >> b) & 1u;
     // 1. MMA t done (as this thread sees it): its accumulator is ready, its key buffer free
     bool ok = false;
-    for (uint32_t w = 0; w < kWaitLimit && !ok; ++w) ok = mbar_try_wait(smem_u32(mbar + b), parity);
+    for (uint32_t w = 0; w < kWaitLimit && !ok; ++w)
+      ok = mbar_try_wait(smem_u32(mbar + b), (phases >> b) & 1u);
     phases ^= 1u << b;
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
     // 2. key tile t + 2 into the freed buffer (its own cp.async group)
@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(kLThreads, D == 64 ? 4 : 3)
         if (dev_err) atomicOr(dev_err, ALHR_DEVERR_TIMEOUT);
       }
       drain_b = b;
-      drain_parity = parity;
+      drain_parity = ((phases >> b) & 1u) ^ 1u;  // the parity waited for above
       break;
     }
     if (t + 1 < ntiles && tid == 0) issue_mma(t + 1);
