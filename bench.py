@@ -363,6 +363,7 @@ def run_alhr(args, dist, rank, world):
               score_bits=wl.score_bits, value_bound=vb)
     path_bytes = sum(t.numel() * t.element_size() for t in (Q, K, V, W, bo, tree, out)
                      if t is not None)
+    sbits = 32 if alhr.score_bits(alhr.make_dims(Q, K, **kw)) == 32 else 64
 
     # one untimed run with every output: counts for the byte model
     alhr.build_tree(K, tree, value_bound=vb)
@@ -404,38 +405,11 @@ def run_alhr(args, dist, rank, world):
     peak_alloc = torch.cuda.max_memory_allocated(dev)
     t_tree = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
     t_fwd = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    out_ref = out.cpu()  # the step's output, which the end-to-end run must reproduce
     t_step = t_tree + t_fwd
     t_job = max_over_ranks(dist, t_step)
     queries = wl.bh * wl.nq
     value = world * queries * args.steps / t_job
-
-    # end to end through the public API, host buffers: every step copies its inputs in from
-    # pinned memory, builds the tree, runs the fused forward and copies the output back, through
-    # tree_routed_sparse_b200.pipeline.HostPipeline (copies of the next and the previous step
-    # overlap this step's kernels on their own streams; L2 flushed on the compute stream before
-    # every step, inside the timed region)
-    from tree_routed_sparse_b200.pipeline import HostPipeline
-    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in inp.items()}
-    outs_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
-    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
-    d2h = outs_host[0].numel() * outs_host[0].element_size()
-    pipe = HostPipeline(host, device=dev, flush=flush, **kw)
-    for s in range(3):
-        pipe.submit(host, outs_host[s & 1])
-    pipe.synchronize()
-    assert torch.equal(outs_host[0], out.cpu()) and torch.equal(outs_host[1], out.cpu())
-    barrier(dist)
-    torch.cuda.synchronize()
-    e2e_start, e2e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_start.record(pipe.copy_in)
-    for s in range(args.e2e_steps):
-        pipe.submit(host, outs_host[s & 1])
-    e2e_end.record(pipe.copy_out)
-    pipe.synchronize()
-    barrier(dist)
-    t_e2e = max_over_ranks(dist, e2e_start.elapsed_time(e2e_end) / 1e3)
-    e2e_value = world * queries * args.e2e_steps / t_e2e
-    del pipe, host, outs_host
 
     # the pages' operating point (about 30 keys read per query): the same inputs, predictor
     # rows of classes >= OP_LIVE_CLASSES zeroed; fused forward only (the tree is unchanged)
@@ -468,6 +442,59 @@ def run_alhr(args, dist, rank, world):
               "queries_per_s": world * queries * args.op_steps / t_op,
               "launch_ms": t_op / args.op_steps * 1e3, "algorithmic_bytes_per_launch": op_bytes,
               "kernel_row_bytes_per_launch": op_kernel_bytes}
+
+    # end to end through the public API, host buffers: every step copies its inputs in from
+    # pinned memory, builds the tree, runs the fused forward and copies the output back, through
+    # tree_routed_sparse_b200.pipeline.HostPipeline (copies of the next and the previous step
+    # overlap this step's kernels on their own streams; L2 flushed on the compute stream before
+    # every step, inside the timed region). The device tensors of the runs above are freed
+    # first; a workload whose double-buffered pipeline does not fit runs single-buffered, and the
+    # number of steps is capped at about two seconds of copies.
+    from tree_routed_sparse_b200.pipeline import HostPipeline
+    import psutil
+    h2d = sum(v.numel() * v.element_size() for v in inp.values() if v is not None)
+    d2h = out_ref.numel() * out_ref.element_size()
+    e2e_skip = None
+    if h2d > (8 << 30):
+        e2e_skip = (f"a step's inputs are {h2d / 2**30:.0f} GiB: the end-to-end run (all inputs "
+                    "copied in from pinned host memory every step) is measured for workloads of "
+                    "at most 8 GiB per step")
+    elif 3 * h2d > psutil.virtual_memory().available:
+        e2e_skip = "not enough free host memory to pin a copy of the inputs"
+    if e2e_skip is None:
+        host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in inp.items()}
+    del inp, Q, K, V, W, bo, tree, out
+    torch.cuda.empty_cache()
+    nbuf, e2e_steps, e2e_value = 0, 0, None
+    if e2e_skip is None:
+        outs_host = [torch.empty(out_ref.shape, dtype=out_ref.dtype).pin_memory()
+                     for _ in range(2)]
+        free, _ = torch.cuda.mem_get_info(dev)
+        nbuf = 2 if 2 * path_bytes < 0.9 * free else 1
+        e2e_steps = max(3, min(args.e2e_steps, int(2.0 / max((h2d + d2h) / 50e9, 1e-6))))
+        pipe = HostPipeline(host, device=dev, flush=flush, buffers=nbuf, **kw)
+        for s in range(3):
+            pipe.submit(host, outs_host[s & 1])
+        pipe.synchronize()
+        assert torch.equal(outs_host[0], out_ref) and torch.equal(outs_host[1], out_ref)
+    # every rank takes the same collective steps, measured or not
+    barrier(dist)
+    torch.cuda.synchronize()
+    t_e2e = 0.0
+    if e2e_skip is None:
+        e2e_start = torch.cuda.Event(enable_timing=True)
+        e2e_end = torch.cuda.Event(enable_timing=True)
+        e2e_start.record(pipe.copy_in)
+        for s in range(e2e_steps):
+            pipe.submit(host, outs_host[s & 1])
+        e2e_end.record(pipe.copy_out)
+        pipe.synchronize()
+        t_e2e = e2e_start.elapsed_time(e2e_end) / 1e3
+        del pipe, host, outs_host
+    barrier(dist)
+    t_e2e = max_over_ranks(dist, t_e2e)
+    if e2e_skip is None:
+        e2e_value = world * queries * e2e_steps / t_e2e
 
     if rank != 0:
         return None
@@ -504,7 +531,7 @@ def run_alhr(args, dist, rank, world):
                         f"heads, each rank its contiguous {wl.bh} (b,h) blocks; no collective "
                         "on the data path"),
         "queries_per_step_per_gpu": queries,
-        "score_bits": 32 if alhr.score_bits(alhr.make_dims(Q, K, **kw)) == 32 else 64,
+        "score_bits": sbits,
         "mean_keys_per_query": mean_keys,
         "mean_budget": mean_budget,
         "roofline": {
@@ -544,11 +571,15 @@ def run_alhr(args, dist, rank, world):
                             "buffer); the library itself allocates nothing")},
         "operating_point_30_keys": op,
         "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-                "how": "HostPipeline: every step copies Q, K, V, W in from pinned host memory "
-                       "and its output back; the next step's copy-in and the previous step's "
-                       "copy-out overlap this step's kernels on their own streams; L2 flushed "
-                       "before every step's kernels inside the timed region"},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps, "skipped": e2e_skip,
+                "how": None if e2e_skip else (
+                    "HostPipeline: every step copies Q, K, V, W in from pinned host memory and "
+                    "its output back; " + (
+                        "the next step's copy-in and the previous step's copy-out overlap this "
+                        "step's kernels on their own streams" if nbuf == 2 else
+                        "single-buffered (two device copies of the step do not fit): the copies "
+                        "wait for the kernels") +
+                    "; L2 flushed before every step's kernels inside the timed region")},
         "gpu_launches": args.steps * (tree_launches + 1),
         "clocks": clocks,
         "wall_s_timed_region": wall,

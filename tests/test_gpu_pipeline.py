@@ -5,7 +5,8 @@ import torch
 pytestmark = pytest.mark.gpu
 
 
-def test_pipeline_matches_direct_calls():
+@pytest.mark.parametrize("buffers", [2, 1])
+def test_pipeline_matches_direct_calls(buffers):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from tree_routed_sparse_b200 import alhr, build, synth
@@ -16,7 +17,7 @@ def test_pipeline_matches_direct_calls():
     hosts = [{k: (None if v is None else v.pin_memory()) for k, v in b.items()} for b in batches]
     outs = [torch.empty((2, 2, 1024, 64), dtype=torch.float32).pin_memory() for _ in batches]
     kw = dict(q_start=0, window=base.window, max_keys=base.max_keys, score_bits=0, value_bound=16)
-    pipe = HostPipeline(hosts[0], **kw)
+    pipe = HostPipeline(hosts[0], buffers=buffers, **kw)
     for h, o in zip(hosts, outs):
         pipe.submit(h, o)
     pipe.synchronize()
