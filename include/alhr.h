@@ -156,10 +156,14 @@ ALHR_API const char* alhr_build_info(void);
  * Launch shape of the per-query kernels (alhr_forward, alhr_route, alhr_predict_budget), a
  * process-wide setting. Trees, budgets, index sets, counts and expansions are identical in every
  * mode; outputs may differ in the last bits of fp32 (another summation order of the value rows).
- *   ALHR_LAUNCH_AUTO (default): latency shape when a launch has at most 8 queries per SM of the
- *     device (decode and other small launches), throughput shape above.
- *   ALHR_LAUNCH_THROUGHPUT: several CTAs per SM, one or two tree rows in flight per lane group.
- *   ALHR_LAUNCH_LATENCY: one CTA per SM, up to twelve rows in flight per lane group.
+ *   ALHR_LAUNCH_AUTO (default): the latency shape when every query of the launch is resident at
+ *     once in it (four warps per query while the four-warp CTAs all fit, about 4 per SM; else
+ *     two warps per query while those fit, about 7-8 per SM): decode and other small launches;
+ *     the throughput shape above.
+ *   ALHR_LAUNCH_THROUGHPUT: one warp per query, two CTAs of 14 warps per SM, each warp looping
+ *     over the launch's queries.
+ *   ALHR_LAUNCH_LATENCY: one CTA of four warps per query, in several waves when the launch has
+ *     more queries than resident CTAs.
  * alhr_set_launch_mode returns ALHR_ERR_INVALID_ARG (and changes nothing) for any other value.
  */
 typedef enum {

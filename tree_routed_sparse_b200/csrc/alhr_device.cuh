@@ -23,7 +23,7 @@ constexpr int kMaxFrontier = 96;    // r <= max_keys - 1 nodes survive a step
 constexpr int kMaxCand = 192;       // a step offers at most 2 r candidates
 constexpr int kMaxWindow = 32;      // the largest neighbour window the kernels accept
 constexpr int kFrontSlots = kMaxFrontier / 32;
-constexpr int kWarps = 8;           // queries in flight per CTA
+constexpr int kWarps = 8;           // warps (queries) per CTA of the unfused attention kernel
 
 template <int D>
 struct Lay {
@@ -305,14 +305,10 @@ __device__ __forceinline__ void gather_values(const int* selk, const float* selp
     float p[UV];
 #pragma unroll
     for (int u = 0; u < UV; ++u) {
+      // a value group past the end loads the last selected row again with weight 0
       const int k = base + u * KPP + kg;
-      if (k < count) {
-        raw[u] = __ldg(reinterpret_cast<const uint4*>(Vh + (long long)selk[k] * D) + vs);
-        p[u] = selp[k];
-      } else {
-        raw[u] = make_uint4(0u, 0u, 0u, 0u);
-        p[u] = 0.f;
-      }
+      raw[u] = __ldg(reinterpret_cast<const uint4*>(Vh + (long long)selk[min(k, count - 1)] * D) + vs);
+      p[u] = k < count ? selp[k] : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < UV; ++u) {
@@ -433,11 +429,21 @@ template <typename S>
 struct WarpBuf {
   CandArray<S, kMaxCand> cand;       // frontier / candidates
   CandArray<S, kMaxFrontier> xnode;  // nodes expanded this step
-  int xrow[kMaxFrontier];    // byte offset of each expanded node's left child row (tree
-                             // block or key rows of the head)
-  S xleft[kMaxFrontier];     // score of that left child
-  int selk[kMaxKeys];        // the selected keys and their softmax weights
-  float selp[kMaxKeys];
+  // The descent's per-step lists and the attention's staged selection are never live at the
+  // same time (the selection is staged after the last step, and a barrier separates it from the
+  // next query's descent), so they share storage: a smaller buffer leaves more of the SM's
+  // unified shared memory / L1 to the cache.
+  union {
+    struct {
+      int xrow[kMaxFrontier];  // byte offset of each expanded node's left child row (tree
+                               // block or key rows of the head)
+      S xleft[kMaxFrontier];   // score of that left child
+    };
+    struct {
+      int selk[kMaxKeys];      // the selected keys and their softmax weights
+      float selp[kMaxKeys];
+    };
+  };
   int plist[32];             // the roots of the descent forest, largest first
   int winsc[kMaxWindow + 4]; // scores of the window keys (+ a spare slot for idle row groups;
                              // padded so that the buffer stays a multiple of 16 bytes)

@@ -94,16 +94,14 @@ __device__ __forceinline__ void cta_child_pass(WarpBuf<S>& B, const char* Th, co
   int x[US][WORDS];
 #pragma unroll
   for (int u = 0; u < US; ++u) {
+    // a row group past the end loads the pass's last row again (in bounds; its score is not
+    // stored), so that no lane spends instructions clearing registers
     const int xi = base + u * NG + gg;
-    if (xi < end) {
-      if constexpr (KIND == 0) ld_tree<D>(Th + B.xrow[xi], sub, x[u]);
-      else if constexpr (KIND == 1) ld_tree16<D>(Th + B.xrow[xi], sub, x[u]);
-      else ld_key<D>(Kh + B.xrow[xi], sub, x[u]);
-      prefetch_grandchildren<D>(Th, Kh, n, narrow, bucket, B.xnode.desc(xi), sub);
-    } else {
-#pragma unroll
-      for (int j = 0; j < WORDS; ++j) x[u][j] = 0;
-    }
+    const int xr = B.xrow[min(xi, end - 1)];
+    if constexpr (KIND == 0) ld_tree<D>(Th + xr, sub, x[u]);
+    else if constexpr (KIND == 1) ld_tree16<D>(Th + xr, sub, x[u]);
+    else ld_key<D>(Kh + xr, sub, x[u]);
+    if (xi < end) prefetch_grandchildren<D>(Th, Kh, n, narrow, bucket, B.xnode.desc(xi), sub);
   }
   __syncwarp();
 #pragma unroll
@@ -135,14 +133,10 @@ __device__ __forceinline__ void gather_values_part(const int* selk, const float*
     float p[UV];
 #pragma unroll
     for (int u = 0; u < UV; ++u) {
+      // a value group past the end loads the last row of the range again with weight 0
       const int k = base + u * KPP + kg;
-      if (k < k1) {
-        raw[u] = __ldg(reinterpret_cast<const uint4*>(Vh + (long long)selk[k] * D) + vs);
-        p[u] = selp[k];
-      } else {
-        raw[u] = make_uint4(0u, 0u, 0u, 0u);
-        p[u] = 0.f;
-      }
+      raw[u] = __ldg(reinterpret_cast<const uint4*>(Vh + (long long)selk[min(k, k1 - 1)] * D) + vs);
+      p[u] = k < k1 ? selp[k] : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < UV; ++u) {

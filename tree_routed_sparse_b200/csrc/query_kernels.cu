@@ -32,10 +32,15 @@ namespace alhr {
 // blocks, a block that is also a root of the descent forest.
 constexpr int kFlagRoot = 1 << 29;
 
-// Register budget: int32 scores keep three CTAs (24 warps) per SM with two tree rows in flight
-// per row group; int64 scores need more registers, so two CTAs (and one int32 row in flight).
-template <typename S>
-constexpr int min_blocks_per_sm() { return sizeof(S) == 4 ? 3 : 2; }
+// Shape of the throughput launch: CTAs of 14 warps (one query each), two per SM, i.e. 28
+// queries in flight per SM at 72 registers per thread, for both score widths. Measured against
+// 8-warp CTAs (three per SM at 80 registers with int32 scores, two at 126 with int64): the extra
+// warps hide more of each query's dependent latency (L2 round trips of the child rows, the
+// selection's reductions), and two large CTAs hold fewer per-CTA copies of the predictor weights
+// in shared memory than seven 4-warp CTAs would, which leaves more of the SM's unified shared
+// memory / L1 to the cache.
+constexpr int kQueryWarps = 14;
+constexpr int kQueryBlocksPerSm = 2;
 // At d = 128 this is the number of int16 rows (two 16-byte loads each) in flight; int32 rows at
 // d = 128 go one per pass.
 template <typename S, int D>
@@ -53,13 +58,10 @@ __device__ __forceinline__ void tree_child_pass(WarpBuf<S>& B, const char* Th, c
   int x[US][16];
 #pragma unroll
   for (int u = 0; u < US; ++u) {
+    // a row group past the end loads the pass's last row again (in bounds; its score is not
+    // stored), so that no lane spends instructions clearing registers
     const int xi = base + u * RPI + grp;
-    if (xi < end) {
-      ld_tree<D>(Th + B.xrow[xi], sub, x[u]);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 16; ++j) x[u][j] = 0;
-    }
+    ld_tree<D>(Th + B.xrow[min(xi, end - 1)], sub, x[u]);
   }
   if constexpr (US > 2) __syncwarp();  // latency shape: reconverge before the group sums
 #pragma unroll
@@ -80,13 +82,8 @@ __device__ __forceinline__ void narrow_child_pass(WarpBuf<S>& B, const char* Th,
   int w[US][8];
 #pragma unroll
   for (int u = 0; u < US; ++u) {
-    const int xi = base + u * RPI + grp;
-    if (xi < end) {
-      ld_tree16<D>(Th + B.xrow[xi], sub, w[u]);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) w[u][j] = 0;
-    }
+    const int xi = base + u * RPI + grp;  // past the end: the last row again, not stored
+    ld_tree16<D>(Th + B.xrow[min(xi, end - 1)], sub, w[u]);
   }
   __syncwarp();  // reconverge before the group sums
 #pragma unroll
@@ -99,15 +96,15 @@ __device__ __forceinline__ void narrow_child_pass(WarpBuf<S>& B, const char* Th,
   }
 }
 
-// The warp-per-query kernel (the throughput shape: several CTAs of eight warps per SM, for
+// The warp-per-query kernel (the throughput shape: two CTAs of 14 warps per SM, for
 // launches that fill the GPU; smaller launches take the CTA-per-query kernel of
 // cta_query_kernels.cu). VAR compiles in the descent variants (ranking by means, leaf buckets;
 // chosen at run time from the arguments); without it the method's descent carries none of their
 // code.
 template <typename S, int D, int MODE, bool VAR>
-__global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>())
+__global__ void __launch_bounds__(kQueryWarps * 32, kQueryBlocksPerSm)
     query_kernel(const QueryArgs a) {
-  constexpr int NW = kWarps;
+  constexpr int NW = kQueryWarps;
   constexpr int TPR = Lay<D>::TPR;
   constexpr int RPI = Lay<D>::RPI;
   // tree rows per group per pass (at d = 128: int16 rows; int32 rows go one per pass)
@@ -458,8 +455,8 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>())
         // left children that are keys: one per group per pass
         for (int base = nhi; base < nx; base += RPI) {
           const int xi = base + grp;
-          int xp[4] = {0, 0, 0, 0};
-          if (xi < nx) ld_key<D>(Kh + B.xrow[xi], sub, xp);
+          int xp[4];
+          ld_key<D>(Kh + B.xrow[min(xi, nx - 1)], sub, xp);  // past the end: not stored
           const int left = group_sum<int, TPR>(dot_key(q, xp));
           if (xi < nx && sub == 0) B.xleft[xi] = S(left);
         }
@@ -484,8 +481,8 @@ __global__ void __launch_bounds__(kWarps * 32, min_blocks_per_sm<S>())
     if constexpr (kAttend && !(kUsesW && !kGBlocks)) {
       for (int base = 0; base < nsel_win; base += RPI) {
         const int x = base + grp;
-        int xp[4] = {0, 0, 0, 0};
-        if (x < nsel_win) ld_key<D>(Kh + (long long)(i - x) * D, sub, xp);
+        int xp[4];
+        ld_key<D>(Kh + (long long)(i - min(x, nsel_win - 1)) * D, sub, xp);  // past: not stored
         const int s = group_sum<int, TPR>(dot_key(q, xp));
         if (x < nsel_win && sub == 0) B.winsc[x] = s;
       }
@@ -670,7 +667,7 @@ cudaError_t launch_query_mode(const QueryArgs& a, cudaStream_t st) {
   constexpr int slot = ((MODE * 2 + (D == 128 ? 1 : 0)) * 2 + (sizeof(S) == 8 ? 1 : 0)) * 2 +
                        (VAR ? 1 : 0);
   static_assert(slot < 64, "occupancy cache slot");
-  constexpr int nw = kWarps;
+  constexpr int nw = kQueryWarps;
   constexpr size_t smem = QuerySmem<S, D, MODE>::bytes_for(nw);
   auto kern = query_kernel<S, D, MODE, VAR>;
   cudaError_t err;
