@@ -160,8 +160,8 @@ ALHR_API const char* alhr_build_info(void);
  *     once in it (four warps per query while the four-warp CTAs all fit, about 4 per SM; else
  *     two warps per query while those fit, about 7-8 per SM): decode and other small launches;
  *     the throughput shape above.
- *   ALHR_LAUNCH_THROUGHPUT: one warp per query, two CTAs of 14 warps per SM, each warp looping
- *     over the launch's queries.
+ *   ALHR_LAUNCH_THROUGHPUT: one warp per query, two CTAs of 14 warps per SM, each warp taking
+ *     the next query of its CTA's share from a counter in shared memory.
  *   ALHR_LAUNCH_LATENCY: one CTA of four warps per query, in several waves when the launch has
  *     more queries than resident CTAs.
  * alhr_set_launch_mode returns ALHR_ERR_INVALID_ARG (and changes nothing) for any other value.
