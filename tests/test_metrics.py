@@ -61,7 +61,8 @@ def test_g_from_blocks_counts_the_blocks_of_the_prefix():
     g_rows = 4 * d + 4 * d + d          # [0,16), [16,20), [20,21)
     roots_rest = 4 * d + d              # [16,18), [18,19)
     assert got == d + g_rows + roots_rest + 2 * d + 3 * 2 * d + 4 * d + 64 * d
-    # the survey's count of the same query: the roots of [0,19) and both window keys
+    # the algorithmic count of the same query (G_i from the roots and the window keys, which the
+    # query reads anyway): the roots of [0,19) and both window keys
     plain = metrics.forward_bytes([20], 32, d, 2, [3], [[0, 0, 0]], [3], predictor=True)
     assert plain == d + (4 * d + 4 * d + d) + 2 * d + 3 * 2 * d + 4 * d + 64 * d
 
